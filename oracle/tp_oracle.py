@@ -1,0 +1,391 @@
+"""CPU oracle for the Megatron-LM tensor-parallel Transformer layer (fp64).
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or run
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it. It shares
+no code with the CUDA library and imports nothing from it; it receives plain
+numpy arrays (bf16 inputs widened exactly to float64) and computes in float64
+with no intermediate rounding.
+
+Sources (web pages on Megatron-LM tensor parallelism), cited by title and
+section:
+  [TP-LLM]  "Tensor Parallelism in Large Language Models: How Megatron-LM
+            Partitions Multi-Layer Perceptrons and Attention Heads"
+            (llms.blog), sections "The Core Primitives", "Partitioning the
+            Multi-Layer Perceptron (MLP) Block", "Partitioning Multi-Head and
+            Grouped-Query Attention", "Sequence Parallelism".
+  [M-LM]    "Megatron-LM" (ai360xpert.com), section "How It Works".
+  [INTRO]   "Introduction to Megatron-LM" (apxml.com course chapter),
+            "Core Contributions" and its ColumnParallelLinear example.
+  [FANOUT]  "Megatron-LM: Training Multi-Billion Parameter Language Models
+            Using Model Parallelism" (fanout.sh), "What you will learn".
+
+Readings where the pages are silent (each is listed with its reason in the
+design notes of the repository):
+  * GeLU is the erf form 0.5 x (1 + erf(x / sqrt 2)).
+  * The column-parallel bias is sliced with the columns and added before the
+    activation; the row-parallel bias is added once, after the sum.
+  * The residual is added once, after the sum.
+  * Causal attention: query t of a sequence sees keys 0..t of the same
+    sequence; attention never crosses sequences.
+  * LayerNorm uses the population variance and eps = 1e-5 unless given.
+  * The layer is pre-LN: h1 = X + Attn(LN1(X)); Y = h1 + MLP(LN2(h1)).
+  * Dropout is the identity (forward pass).
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against
+closed forms, brute-force scalar loops, textbook values and the identities
+the pages state.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+SPLIT_COLUMN = 0
+SPLIT_ROW = 1
+SPLIT_QKV_HEADS = 2
+
+
+# --------------------------------------------------------------------------
+# elementwise pieces
+# --------------------------------------------------------------------------
+
+def gelu(x: np.ndarray) -> np.ndarray:
+    """GeLU(x) = x * Phi(x), Phi the standard normal CDF, in its erf form.
+
+    The pages name "GeLU" only ([M-LM] "How It Works", [TP-LLM] MLP block);
+    the erf form is the plainest reading.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + _erf(x / math.sqrt(2.0)))
+
+
+def layernorm(x: np.ndarray, gamma: np.ndarray, beta: np.ndarray,
+              eps: float = 1e-5) -> np.ndarray:
+    """Per-token LayerNorm over the hidden dimension, population variance.
+
+    [TP-LLM] "Sequence Parallelism": LayerNorm is replicated on every
+    tensor-parallel rank and acts along h independently for every token.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * gamma + beta
+
+
+def softmax_rows(s: np.ndarray) -> np.ndarray:
+    """Row softmax, max-subtracted; -inf entries get probability exactly 0."""
+    m = np.max(s, axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+# --------------------------------------------------------------------------
+# the shard index maps ([TP-LLM] "The Core Primitives"; attention section)
+# --------------------------------------------------------------------------
+
+def _check_div(what: str, value: int, n: int) -> None:
+    if n <= 0 or value % n != 0:
+        raise ValueError(f"{what}={value} is not divisible by N={n}")
+
+
+def shard_index_map(kind: int, h_in: int, h_out: int, n_shards: int,
+                    head_dim: int = 0):
+    """Which shard owns each split index, and its position inside the shard.
+
+    * column split: W = [W_1 ... W_N] along H_out, each W_i of width
+      H_out / N ([TP-LLM] "Column-Parallel Linear Layer"); index = column.
+    * row split: W = [W_1; ...; W_N] along H_in, each of height H_in / N
+      ([TP-LLM] "Row-Parallel Linear Layer"); index = row.
+    * QKV head split: W_QKV = [W_Q | W_K | W_V] (each h x h, h = h_out / 3);
+      shard i owns heads [i n_h/N, (i+1) n_h/N) of each projection, head k
+      being columns [k d, (k+1) d) ([TP-LLM] "Partitioning Multi-Head ...
+      Attention", Q, K, V projections). Inside a shard the local columns are
+      ordered [Q_i | K_i | V_i]. index = column of W_QKV.
+
+    Returns (owner, local) int64 arrays over the split index.
+    """
+    if kind == SPLIT_COLUMN:
+        _check_div("h_out", h_out, n_shards)
+        w = h_out // n_shards
+        j = np.arange(h_out, dtype=np.int64)
+        return j // w, j % w
+    if kind == SPLIT_ROW:
+        _check_div("h_in", h_in, n_shards)
+        w = h_in // n_shards
+        r = np.arange(h_in, dtype=np.int64)
+        return r // w, r % w
+    if kind == SPLIT_QKV_HEADS:
+        if h_out % 3 != 0:
+            raise ValueError("QKV weight must have 3h columns")
+        h = h_out // 3
+        if head_dim <= 0 or h % head_dim != 0:
+            raise ValueError("h must be a multiple of head_dim")
+        n_heads = h // head_dim
+        _check_div("n_heads", n_heads, n_shards)
+        hs = h // n_shards                 # columns of one projection per shard
+        j = np.arange(h_out, dtype=np.int64)
+        part, within_part = j // h, j % h  # part 0 = Q, 1 = K, 2 = V
+        head = within_part // head_dim
+        owner = head // (n_heads // n_shards)
+        local = part * hs + (within_part - owner * hs)
+        return owner, local
+    raise ValueError(f"unknown split kind {kind}")
+
+
+def shard_matrices(W: np.ndarray, kind: int, n_shards: int,
+                   head_dim: int = 0) -> list:
+    """The N logical shards W_i (H_in x H_out/N, or H_in/N x H_out, or the
+    head-sliced [Q_i | K_i | V_i] of width 3h/N), built from the index map."""
+    h_in, h_out = W.shape
+    owner, local = shard_index_map(kind, h_in, h_out, n_shards, head_dim)
+    shards = []
+    for i in range(n_shards):
+        sel = np.nonzero(owner == i)[0]
+        order = sel[np.argsort(local[sel], kind="stable")]
+        shards.append(W[order, :] if kind == SPLIT_ROW else W[:, order])
+    return shards
+
+
+def packed_shards(W: np.ndarray, kind: int, n_shards: int,
+                  head_dim: int = 0) -> np.ndarray:
+    """Byte layout the GPU consumes: shard i stored transposed (K-major),
+    i.e. out[i] = W_i^T, shape [N, cols_per_shard, rows_per_shard]."""
+    return np.stack([np.ascontiguousarray(s.T)
+                     for s in shard_matrices(W, kind, n_shards, head_dim)])
+
+
+def shard_vector(b: np.ndarray, kind: int, n_shards: int,
+                 head_dim: int = 0) -> np.ndarray:
+    """A column bias sliced like the columns it belongs to: [N, H_out/N]."""
+    return packed_shards(np.asarray(b).reshape(1, -1), kind, n_shards,
+                         head_dim)[:, :, 0]
+
+
+# --------------------------------------------------------------------------
+# the parallel linear primitives ([TP-LLM] "The Core Primitives")
+# --------------------------------------------------------------------------
+
+def linear(X: np.ndarray, W: np.ndarray, b=None) -> np.ndarray:
+    """Y = X W (+ b), X in R^{B x H_in}, W in R^{H_in x H_out}."""
+    Y = np.asarray(X, dtype=np.float64) @ np.asarray(W, dtype=np.float64)
+    if b is not None:
+        Y = Y + b
+    return Y
+
+
+def column_parallel_linear(X, W, b, n_shards: int, act=None,
+                           kind: int = SPLIT_COLUMN, head_dim: int = 0) -> list:
+    """Y_i = act(X W_i + b_i) on every shard; X is replicated, no exchange.
+
+    [TP-LLM] "Column-Parallel Linear Layer" (Y_i = X W_i) and its note that an
+    element-wise function can be applied to the local slice; [M-LM] step 1
+    (GeLU(X A_i) per GPU).
+    """
+    Ws = shard_matrices(W, kind, n_shards, head_dim)
+    bs = (shard_matrices(np.asarray(b).reshape(1, -1), kind, n_shards,
+                         head_dim) if b is not None else [None] * n_shards)
+    out = []
+    for Wi, bi in zip(Ws, bs):
+        Yi = linear(X, Wi, None if bi is None else bi[0])
+        out.append(act(Yi) if act is not None else Yi)
+    return out
+
+
+def row_parallel_linear(X_shards: list, W: np.ndarray, n_shards: int) -> list:
+    """Partial products Y_i = X_i W_i, each full size B x H_out.
+
+    [TP-LLM] "Row-Parallel Linear Layer" (Y_i = X_i W_i); [M-LM] step 2.
+    """
+    Ws = shard_matrices(W, SPLIT_ROW, n_shards)
+    return [linear(Xi, Wi) for Xi, Wi in zip(X_shards, Ws)]
+
+
+def reduce_partials(partials: list, bias=None, residual=None) -> np.ndarray:
+    """Y = sum_i Y_i (+ b) (+ R): the all-reduce sum of the row-parallel
+    partials ([TP-LLM] "Row-Parallel Linear Layer", Y = sum_i Y_i = XW;
+    [M-LM] step 3), with the output bias and the residual added once."""
+    Y = np.zeros_like(partials[0])
+    for P in partials:
+        Y = Y + P
+    if bias is not None:
+        Y = Y + bias
+    if residual is not None:
+        Y = Y + residual
+    return Y
+
+
+def split_columns(X: np.ndarray, n_shards: int) -> list:
+    """X = [X_1 ... X_N] along its channel dimension ([TP-LLM] row-parallel
+    input)."""
+    _check_div("channels", X.shape[1], n_shards)
+    w = X.shape[1] // n_shards
+    return [X[:, i * w:(i + 1) * w] for i in range(n_shards)]
+
+
+# --------------------------------------------------------------------------
+# blocks, unsharded (the definition) and sharded (the method)
+# --------------------------------------------------------------------------
+
+def mlp(X, A, b1, B, b2=None, residual=None) -> np.ndarray:
+    """MLP(X) = GeLU(X A + b1) B + b2 (+ R), unsharded.
+
+    [M-LM] "How It Works" (Y = GeLU(X A) B); [TP-LLM] MLP block
+    (sigma(X W_in) W_out, W_in h x 4h, W_out 4h x h).
+    """
+    return reduce_partials([linear(gelu(linear(X, A, b1)), B)], b2, residual)
+
+
+def mlp_sharded(X, A, b1, B, b2, residual, n_shards: int) -> np.ndarray:
+    """The tensor-parallel route: column-parallel A with per-shard bias+GeLU,
+    row-parallel B, one sum of the N partials ([TP-LLM] "Partitioning the
+    Multi-Layer Perceptron (MLP) Block" steps 1-4)."""
+    A_i = column_parallel_linear(X, A, b1, n_shards, act=gelu)
+    P_i = row_parallel_linear(A_i, B, n_shards)
+    return reduce_partials(P_i, b2, residual)
+
+
+def attention_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray,
+                   causal: bool) -> np.ndarray:
+    """softmax(Q K^T / sqrt(d_k)) V for one head of one sequence
+    ([TP-LLM] "Local Self-Attention Computation"); with ``causal`` query t
+    sees keys 0..t only."""
+    d = Q.shape[1]
+    S = (Q @ K.T) / math.sqrt(d)
+    if causal:
+        t = np.arange(Q.shape[0])[:, None]
+        s = np.arange(K.shape[0])[None, :]
+        S = np.where(s <= t, S, -np.inf)
+    return softmax_rows(S) @ V
+
+
+def attention_heads(Q, K, V, batch: int, seq: int, n_heads: int,
+                    causal: bool) -> np.ndarray:
+    """Every (sequence, head) pair independently; head k is columns
+    [k d, (k+1) d); the head outputs are concatenated in head order."""
+    M, h = Q.shape
+    d = h // n_heads
+    O = np.zeros((M, h))
+    for s in range(batch):
+        r = slice(s * seq, (s + 1) * seq)
+        for k in range(n_heads):
+            c = slice(k * d, (k + 1) * d)
+            O[r, c] = attention_head(Q[r, c], K[r, c], V[r, c], causal)
+    return O
+
+
+def self_attention(X, Wqkv, bqkv, Wo, bo, residual, batch: int, seq: int,
+                   n_heads: int, causal: bool = True) -> np.ndarray:
+    """Multi-head self-attention block, unsharded:
+    [Q|K|V] = X [W_Q|W_K|W_V] + b_QKV; O = concat_k head_k; Y = O W_O + b_O
+    (+ R). [TP-LLM] "Partitioning Multi-Head and Grouped-Query Attention"
+    (d_k = h / h_heads)."""
+    h = X.shape[1]
+    QKV = linear(X, Wqkv, bqkv)
+    O = attention_heads(QKV[:, :h], QKV[:, h:2 * h], QKV[:, 2 * h:],
+                        batch, seq, n_heads, causal)
+    return reduce_partials([linear(O, Wo)], bo, residual)
+
+
+def self_attention_sharded(X, Wqkv, bqkv, Wo, bo, residual, batch: int,
+                           seq: int, n_heads: int, n_shards: int,
+                           causal: bool = True) -> np.ndarray:
+    """The tensor-parallel route: QKV column-parallel by whole heads, local
+    attention for the shard's heads, heads concatenated locally, W_O
+    row-parallel, one sum of the partials ([TP-LLM] attention steps 1-4)."""
+    h = X.shape[1]
+    d = h // n_heads
+    hs = h // n_shards
+    QKV_i = column_parallel_linear(X, Wqkv, bqkv, n_shards,
+                                   kind=SPLIT_QKV_HEADS, head_dim=d)
+    O_i = [attention_heads(q[:, :hs], q[:, hs:2 * hs], q[:, 2 * hs:],
+                           batch, seq, n_heads // n_shards, causal)
+           for q in QKV_i]
+    P_i = row_parallel_linear(O_i, Wo, n_shards)
+    return reduce_partials(P_i, bo, residual)
+
+
+def transformer_layer(X, p: dict, batch: int, seq: int, n_heads: int,
+                      eps: float = 1e-5, causal: bool = True) -> np.ndarray:
+    """Pre-LN layer: h1 = X + Attn(LN1(X)); Y = h1 + MLP(LN2(h1)).
+
+    LayerNorm, dropout (identity here) and the residual adds are replicated
+    around the two tensor-parallel blocks ([TP-LLM] "Sequence Parallelism",
+    standard formulation).
+    """
+    x1 = layernorm(X, p["ln1_g"], p["ln1_b"], eps)
+    h1 = self_attention(x1, p["Wqkv"], p["bqkv"], p["Wo"], p["bo"], X,
+                        batch, seq, n_heads, causal)
+    x2 = layernorm(h1, p["ln2_g"], p["ln2_b"], eps)
+    return mlp(x2, p["A"], p["b1"], p["B"], p["b2"], h1)
+
+
+# --------------------------------------------------------------------------
+# the same definitions restricted to a subset of output token rows
+# (used to check full-size workloads on sampled rows)
+# --------------------------------------------------------------------------
+
+def mlp_rows(X, A, b1, B, b2, residual, rows) -> np.ndarray:
+    """Rows ``rows`` of mlp(): every output row depends on its input row only."""
+    R = None if residual is None else residual[rows]
+    return mlp(X[rows], A, b1, B, b2, R)
+
+
+def self_attention_rows(X, Wqkv, bqkv, Wo, bo, residual, batch: int,
+                        seq: int, n_heads: int, rows,
+                        causal: bool = True) -> np.ndarray:
+    """Rows ``rows`` of self_attention(). Query row r (sequence r // seq,
+    position r % seq) attends to the keys of its own sequence (only up to
+    its position when causal), so K and V are projected for the whole
+    sequences the sampled rows belong to, Q for the sampled rows only."""
+    rows = np.asarray(rows, dtype=np.int64)
+    h = X.shape[1]
+    d = h // n_heads
+    Wq, Wk, Wv = Wqkv[:, :h], Wqkv[:, h:2 * h], Wqkv[:, 2 * h:]
+    bq, bk, bv = bqkv[:h], bqkv[h:2 * h], bqkv[2 * h:]
+    O = np.zeros((len(rows), h))
+    for s in np.unique(rows // seq):
+        sel = np.nonzero(rows // seq == s)[0]
+        Xs = X[s * seq:(s + 1) * seq]
+        K = linear(Xs, Wk, bk)
+        V = linear(Xs, Wv, bv)
+        Q = linear(X[rows[sel]], Wq, bq)
+        pos = rows[sel] - s * seq
+        for k in range(n_heads):
+            c = slice(k * d, (k + 1) * d)
+            S = (Q[:, c] @ K[:, c].T) / math.sqrt(d)
+            if causal:
+                S = np.where(np.arange(seq)[None, :] <= pos[:, None], S,
+                             -np.inf)
+            O[sel, c] = softmax_rows(S) @ V[:, c]
+    R = None if residual is None else residual[rows]
+    return reduce_partials([linear(O, Wo)], bo, R)
+
+
+def transformer_layer_rows(X, p: dict, batch: int, seq: int, n_heads: int,
+                           rows, eps: float = 1e-5,
+                           causal: bool = True) -> np.ndarray:
+    """Rows ``rows`` of transformer_layer()."""
+    rows = np.asarray(rows, dtype=np.int64)
+    x1 = layernorm(X, p["ln1_g"], p["ln1_b"], eps)
+    h1 = self_attention_rows(x1, p["Wqkv"], p["bqkv"], p["Wo"], p["bo"], X,
+                             batch, seq, n_heads, rows, causal)
+    x2 = layernorm(h1, p["ln2_g"], p["ln2_b"], eps)
+    return mlp(x2, p["A"], p["b1"], p["B"], p["b2"], h1)
+
+
+# --------------------------------------------------------------------------
+# algorithmic work, for throughput figures
+# --------------------------------------------------------------------------
+
+def gemm_flops(m: int, n: int, k: int) -> int:
+    return 2 * m * n * k
+
+
+def attention_flops(batch: int, seq: int, n_heads: int, d: int,
+                    causal: bool) -> float:
+    """QK^T and PV: 4 S^2 d per (sequence, head); half of it when causal."""
+    f = 4.0 * seq * seq * d * n_heads * batch
+    return f / 2 if causal else f
