@@ -1,0 +1,451 @@
+"""Benchmark of the tensor-parallel Transformer layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--shards N] [--no-cpu-baseline]
+
+A step is one forward pass of the whole hot path over one batch: the
+pre-LN layer (LN1 -> QKV column-parallel -> local attention -> W_O
+row-parallel -> partial sum + residual + LN2 -> MLP column-parallel +
+GeLU -> row-parallel -> partial sum + residual) on 2 x 2048 tokens, h 4096,
+32 heads x 128, FFN 16384, N = 8 shards, through tp_layer_forward. Inputs
+are seeded synthetic bf16 (see tensor_transformer_layer_linear_b200/synth.py)
+and already resident in HBM when timing starts; the per-step working set
+(weights 402 MB, partials 537 MB) is far larger than the 126 MB L2, so no
+flush is needed between steps.
+
+Printed (rank 0, one JSON line): whole-job TFLOP/s of algorithmic work,
+the dominant kernel's roofline (from CUDA events around every launch in
+the timed region), the partial-sum reduction's HBM bandwidth, an end-to-end
+figure through the C ABI with host buffers, the fp64 oracle timed on the
+host cores on a bounded sample, SM clocks sampled during the timed region,
+and the number of library kernel launches.
+
+With --gpus N > 1 (launched under torch.distributed.run) every rank runs the
+same single-GPU step on its own batch (independent replicas, no data-path
+collective; weak scaling); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from tensor_transformer_layer_linear_b200 import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "layer_2x2048_h4096_32x128_f16384_n8"
+METRIC = "TP-layer fwd TFLOP/s & % BF16 peak (1 B200); partial-reduce GB/s & % HBM"
+L2_BYTES = 126 * 1024 * 1024
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+# committed ncu captures under profiles/, keyed by (workload, kernel). None
+# until a capture of the current kernel exists.
+NCU_TRAFFIC = {}
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# --------------------------------------------------------------------------
+# algorithmic work per step (what the method must compute, not what runs)
+# --------------------------------------------------------------------------
+
+def work(cfg: dict) -> dict:
+    """Per-step algorithmic FLOPs per kernel kind and bytes per reduction kind."""
+    M = cfg["batch"] * cfg["seq"]
+    h = cfg["h"]
+    n = cfg["n_shards"]
+    kind = cfg["kind"]
+    fl = {"gemm_column_parallel": 0.0, "gemm_row_parallel": 0.0, "attention": 0.0}
+    by = {}
+    if kind in ("attn", "layer"):
+        fl["gemm_column_parallel"] += 2.0 * M * h * 3 * h
+        d = h // cfg["n_heads"]
+        fl["attention"] += 4.0 * cfg["seq"] ** 2 * d * cfg["n_heads"] * cfg["batch"] / (
+            2 if cfg.get("causal", True) else 1)
+        fl["gemm_row_parallel"] += 2.0 * M * h * h
+    if kind in ("mlp", "layer"):
+        F = cfg["ffn"]
+        fl["gemm_column_parallel"] += 2.0 * M * h * F
+        fl["gemm_row_parallel"] += 2.0 * M * F * h
+    partial_read = n * M * h * 4
+    act = M * h * 2
+    if kind == "layer":
+        by["reduce_partials"] = partial_read + act + h * 2 + act          # + residual, bias, write
+        by["reduce_partials_layernorm"] = partial_read + act + 3 * h * 2 + 2 * act
+        by["layernorm"] = act + 2 * h * 2 + act
+    else:
+        res = act if cfg.get("residual") else 0
+        by["reduce_partials"] = partial_read + res + h * 2 + act
+    return dict(flops=fl, bytes=by, total_flops=sum(fl.values()))
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.out = []
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            gid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gid, f"--query-gpu={CLOCK_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            text, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            text, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in text.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# the CPU oracle as a baseline (test infrastructure; timed, never on the path)
+# --------------------------------------------------------------------------
+
+def oracle_sample(cfg: dict, inp: dict, tokens: int):
+    """Run the fp64 oracle on the first `tokens` tokens of sequence 0 (a causal
+    prefix: its outputs are exactly those rows of the full workload).
+    Returns (seconds, algorithmic flops of the sample, threads used)."""
+    from threadpoolctl import threadpool_info
+    from oracle import tp_oracle as O
+    sub = dict(cfg, batch=1, seq=tokens)
+    T = tokens
+    f64 = synth.bf16_bits_to_f64
+    x = f64(inp["X"][:T])
+    t0 = time.perf_counter()
+    if cfg["kind"] == "layer":
+        p = {k: f64(v) for k, v in inp.items() if k != "X"}
+        O.transformer_layer(x, p, 1, T, cfg["n_heads"], cfg.get("ln_eps", 1e-5))
+    elif cfg["kind"] == "attn":
+        R = x if cfg.get("residual") else None
+        O.self_attention(x, f64(inp["Wqkv"]), f64(inp["bqkv"]), f64(inp["Wo"]), f64(inp["bo"]),
+                         R, 1, T, cfg["n_heads"], cfg.get("causal", True))
+    else:
+        R = x if cfg.get("residual") else None
+        O.mlp(x, f64(inp["A"]), f64(inp["b1"]), f64(inp["B"]), f64(inp["b2"]), R)
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return dt, work(sub)["total_flops"], threads
+
+
+def sample_tokens(cfg: dict) -> int:
+    return min(cfg["seq"], 512)
+
+
+def run_reference(args, cfg) -> None:
+    """The reference arm: the fp64 CPU oracle, timed on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = synth.make_inputs(cfg)
+    T = sample_tokens(cfg)
+    times, flops, threads = [], 0.0, 1
+    for i in range(args.warmup + args.steps):
+        dt, flops, threads = oracle_sample(cfg, inp, T)
+        if i >= args.warmup:
+            times.append(dt)
+    mean = sum(times) / len(times)
+    value = flops / mean / 1e12
+    sample = (f"first {T} tokens of sequence 0 (causal prefix) of {cfg['name']}, fp64 numpy "
+              f"oracle, {flops / 1e9:.1f} GFLOP algorithmic per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg["name"], "n_shards": cfg["n_shards"], "sample_tokens": T},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+class Model:
+    """Device-resident sharded weights + workspace for one workload."""
+
+    def __init__(self, tp, torch, cfg: dict, inp: dict):
+        self.tp, self.torch, self.cfg = tp, torch, cfg
+        to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).cuda()
+        dev = {k: to_dev(v) for k, v in inp.items()}
+        n, h = cfg["n_shards"], cfg["h"]
+        self.M = cfg["batch"] * cfg["seq"]
+
+        def shard(name, h_in, h_out, kind, hd=0):
+            out = torch.empty(h_in * h_out, dtype=torch.int16, device="cuda")
+            tp.tp_shard_weights(dev[name], h_in, h_out, n, kind, hd, out)
+            return out
+
+        self.X = dev["X"]
+        kind = cfg["kind"]
+        if kind in ("attn", "layer"):
+            d = h // cfg["n_heads"]
+            self.Wqkv = shard("Wqkv", h, 3 * h, 2, d)
+            self.bqkv = shard("bqkv", 1, 3 * h, 2, d)
+            self.Wo = shard("Wo", h, h, 1)
+            self.bo = dev["bo"]
+        if kind in ("mlp", "layer"):
+            F = cfg["ffn"]
+            self.A = shard("A", h, F, 0)
+            self.B = shard("B", F, h, 1)
+            self.b1, self.b2 = dev["b1"], dev["b2"]
+        if kind == "layer":
+            self.w = tp.make_layer_weights(
+                ln1_gamma=dev["ln1_g"], ln1_beta=dev["ln1_b"], Wqkv_shards=self.Wqkv,
+                bqkv_shards=self.bqkv, Wo_shards=self.Wo, bo=self.bo, ln2_gamma=dev["ln2_g"],
+                ln2_beta=dev["ln2_b"], A_shards=self.A, b1_shards=self.b1, B_shards=self.B,
+                b2=self.b2)
+            self.dev_keep = dev
+        wsk = {"mlp": tp.TP_WS_MLP, "attn": tp.TP_WS_ATTN, "layer": tp.TP_WS_LAYER}[kind]
+        self.ws_bytes = tp.tp_workspace_bytes(wsk, self.M, h, cfg.get("ffn", 0), n)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        self.Y = torch.empty((self.M, h), dtype=torch.int16, device="cuda")
+        torch.cuda.synchronize()
+
+    def step(self, X=None, Y=None):
+        tp, cfg = self.tp, self.cfg
+        X = self.X if X is None else X
+        Y = self.Y if Y is None else Y
+        n, h = cfg["n_shards"], cfg["h"]
+        if cfg["kind"] == "layer":
+            tp.tp_layer_forward(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"], cfg["ffn"], n,
+                                self.w, cfg.get("ln_eps", 1e-5), self.ws, self.ws_bytes, Y)
+        elif cfg["kind"] == "attn":
+            tp.tp_attn_forward(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"],
+                               cfg.get("causal", True), n, self.Wqkv, self.bqkv, self.Wo,
+                               self.bo, X if cfg.get("residual") else None, self.ws,
+                               self.ws_bytes, Y)
+        else:
+            tp.tp_mlp_forward(X, self.M, h, cfg["ffn"], n, self.A, self.b1, self.B, self.b2,
+                              X if cfg.get("residual") else None, self.ws, self.ws_bytes, Y)
+
+
+def run_ours(args, cfg) -> None:
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    from tensor_transformer_layer_linear_b200 import tp
+
+    pk = peaks()
+    inp = synth.make_inputs(cfg, seed=rank)
+    model = Model(tp, torch, cfg, inp)
+    w = work(cfg)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        model.step()
+    assert tp.tp_get_last_error() == tp.TP_OK
+    barrier()
+
+    # device-timed region (inputs resident in HBM)
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    tp.tp_trace_begin(64 * args.steps)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        model.step()
+    ev1.record(stream)
+    barrier()
+    recs, launches = tp.tp_trace_end()
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    st = tp.tp_get_last_error()
+    if st != tp.TP_OK:
+        raise RuntimeError(f"device error during the timed region: {tp.tp_status_string(st)}")
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end-to-end through the public API with host buffers: pinned X in,
+    # layer, Y out, every step
+    M, h = model.M, cfg["h"]
+    Xh = torch.from_numpy(inp["X"].view(np.int16)).pin_memory()
+    Yh = torch.empty((M, h), dtype=torch.int16).pin_memory()
+    Xd = torch.empty_like(model.X)
+    Yd = torch.empty_like(model.Y)
+    for _ in range(2):
+        Xd.copy_(Xh, non_blocking=True)
+        model.step(Xd, Yd)
+        Yh.copy_(Yd, non_blocking=True)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        Xd.copy_(Xh, non_blocking=True)
+        model.step(Xd, Yd)
+        Yh.copy_(Yd, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # per-kernel figures from the trace of the timed region
+    per = {}
+    for name, kms in recs:
+        a = per.setdefault(name, [0, 0.0])
+        a[0] += 1
+        a[1] += kms
+    total_k = sum(v[1] for v in per.values())
+    dom = max(per, key=lambda k: per[k][1])
+    steps_traced = args.steps
+
+    def kernel_fig(name):
+        n_l, t_ms = per[name]
+        if name in w["flops"] and w["flops"][name] > 0:
+            units = w["flops"][name] * steps_traced
+            achieved = units / (t_ms * 1e-3) / 1e12
+            return dict(bound="tensor", achieved=achieved, peak=pk["bf16"], unit="TFLOP/s",
+                        frac=achieved / pk["bf16"], launches=n_l,
+                        avg_launch_ms=t_ms / n_l, share=t_ms / total_k,
+                        traffic=NCU_TRAFFIC.get((cfg["name"], name)))
+        units = w["bytes"][name] * steps_traced
+        achieved = units / (t_ms * 1e-3) / 1e9
+        return dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
+                    frac=achieved / pk["hbm"], launches=n_l, avg_launch_ms=t_ms / n_l,
+                    share=t_ms / total_k, traffic=NCU_TRAFFIC.get((cfg["name"], name)))
+
+    roof = kernel_fig(dom)
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{pk['source']} (burst bf16 {pk['bf16']} TFLOP/s, HBM {pk['hbm']} GB/s)"
+    kernels = {k: kernel_fig(k) for k in per}
+    reduce_fig = kernels.get("reduce_partials")
+
+    value = w["total_flops"] * world / (ms * 1e-3) / 1e12
+    e2e_value = w["total_flops"] * world / (e2e_ms * 1e-3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        T = sample_tokens(cfg)
+        dt, fl, threads = oracle_sample(cfg, inp, T)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"first {T} tokens of sequence 0 (causal prefix) of {cfg['name']}, "
+                         f"fp64 numpy oracle, {fl / 1e9:.1f} GFLOP in {dt:.2f} s"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg["name"], "tokens": M, "h": h, "n_shards": cfg["n_shards"],
+                   "heads": cfg.get("n_heads"), "ffn": cfg.get("ffn"),
+                   "l2": "inputs larger than L2 (per-step working set "
+                         f"{(w['bytes'].get('reduce_partials', 0) + 4 * h * h * 2) / 1e6:.0f}+ MB "
+                         "vs 126 MB L2), no flush",
+                   "parallelism": f"{cfg['n_shards']} tensor-parallel shards on one GPU"
+                                  + (f", {world} independent replicas" if world > 1 else "")},
+        "roofline": roof,
+        "partial_reduce": reduce_fig,
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * h * 2,
+                "d2h_bytes_per_step": M * h * 2, "ms_per_step": e2e_ms},
+        "clocks": clocks,
+        "gpu_launches": launches,
+        "gflop_per_step": w["total_flops"] / 1e9,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--shards", type=int, default=0, help="override the shard count N")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = synth.config(args.workload)
+    if args.shards:
+        cfg["n_shards"] = args.shards
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,262 @@
+/*
+ * tp.h - C ABI of libtp.so: the Megatron-LM tensor-parallel Transformer layer
+ * on one B200 (sm_100a), with the N tensor-parallel shards held as N
+ * independent shard buffers of one GPU.
+ *
+ * Sources, cited by page title and section:
+ *   [TP-LLM] "Tensor Parallelism in Large Language Models: How Megatron-LM
+ *            Partitions Multi-Layer Perceptrons and Attention Heads"
+ *            (llms.blog): "The Core Primitives: Column-Parallel and
+ *            Row-Parallel Linear Layers", "Partitioning the Multi-Layer
+ *            Perceptron (MLP) Block", "Partitioning Multi-Head and
+ *            Grouped-Query Attention", "Sequence Parallelism".
+ *   [M-LM]   "Megatron-LM" (ai360xpert.com), "How It Works".
+ *   [INTRO]  "Introduction to Megatron-LM" (apxml.com), "Core Contributions"
+ *            (ColumnParallelLinear(in_features, out_features,
+ *            tensor_model_parallel_size) example).
+ *
+ * Conventions shared by every call
+ *   - Problem statement of [TP-LLM] "The Core Primitives": X in R^{B x H_in},
+ *     W in R^{H_in x H_out}, Y = X W, shard count N. B counts tokens
+ *     (batch x sequence).
+ *   - Tensors are DEVICE pointers unless a name says host_. bf16 tensors are
+ *     passed as uint16_t bit patterns, fp32 as float. Every matrix is
+ *     row-major and contiguous. Device pointers must be 16-byte aligned.
+ *   - The caller owns every buffer (allocated and freed by the caller); the
+ *     library allocates no device memory. Intermediates of the block calls
+ *     live in a caller-provided workspace sized by tp_workspace_bytes().
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream). Argument errors are returned before anything is
+ *     launched. A device-side failure (a bounded wait that expired inside a
+ *     kernel) is recorded in a per-device error word and reported by
+ *     tp_get_last_error(); no kernel traps or spins without a bound.
+ *   - Weight shards use the packed layout produced by tp_shard_weights():
+ *     shard i is stored transposed (K-major), contiguous, one after another.
+ *   - Arithmetic: bf16 inputs, fp32 accumulation, bf16 activations between
+ *     the kernels, fp32 row-parallel partial sums.
+ */
+#ifndef TP_H
+#define TP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TP_OK = 0,
+    TP_ERR_NULL = 1,        /* a required pointer is NULL */
+    TP_ERR_SHAPE = 2,       /* a size <= 0, a dimension not divisible by N
+                               (H_out % N, H_in % N, heads % N), or a size
+                               not a multiple of 8 elements where stated */
+    TP_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned */
+    TP_ERR_WORKSPACE = 4,   /* ws_bytes < tp_workspace_bytes(...) */
+    TP_ERR_UNSUPPORTED = 5, /* an option the kernels do not implement
+                               (e.g. head_dim != 128), or not an sm_100 GPU */
+    TP_ERR_CUDA = 6,        /* a CUDA runtime or driver call failed */
+    TP_ERR_TIMEOUT = 7      /* a bounded wait inside a kernel expired */
+} tp_status;
+
+typedef enum {
+    /* [TP-LLM] "Column-Parallel Linear Layer": W = [W_1 ... W_N] along
+       H_out, W_i in R^{H_in x H_out/N}. Packed shard i = W_i^T, shape
+       [H_out/N][H_in]. */
+    TP_SPLIT_COLUMN = 0,
+    /* [TP-LLM] "Row-Parallel Linear Layer": W = [W_1; ...; W_N] along H_in,
+       W_i in R^{H_in/N x H_out}. Packed shard i = W_i^T, shape
+       [H_out][H_in/N]. */
+    TP_SPLIT_ROW = 1,
+    /* [TP-LLM] attention, "Q, K, V Projections": W = [W_Q | W_K | W_V]
+       (H_out = 3h), each sliced column-wise by whole heads; shard i owns
+       heads [i n_h/N, (i+1) n_h/N), head k being columns [k d, (k+1) d) of
+       each projection. Packed shard i = [Q_i | K_i | V_i]^T, shape
+       [3h/N][H_in]. */
+    TP_SPLIT_QKV_HEADS = 2
+} tp_split;
+
+typedef enum {
+    TP_ACT_NONE = 0,
+    /* GeLU(x) = 0.5 x (1 + erf(x / sqrt 2)), applied per column shard
+       ([TP-LLM] "Column-Parallel Linear Layer": an element-wise function is
+       applied to the local slice; [M-LM] step 1). */
+    TP_ACT_GELU_ERF = 1
+} tp_act;
+
+typedef enum { TP_WS_MLP = 0, TP_WS_ATTN = 1, TP_WS_LAYER = 2 } tp_ws_kind;
+
+/* Weights of one pre-LN layer, all device pointers in the packed shard
+   layouts below. h = hidden, F = FFN width, N = shards. */
+typedef struct {
+    const uint16_t* ln1_gamma;   /* [h] */
+    const uint16_t* ln1_beta;    /* [h] */
+    const uint16_t* Wqkv_shards; /* TP_SPLIT_QKV_HEADS of [h][3h]: [N][3h/N][h] */
+    const uint16_t* bqkv_shards; /* TP_SPLIT_QKV_HEADS of [1][3h]: [N][3h/N] */
+    const uint16_t* Wo_shards;   /* TP_SPLIT_ROW of [h][h]: [N][h][h/N] */
+    const uint16_t* bo;          /* [h], added once after the sum */
+    const uint16_t* ln2_gamma;   /* [h] */
+    const uint16_t* ln2_beta;    /* [h] */
+    const uint16_t* A_shards;    /* TP_SPLIT_COLUMN of [h][F]: [N][F/N][h] */
+    const uint16_t* b1_shards;   /* [N][F/N] (= the F-vector b1 itself) */
+    const uint16_t* B_shards;    /* TP_SPLIT_ROW of [F][h]: [N][h][F/N] */
+    const uint16_t* b2;          /* [h], added once after the sum */
+} tp_layer_weights;
+
+/* tp_shard_weights - pack W (H_in x H_out, bf16) into N shards.
+ * [TP-LLM] "The Core Primitives" (column and row splits); attention section
+ * (head split). out[i] = W_i^T, contiguous: [N][cols_i][rows_i] with
+ * (cols_i, rows_i) = (H_out/N, H_in) for COLUMN, (H_out, H_in/N) for ROW,
+ * (H_out/N, H_in) for QKV_HEADS (H_out = 3h, head_dim = d). A bias vector is
+ * packed by passing it as a 1 x H_out matrix. Exact copy (bit-for-bit).
+ * Errors: TP_ERR_SHAPE if the split dimension is not divisible by N (or, for
+ * QKV_HEADS, H_out % 3, h % head_dim or n_heads % N is not 0). W and out
+ * must not overlap. */
+tp_status tp_shard_weights(const uint16_t* W, int64_t h_in, int64_t h_out,
+                           int n_shards, int kind, int64_t head_dim,
+                           uint16_t* W_shards, void* stream);
+
+/* tp_shard_index_map - host-only: for every split index (a column of W for
+ * COLUMN and QKV_HEADS, a row for ROW) the owning shard and the position
+ * inside it. host_owner and host_local are HOST arrays of length H_out
+ * (COLUMN, QKV_HEADS) or H_in (ROW). Launches nothing. */
+tp_status tp_shard_index_map(int kind, int64_t h_in, int64_t h_out,
+                             int n_shards, int64_t head_dim,
+                             int32_t* host_owner, int64_t* host_local);
+
+/* tp_column_linear - Y_i = act(X W_i + b_i) for every shard i, one launch.
+ * [TP-LLM] "Column-Parallel Linear Layer" (X replicated, Y_i = X W_i, no
+ * communication; element-wise activation on the local slice).
+ * X [B][H_in]; W_shards [N][H_out/N][H_in] (packed); bias_shards [N][H_out/N]
+ * or NULL; Y_shards [N][B][H_out/N] (shard-major: the column gather of
+ * [INTRO] is a view, not a copy). H_in and H_out/N must be multiples of 8. */
+tp_status tp_column_linear(const uint16_t* X, int64_t B, int64_t h_in,
+                           const uint16_t* W_shards,
+                           const uint16_t* bias_shards, int64_t h_out,
+                           int n_shards, int act, uint16_t* Y_shards,
+                           void* stream);
+
+/* tp_row_linear - partials P_i = X_i W_i (each B x H_out, fp32), one launch.
+ * [TP-LLM] "Row-Parallel Linear Layer" (X = [X_1 ... X_N] along channels,
+ * Y_i = X_i W_i full size). X_shards [N][B][H_in/N]; W_shards
+ * [N][H_out][H_in/N] (packed); partials [N][B][H_out] fp32. H_in/N and H_out
+ * must be multiples of 8. */
+tp_status tp_row_linear(const uint16_t* X_shards, int64_t B, int64_t h_in,
+                        const uint16_t* W_shards, int64_t h_out, int n_shards,
+                        float* partials, void* stream);
+
+/* tp_reduce_partials - Y = sum_{i<N} P_i + bias + residual, bf16 out.
+ * [TP-LLM] "Row-Parallel Linear Layer" (Y = sum_i Y_i = X W, the all-reduce
+ * sum) done as one on-device sum of N shard buffers, fp32 in shard order,
+ * one rounding to bf16. partials [N][B][H_out] fp32; bias [H_out] or NULL;
+ * residual [B][H_out] or NULL; Y [B][H_out]. H_out % 8 == 0. */
+tp_status tp_reduce_partials(const float* partials, int n_shards, int64_t B,
+                             int64_t h_out, const uint16_t* bias,
+                             const uint16_t* residual, uint16_t* Y,
+                             void* stream);
+
+/* tp_reduce_partials_layernorm - the same sum, plus LN of it:
+ * S = bf16(sum_i P_i + bias + residual) written to Y_sum, and
+ * Y_ln = LN(S) = gamma (S - mean) / sqrt(var + eps) + beta (population
+ * variance, fp32 statistics). The residual stream of a pre-LN layer and the
+ * next LayerNorm in one pass ([TP-LLM] "Sequence Parallelism": LayerNorm and
+ * residual adds are replicated around the blocks). H_out % 8 == 0 and
+ * H_out <= 16384. */
+tp_status tp_reduce_partials_layernorm(const float* partials, int n_shards,
+                                       int64_t B, int64_t h_out,
+                                       const uint16_t* bias,
+                                       const uint16_t* residual,
+                                       const uint16_t* gamma,
+                                       const uint16_t* beta, float eps,
+                                       uint16_t* Y_sum, uint16_t* Y_ln,
+                                       void* stream);
+
+/* tp_layernorm - Y = gamma (X - mean) / sqrt(var + eps) + beta per token row
+ * (population variance, fp32 statistics). X, Y [B][h]; gamma, beta [h].
+ * h % 8 == 0 and h <= 16384. */
+tp_status tp_layernorm(const uint16_t* X, int64_t B, int64_t h,
+                       const uint16_t* gamma, const uint16_t* beta, float eps,
+                       uint16_t* Y, void* stream);
+
+/* tp_attention - local scaled dot-product attention of every shard's heads:
+ * Head = softmax(Q K^T / sqrt(d_k)) V per (sequence, head), d_k = h/n_heads
+ * ([TP-LLM] "Local Self-Attention Computation"). With causal != 0 query t
+ * of a sequence sees keys 0..t of the same sequence; attention never
+ * crosses sequences. QKV_shards [N][batch*seq][3h/N] with each shard's
+ * columns [Q_i | K_i | V_i] (the output of tp_column_linear on
+ * TP_SPLIT_QKV_HEADS weights); O_shards [N][batch*seq][h/N], the shard's
+ * head outputs concatenated in head order. head_dim must be 128. */
+tp_status tp_attention(const uint16_t* QKV_shards, int64_t batch,
+                       int64_t seq, int64_t h, int64_t n_heads, int causal,
+                       int n_shards, uint16_t* O_shards, void* stream);
+
+/* tp_mlp_forward - Y = GeLU(X A + b1) B + b2 + residual, by the
+ * tensor-parallel route: column-parallel A with per-shard bias + GeLU,
+ * row-parallel B into N fp32 partials, one on-device sum with b2 and the
+ * residual ([TP-LLM] "Partitioning the Multi-Layer Perceptron (MLP) Block";
+ * [M-LM] "How It Works"). X [B][h]; A_shards [N][F/N][h]; b1_shards [N][F/N]
+ * or NULL; B_shards [N][h][F/N]; b2 [h] or NULL; residual [B][h] or NULL;
+ * Y [B][h]. ws >= tp_workspace_bytes(TP_WS_MLP, B, h, F, N) bytes. */
+tp_status tp_mlp_forward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn,
+                         int n_shards, const uint16_t* A_shards,
+                         const uint16_t* b1_shards, const uint16_t* B_shards,
+                         const uint16_t* b2, const uint16_t* residual,
+                         void* ws, size_t ws_bytes, uint16_t* Y, void* stream);
+
+/* tp_attn_forward - Y = concat_heads(attention) W_O + b_O + residual by the
+ * tensor-parallel route: QKV column-parallel by whole heads (+ bias), local
+ * attention per shard, W_O row-parallel into N partials, one sum
+ * ([TP-LLM] "Partitioning Multi-Head and Grouped-Query Attention" steps
+ * 1-4). X [batch*seq][h]; Wqkv_shards [N][3h/N][h]; bqkv_shards [N][3h/N] or
+ * NULL; Wo_shards [N][h][h/N]; bo [h] or NULL; residual [batch*seq][h] or
+ * NULL; Y [batch*seq][h]. head_dim = h/n_heads must be 128.
+ * ws >= tp_workspace_bytes(TP_WS_ATTN, batch*seq, h, 0, N). */
+tp_status tp_attn_forward(const uint16_t* X, int64_t batch, int64_t seq,
+                          int64_t h, int64_t n_heads, int causal,
+                          int n_shards, const uint16_t* Wqkv_shards,
+                          const uint16_t* bqkv_shards,
+                          const uint16_t* Wo_shards, const uint16_t* bo,
+                          const uint16_t* residual, void* ws, size_t ws_bytes,
+                          uint16_t* Y, void* stream);
+
+/* tp_layer_forward - pre-LN Transformer layer, causal attention:
+ * h1 = X + Attn(LN1(X)); Y = h1 + MLP(LN2(h1)), both blocks by the
+ * tensor-parallel route with one partial-sum reduction each.
+ * X, Y [batch*seq][h]; w: see tp_layer_weights.
+ * ws >= tp_workspace_bytes(TP_WS_LAYER, batch*seq, h, F, N). */
+tp_status tp_layer_forward(const uint16_t* X, int64_t batch, int64_t seq,
+                           int64_t h, int64_t n_heads, int64_t ffn,
+                           int n_shards, const tp_layer_weights* w,
+                           float ln_eps, void* ws, size_t ws_bytes,
+                           uint16_t* Y, void* stream);
+
+/* Workspace bytes for tp_mlp_forward (kind TP_WS_MLP), tp_attn_forward
+ * (TP_WS_ATTN, ffn ignored) or tp_layer_forward (TP_WS_LAYER). tokens =
+ * batch * seq. Returns 0 for invalid arguments. */
+size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn,
+                          int n_shards);
+
+/* Synchronizes `stream`, then reads and clears the current device's error
+ * word. TP_ERR_TIMEOUT if a kernel gave up a bounded wait since the last
+ * call, TP_ERR_CUDA if the stream reports a CUDA error, else TP_OK. */
+tp_status tp_get_last_error(void* stream);
+
+/* Static string for a status code. */
+const char* tp_status_string(int status);
+
+/* Kernel launch trace (used by benchmarks): while enabled, every kernel the
+ * library launches is bracketed by two CUDA events on its stream.
+ * tp_trace_begin(max_records) starts a trace (max_records launches at most;
+ * later launches are counted but not timed); tp_trace_end() synchronizes
+ * the device and returns the number of launches seen. tp_trace_record(k)
+ * gives launch k's kernel id (host_kernel_id) and its device time in
+ * milliseconds (host_ms). Kernel ids are those of tp_kernel_name(). */
+tp_status tp_trace_begin(int max_records);
+int tp_trace_end(void);
+tp_status tp_trace_record(int k, int* host_kernel_id, float* host_ms);
+const char* tp_kernel_name(int kernel_id);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TP_H */

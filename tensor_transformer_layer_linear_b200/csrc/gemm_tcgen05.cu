@@ -1,0 +1,352 @@
+// Column- and row-parallel projections on the 5th-generation tensor cores.
+//
+// One persistent, warp-specialized kernel computes every shard's GEMM in a
+// single launch ("Tensor Parallelism in Large Language Models", sections
+// "Column-Parallel Linear Layer" and "Row-Parallel Linear Layer": each of
+// the N shards computes X W_i, resp. X_i W_i, with no exchange):
+//
+//   warp 0      TMA producer: 128-byte-swizzled A and B tiles (BK = 64) into
+//               a ring of shared-memory stages, completion on mbarriers.
+//   warp 1      owns TMEM (two BM x BN fp32 accumulators) and one thread
+//               issues tcgen05.mma (M = 128, N = BN, K = 16) per stage,
+//               releasing the stage with tcgen05.commit.
+//   warps 2-5   epilogue: tcgen05.ld of the finished accumulator, then the
+//               column-parallel bias + GeLU (bf16 out) or the row-parallel
+//               fp32 partial store, overlapping the next tile's mainloop.
+//
+// Tiles are (shard g, m-block, n-block), m fastest, strided over the
+// CTAs. Every barrier wait is bounded; on expiry the CTA records an error
+// bit, stops all roles, waits for its own copies and MMAs in flight, frees
+// TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "tp_device.cuh"
+#include "tp_internal.h"
+
+namespace tpk {
+
+constexpr int BM = 128;
+constexpr int BK = 64;             // 64 bf16 = 128 bytes = one swizzle row
+constexpr int kGemmThreads = 192;  // 6 warps
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kNumBars * 8 + 16;
+};
+
+struct GemmParams {
+  int M, Nc, K, G;
+  int num_m, num_n, num_k, num_tiles;
+  int a_batched;
+  int act;
+  void* out;
+  const uint16_t* bias;
+  unsigned* err;
+};
+
+template <int BN, bool OUT_F32>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t* tiles = smem_raw + pad;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tiles + C::kStages * C::kStageBytes);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const int mb = tile % p.num_m;
+        const int rest = tile / p.num_m;
+        const int nb = rest % p.num_n;
+        const int g = rest / p.num_n;
+        for (int kb = 0; kb < p.num_k; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = smem_u32(tiles + stage * C::kStageBytes);
+          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+          tma_load_3d(sa, &tmA, full_bar(stage), kb * BK, mb * BM, p.a_batched ? g : 0);
+          tma_load_3d(sa + C::kABytes, &tmB, full_bar(stage), kb * BK, nb * BN, g);
+          ++issued;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        atomicOr(p.err, ERR_WAIT_PRODUCER);
+        *abort_flag = 1;
+      }
+      // Every armed stage must have landed before the CTA may exit.
+      for (int s = 0; s < C::kStages && s < issued; ++s) {
+        const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+        int never = 0;
+        if (!mbar_wait(full_bar(s), par, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.num_k; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(tiles + stage * C::kStageBytes);
+          const uint32_t sb = sa + C::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            umma_bf16(d_tmem, umma_desc_sw128(sa + kk * 32), umma_desc_sw128(sb + kk * 32), idesc,
+                      (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(empty_bar(stage));
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        atomicOr(p.err, ERR_WAIT_MMA);
+        *abort_flag = 1;
+      }
+      // All MMAs issued by this thread must be complete before TMEM is freed.
+      umma_commit(drain_bar);
+      int never = 0;
+      if (!mbar_wait(drain_bar, 0, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lanes [32 q, 32 q + 32) are this warp's
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int mb = tile % p.num_m;
+      const int rest = tile / p.num_m;
+      const int nb = rest % p.num_n;
+      const int g = rest / p.num_n;
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int row = mb * BM + q * 32 + lane;
+      const bool row_ok = row < p.M;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const int64_t out_row = (static_cast<int64_t>(g) * p.M + row) * p.Nc;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tbase + c * 32, r);
+        tmem_ld_wait();
+        const int col0 = nb * BN + c * 32;
+        if (row_ok && col0 < p.Nc) {
+          if constexpr (OUT_F32) {
+            float* out = static_cast<float*>(p.out) + out_row;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int col = col0 + 4 * j;
+              if (col < p.Nc) {
+                float4 v = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                       __uint_as_float(r[4 * j + 2]),
+                                       __uint_as_float(r[4 * j + 3]));
+                *reinterpret_cast<float4*>(out + col) = v;
+              }
+            }
+          } else {
+            uint16_t* out = static_cast<uint16_t*>(p.out) + out_row;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int col = col0 + 8 * j;
+              if (col < p.Nc) {
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * j + e]);
+                if (p.bias != nullptr) {
+                  const uint4 b = *reinterpret_cast<const uint4*>(
+                      p.bias + static_cast<int64_t>(g) * p.Nc + col);
+                  v[0] += bf16_lo(b.x); v[1] += bf16_hi(b.x);
+                  v[2] += bf16_lo(b.y); v[3] += bf16_hi(b.y);
+                  v[4] += bf16_lo(b.z); v[5] += bf16_hi(b.z);
+                  v[6] += bf16_lo(b.w); v[7] += bf16_hi(b.w);
+                }
+                if (p.act == 1) {
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) v[e] = gelu_erf(v[e]);
+                }
+                uint4 o;
+                o.x = pack_bf16x2(v[0], v[1]);
+                o.y = pack_bf16x2(v[2], v[3]);
+                o.z = pack_bf16x2(v[4], v[5]);
+                o.w = pack_bf16x2(v[6], v[7]);
+                *reinterpret_cast<uint4*>(out + col) = o;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(p.err, ERR_WAIT_EPILOGUE);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [d2][d1][d0] bf16 tensor, boxes of box0 x box1 x 1 with the 128-byte swizzle;
+// out-of-range elements read as zero.
+static bool encode_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint32_t box0, uint32_t box1) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, bool OUT_F32>
+static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, int num_sms) {
+  using C = GemmCfg<BN>;
+  CUtensorMap tmA, tmB;
+  if (!encode_3d(&tmA, pr.A, pr.K, pr.M, pr.a_batched ? pr.G : 1, BK, BM)) return 1;
+  if (!encode_3d(&tmB, pr.B, pr.K, pr.Nc, pr.G, BK, BN)) return 1;
+  GemmParams p;
+  p.M = pr.M;
+  p.Nc = pr.Nc;
+  p.K = pr.K;
+  p.G = pr.G;
+  p.num_m = (pr.M + BM - 1) / BM;
+  p.num_n = (pr.Nc + BN - 1) / BN;
+  p.num_k = (pr.K + BK - 1) / BK;
+  p.num_tiles = p.num_m * p.num_n * pr.G;
+  p.a_batched = pr.a_batched ? 1 : 0;
+  p.act = pr.act;
+  p.out = pr.D;
+  p.bias = static_cast<const uint16_t*>(pr.bias);
+  p.err = err;
+  auto kern = gemm_tcgen05_kernel<BN, OUT_F32>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+  kern<<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmA, tmB, p);
+  return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
+
+int launch_gemm(const GemmProblem& p, cudaStream_t s, unsigned* err, int num_sms) {
+  const bool wide = p.Nc > 128;
+  if (p.out_f32)
+    return wide ? launch_gemm_t<256, true>(p, s, err, num_sms)
+                : launch_gemm_t<128, true>(p, s, err, num_sms);
+  return wide ? launch_gemm_t<256, false>(p, s, err, num_sms)
+              : launch_gemm_t<128, false>(p, s, err, num_sms);
+}
+
+}  // namespace tpk

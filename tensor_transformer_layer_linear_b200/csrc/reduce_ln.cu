@@ -1,0 +1,225 @@
+// The block-output reduction of the N row-parallel partials, and the
+// replicated LayerNorm around the blocks.
+//
+// "Tensor Parallelism in Large Language Models", "Row-Parallel Linear
+// Layer": the true output is Y = sum_i Y_i, obtained across GPUs by an
+// all-reduce sum. With the N shards held as N buffers of one GPU the
+// all-reduce is a streaming sum of N fp32 partials, fused here with the
+// output bias and the residual add (each added once), one bf16 rounding.
+// The kernel is HBM-bound: it reads N*rows*h*4 + rows*h*2 + h*2 bytes and
+// writes rows*h*2, with 128-bit loads and stores, partials streamed with
+// evict-first loads, grid sized to a multiple of the SM count.
+//
+// LayerNorm ("Sequence Parallelism": LayerNorm, dropout and residual adds are
+// replicated on every rank): one CTA per token row, fp32 statistics with
+// warp shuffles, population variance; it can be fused behind the sum so the
+// residual stream h1 and LN(h1) leave in one pass.
+#include "tp_device.cuh"
+#include "tp_internal.h"
+
+namespace tpk {
+
+__device__ __forceinline__ void add_bf16x8(float (&a)[8], const uint4& b) {
+  a[0] += bf16_lo(b.x); a[1] += bf16_hi(b.x);
+  a[2] += bf16_lo(b.y); a[3] += bf16_hi(b.y);
+  a[4] += bf16_lo(b.z); a[5] += bf16_hi(b.z);
+  a[6] += bf16_lo(b.w); a[7] += bf16_hi(b.w);
+}
+
+__device__ __forceinline__ uint4 to_bf16x8(const float (&a)[8]) {
+  uint4 o;
+  o.x = pack_bf16x2(a[0], a[1]);
+  o.y = pack_bf16x2(a[2], a[3]);
+  o.z = pack_bf16x2(a[4], a[5]);
+  o.w = pack_bf16x2(a[6], a[7]);
+  return o;
+}
+
+// Sum of the N partials at element offset e (8 consecutive fp32), in shard
+// order 0..N-1. NS > 0: compile-time N (all loads issued before the adds).
+template <int NS>
+__device__ __forceinline__ void sum_partials8(const float* __restrict__ P, int n_shards,
+                                              int64_t stride, int64_t e, float (&acc)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  if constexpr (NS > 0) {
+    float4 v[NS][2];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      const float4* src = reinterpret_cast<const float4*>(P + s * stride + e);
+      v[s][0] = __ldcs(src);
+      v[s][1] = __ldcs(src + 1);
+    }
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      acc[0] += v[s][0].x; acc[1] += v[s][0].y; acc[2] += v[s][0].z; acc[3] += v[s][0].w;
+      acc[4] += v[s][1].x; acc[5] += v[s][1].y; acc[6] += v[s][1].z; acc[7] += v[s][1].w;
+    }
+  } else {
+    for (int s = 0; s < n_shards; ++s) {
+      const float4* src = reinterpret_cast<const float4*>(P + s * stride + e);
+      const float4 a = __ldcs(src), b = __ldcs(src + 1);
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+  }
+}
+
+template <int NS>
+__global__ void __launch_bounds__(256) reduce_partials_kernel(
+    const float* __restrict__ P, int n_shards, int64_t n_elems, int h,
+    const uint16_t* __restrict__ bias, const uint16_t* __restrict__ res,
+    uint16_t* __restrict__ Y) {
+  const int64_t n8 = n_elems >> 3;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t e = i << 3;
+    float acc[8];
+    sum_partials8<NS>(P, n_shards, n_elems, e, acc);
+    if (bias != nullptr) add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(bias + e % h)));
+    if (res != nullptr) add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(res + e)));
+    *reinterpret_cast<uint4*>(Y + e) = to_bf16x8(acc);
+  }
+}
+
+constexpr int kRowThreads = 256;
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < kRowThreads / 32; ++i) t += red[i];
+  __syncthreads();
+  return t;
+}
+
+// One CTA per row. CH = 8-element chunks per thread (h <= CH * 8 * 256).
+template <int CH, int NS>
+__global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
+    const float* __restrict__ P, int n_shards, int64_t stride, int h,
+    const uint16_t* __restrict__ bias, const uint16_t* __restrict__ res,
+    const uint16_t* __restrict__ gamma, const uint16_t* __restrict__ beta, float eps,
+    uint16_t* __restrict__ Ysum, uint16_t* __restrict__ Yln) {
+  __shared__ float red[kRowThreads / 32];
+  const int64_t row_off = static_cast<int64_t>(blockIdx.x) * h;
+  const int nch = h >> 3;
+  float v[CH][8];
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    const int ch = threadIdx.x + c * kRowThreads;
+    if (ch < nch) {
+      const int64_t e = row_off + (ch << 3);
+      if (n_shards > 0) {
+        sum_partials8<NS>(P, n_shards, stride, e, v[c]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[c][j] = 0.f;
+      }
+      if (bias != nullptr) add_bf16x8(v[c], __ldg(reinterpret_cast<const uint4*>(bias + (ch << 3))));
+      if (res != nullptr) add_bf16x8(v[c], __ldg(reinterpret_cast<const uint4*>(res + e)));
+      const uint4 o = to_bf16x8(v[c]);
+      if (Ysum != nullptr) *reinterpret_cast<uint4*>(Ysum + e) = o;
+      // statistics of the rounded values, as a separate LayerNorm would see them
+      v[c][0] = bf16_lo(o.x); v[c][1] = bf16_hi(o.x);
+      v[c][2] = bf16_lo(o.y); v[c][3] = bf16_hi(o.y);
+      v[c][4] = bf16_lo(o.z); v[c][5] = bf16_hi(o.z);
+      v[c][6] = bf16_lo(o.w); v[c][7] = bf16_hi(o.w);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s += v[c][j];
+    }
+  }
+  if (Yln == nullptr) return;
+  const float mean = block_sum(s, red) / static_cast<float>(h);
+  float q = 0.f;
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    const int ch = threadIdx.x + c * kRowThreads;
+    if (ch < nch) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float d = v[c][j] - mean;
+        q += d * d;
+      }
+    }
+  }
+  const float var = block_sum(q, red) / static_cast<float>(h);
+  const float rstd = rsqrtf(var + eps);
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    const int ch = threadIdx.x + c * kRowThreads;
+    if (ch < nch) {
+      const uint4 g = __ldg(reinterpret_cast<const uint4*>(gamma + (ch << 3)));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(beta + (ch << 3)));
+      float gv[8] = {bf16_lo(g.x), bf16_hi(g.x), bf16_lo(g.y), bf16_hi(g.y),
+                     bf16_lo(g.z), bf16_hi(g.z), bf16_lo(g.w), bf16_hi(g.w)};
+      float bv[8] = {bf16_lo(b.x), bf16_hi(b.x), bf16_lo(b.y), bf16_hi(b.y),
+                     bf16_lo(b.z), bf16_hi(b.z), bf16_lo(b.w), bf16_hi(b.w)};
+      float y[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[j] = (v[c][j] - mean) * rstd * gv[j] + bv[j];
+      *reinterpret_cast<uint4*>(Yln + row_off + (ch << 3)) = to_bf16x8(y);
+    }
+  }
+}
+
+int launch_reduce(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
+                  const void* residual, void* Y, cudaStream_t s, int num_sms) {
+  const int64_t n = rows * h;
+  const int64_t n8 = n / 8;
+  int64_t blocks = (n8 + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  auto b = static_cast<const uint16_t*>(bias);
+  auto r = static_cast<const uint16_t*>(residual);
+  auto y = static_cast<uint16_t*>(Y);
+  const int hh = static_cast<int>(h);
+  switch (n_shards) {
+    case 1: reduce_partials_kernel<1><<<blocks, 256, 0, s>>>(P, 1, n, hh, b, r, y); break;
+    case 2: reduce_partials_kernel<2><<<blocks, 256, 0, s>>>(P, 2, n, hh, b, r, y); break;
+    case 4: reduce_partials_kernel<4><<<blocks, 256, 0, s>>>(P, 4, n, hh, b, r, y); break;
+    case 8: reduce_partials_kernel<8><<<blocks, 256, 0, s>>>(P, 8, n, hh, b, r, y); break;
+    case 16: reduce_partials_kernel<16><<<blocks, 256, 0, s>>>(P, 16, n, hh, b, r, y); break;
+    default: reduce_partials_kernel<0><<<blocks, 256, 0, s>>>(P, n_shards, n, hh, b, r, y); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
+
+template <int CH>
+static void launch_rows_ch(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
+                           const void* residual, const void* gamma, const void* beta, float eps,
+                           void* Y_sum, void* Y_ln, cudaStream_t s) {
+  auto b = static_cast<const uint16_t*>(bias);
+  auto r = static_cast<const uint16_t*>(residual);
+  auto g = static_cast<const uint16_t*>(gamma);
+  auto be = static_cast<const uint16_t*>(beta);
+  auto ys = static_cast<uint16_t*>(Y_sum);
+  auto yl = static_cast<uint16_t*>(Y_ln);
+  const int64_t stride = rows * h;
+  const int hh = static_cast<int>(h);
+  const dim3 grid(static_cast<unsigned>(rows));
+  switch (n_shards) {
+    case 4: rows_sum_ln_kernel<CH, 4><<<grid, kRowThreads, 0, s>>>(P, 4, stride, hh, b, r, g, be, eps, ys, yl); break;
+    case 8: rows_sum_ln_kernel<CH, 8><<<grid, kRowThreads, 0, s>>>(P, 8, stride, hh, b, r, g, be, eps, ys, yl); break;
+    default: rows_sum_ln_kernel<CH, 0><<<grid, kRowThreads, 0, s>>>(P, n_shards, stride, hh, b, r, g, be, eps, ys, yl); break;
+  }
+}
+
+int launch_rows_sum_ln(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
+                       const void* residual, const void* gamma, const void* beta, float eps,
+                       void* Y_sum, void* Y_ln, cudaStream_t s) {
+  if (rows <= 0) return 0;
+  const int64_t nch = h / 8;
+  if (nch <= kRowThreads) launch_rows_ch<1>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  else if (nch <= 2 * kRowThreads) launch_rows_ch<2>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  else if (nch <= 4 * kRowThreads) launch_rows_ch<4>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  else launch_rows_ch<8>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
+
+}  // namespace tpk

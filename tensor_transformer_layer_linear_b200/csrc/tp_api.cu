@@ -1,0 +1,513 @@
+// The C ABI of libtp.so (declared in include/tp.h): argument checks,
+// workspace carving, the order of kernel launches for the MLP, attention and
+// layer blocks, the per-device error word and the launch trace.
+//
+// Block structure ("Tensor Parallelism in Large Language Models"):
+//   MLP       ColumnParallelLinear(A) + bias + GeLU  ->  RowParallelLinear(B)
+//             -> one sum of the N partials (+ b2 + residual)
+//   attention ColumnParallelLinear(W_QKV, whole heads) -> local attention
+//             -> RowParallelLinear(W_O) -> one sum (+ b_O + residual)
+//   layer     LN1 -> attention -> sum fused with the residual and LN2
+//             -> MLP -> sum (+ residual)
+// so every block has exactly one reduction, as the pages require.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "../../include/tp.h"
+#include "tp_internal.h"
+
+namespace {
+
+__device__ unsigned int g_tp_error_word;
+
+struct DevInfo {
+  bool ready = false;
+  tp_status status = TP_OK;
+  int num_sms = 0;
+  unsigned* err = nullptr;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+DevInfo g_dev[kMaxDevices];
+
+tp_status device_info(DevInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TP_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return TP_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      return TP_ERR_CUDA;
+    }
+    d.num_sms = sms;
+    if (major != 10) {
+      d.status = TP_ERR_UNSUPPORTED;  // the kernels are built for sm_100a only
+    } else {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_tp_error_word) != cudaSuccess) return TP_ERR_CUDA;
+      d.err = static_cast<unsigned*>(p);
+      d.status = TP_OK;
+    }
+    d.ready = true;
+  }
+  *out = d;
+  return d.status;
+}
+
+// ------------------------------------------------------------------ trace
+struct TraceRec {
+  int kid;
+  cudaEvent_t a, b;
+};
+std::atomic<bool> g_trace_on{false};
+std::mutex g_trace_mu;
+std::vector<cudaEvent_t> g_ev_pool;
+std::vector<TraceRec> g_trace;
+std::vector<float> g_trace_ms;
+int g_trace_max = 0;
+int g_trace_seen = 0;
+
+struct TraceScope {
+  cudaEvent_t end = nullptr;
+  cudaStream_t s;
+  TraceScope(int kid, cudaStream_t st) : s(st) {
+    if (!g_trace_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    const int k = g_trace_seen++;
+    if (k >= g_trace_max) return;
+    TraceRec r{kid, g_ev_pool[2 * k], g_ev_pool[2 * k + 1]};
+    g_trace.push_back(r);
+    cudaEventRecord(r.a, s);
+    end = r.b;
+  }
+  ~TraceScope() {
+    if (end != nullptr) cudaEventRecord(end, s);
+  }
+};
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+inline size_t round256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+constexpr int64_t kIntMax = 2147483647;
+
+tp_status gemm_status(int rc) {
+  return rc == 0 ? TP_OK : TP_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tp_status_string(int st) {
+  switch (st) {
+    case TP_OK: return "TP_OK";
+    case TP_ERR_NULL: return "TP_ERR_NULL: a required pointer is NULL";
+    case TP_ERR_SHAPE: return "TP_ERR_SHAPE: a size is invalid or not divisible by the shard count";
+    case TP_ERR_ALIGN: return "TP_ERR_ALIGN: a device pointer is not 16-byte aligned";
+    case TP_ERR_WORKSPACE: return "TP_ERR_WORKSPACE: workspace too small";
+    case TP_ERR_UNSUPPORTED: return "TP_ERR_UNSUPPORTED: option or device not supported (needs sm_100)";
+    case TP_ERR_CUDA: return "TP_ERR_CUDA: a CUDA call failed";
+    case TP_ERR_TIMEOUT: return "TP_ERR_TIMEOUT: a bounded wait inside a kernel expired";
+    default: return "unknown tp_status";
+  }
+}
+
+const char* tp_kernel_name(int kid) {
+  switch (kid) {
+    case tpk::KID_SHARD: return "shard_transpose";
+    case tpk::KID_GEMM_COLUMN: return "gemm_column_parallel";
+    case tpk::KID_GEMM_ROW: return "gemm_row_parallel";
+    case tpk::KID_REDUCE: return "reduce_partials";
+    case tpk::KID_REDUCE_LN: return "reduce_partials_layernorm";
+    case tpk::KID_LAYERNORM: return "layernorm";
+    case tpk::KID_ATTENTION: return "attention";
+    default: return "unknown";
+  }
+}
+
+tp_status tp_trace_begin(int max_records) {
+  if (max_records < 0) return TP_ERR_SHAPE;
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  while (static_cast<int>(g_ev_pool.size()) < 2 * max_records) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return TP_ERR_CUDA;
+    g_ev_pool.push_back(e);
+  }
+  g_trace.clear();
+  g_trace_ms.clear();
+  g_trace_max = max_records;
+  g_trace_seen = 0;
+  g_trace_on.store(true);
+  return TP_OK;
+}
+
+int tp_trace_end(void) {
+  g_trace_on.store(false);
+  cudaDeviceSynchronize();
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  g_trace_ms.assign(g_trace.size(), -1.f);
+  for (size_t k = 0; k < g_trace.size(); ++k) {
+    float ms = -1.f;
+    if (cudaEventElapsedTime(&ms, g_trace[k].a, g_trace[k].b) == cudaSuccess) g_trace_ms[k] = ms;
+  }
+  return g_trace_seen;
+}
+
+tp_status tp_trace_record(int k, int* host_kernel_id, float* host_ms) {
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  if (k < 0 || k >= static_cast<int>(g_trace_ms.size())) return TP_ERR_SHAPE;
+  if (host_kernel_id) *host_kernel_id = g_trace[k].kid;
+  if (host_ms) *host_ms = g_trace_ms[k];
+  return TP_OK;
+}
+
+tp_status tp_get_last_error(void* stream) {
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return TP_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  unsigned w = 0;
+  if (cudaMemcpyFromSymbol(&w, g_tp_error_word, sizeof(w)) != cudaSuccess) return TP_ERR_CUDA;
+  if (w != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_tp_error_word, &zero, sizeof(zero)) != cudaSuccess) return TP_ERR_CUDA;
+    return TP_ERR_TIMEOUT;
+  }
+  return TP_OK;
+}
+
+tp_status tp_shard_index_map(int kind, int64_t h_in, int64_t h_out, int n_shards,
+                             int64_t head_dim, int32_t* host_owner, int64_t* host_local) {
+  if (host_owner == nullptr || host_local == nullptr) return TP_ERR_NULL;
+  if (h_in <= 0 || h_out <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (kind == TP_SPLIT_COLUMN) {
+    if (h_out % n_shards) return TP_ERR_SHAPE;
+    const int64_t w = h_out / n_shards;
+    for (int64_t j = 0; j < h_out; ++j) {
+      host_owner[j] = static_cast<int32_t>(j / w);
+      host_local[j] = j % w;
+    }
+    return TP_OK;
+  }
+  if (kind == TP_SPLIT_ROW) {
+    if (h_in % n_shards) return TP_ERR_SHAPE;
+    const int64_t w = h_in / n_shards;
+    for (int64_t r = 0; r < h_in; ++r) {
+      host_owner[r] = static_cast<int32_t>(r / w);
+      host_local[r] = r % w;
+    }
+    return TP_OK;
+  }
+  if (kind == TP_SPLIT_QKV_HEADS) {
+    if (h_out % 3 || head_dim <= 0) return TP_ERR_SHAPE;
+    const int64_t h = h_out / 3;
+    if (h % head_dim) return TP_ERR_SHAPE;
+    const int64_t heads = h / head_dim;
+    if (heads % n_shards) return TP_ERR_SHAPE;
+    const int64_t hps = heads / n_shards, hs = h / n_shards;
+    for (int64_t j = 0; j < h_out; ++j) {
+      const int64_t part = j / h, within = j % h;
+      const int64_t owner = (within / head_dim) / hps;
+      host_owner[j] = static_cast<int32_t>(owner);
+      host_local[j] = part * hs + (within - owner * hs);
+    }
+    return TP_OK;
+  }
+  return TP_ERR_SHAPE;
+}
+
+tp_status tp_shard_weights(const uint16_t* W, int64_t h_in, int64_t h_out, int n_shards, int kind,
+                           int64_t head_dim, uint16_t* W_shards, void* stream) {
+  if (W == nullptr || W_shards == nullptr) return TP_ERR_NULL;
+  if (h_in <= 0 || h_out <= 0 || n_shards <= 0 || n_shards > 65535) return TP_ERR_SHAPE;
+  if (kind == TP_SPLIT_COLUMN) {
+    if (h_out % n_shards) return TP_ERR_SHAPE;
+  } else if (kind == TP_SPLIT_ROW) {
+    if (h_in % n_shards) return TP_ERR_SHAPE;
+  } else if (kind == TP_SPLIT_QKV_HEADS) {
+    if (h_out % 3 || head_dim <= 0 || (h_out / 3) % head_dim || ((h_out / 3) / head_dim) % n_shards)
+      return TP_ERR_SHAPE;
+  } else {
+    return TP_ERR_SHAPE;
+  }
+  const int64_t cols = (kind == TP_SPLIT_ROW) ? h_out : h_out / n_shards;
+  const int64_t rows = (kind == TP_SPLIT_ROW) ? h_in / n_shards : h_in;
+  if ((rows + 31) / 32 > kIntMax || (cols + 31) / 32 > 65535) return TP_ERR_SHAPE;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_SHARD, as_stream(stream));
+  return tpk::launch_shard(W, h_in, h_out, n_shards, kind, head_dim, W_shards, as_stream(stream)) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_column_linear(const uint16_t* X, int64_t B, int64_t h_in, const uint16_t* W_shards,
+                           const uint16_t* bias_shards, int64_t h_out, int n_shards, int act,
+                           uint16_t* Y_shards, void* stream) {
+  if (X == nullptr || W_shards == nullptr || Y_shards == nullptr) return TP_ERR_NULL;
+  if (B <= 0 || h_in <= 0 || h_out <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (h_out % n_shards) return TP_ERR_SHAPE;
+  const int64_t nc = h_out / n_shards;
+  if (h_in % 8 || nc % 8) return TP_ERR_SHAPE;
+  if (B > kIntMax || h_in > kIntMax || nc > kIntMax) return TP_ERR_SHAPE;
+  if (act != TP_ACT_NONE && act != TP_ACT_GELU_ERF) return TP_ERR_UNSUPPORTED;
+  if (!al16(X) || !al16(W_shards) || !al16(Y_shards) || (bias_shards && !al16(bias_shards)))
+    return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  tpk::GemmProblem p;
+  p.A = X;
+  p.B = W_shards;
+  p.D = Y_shards;
+  p.bias = bias_shards;
+  p.M = static_cast<int>(B);
+  p.Nc = static_cast<int>(nc);
+  p.K = static_cast<int>(h_in);
+  p.G = n_shards;
+  p.a_batched = false;
+  p.out_f32 = false;
+  p.act = act;
+  TraceScope ts(tpk::KID_GEMM_COLUMN, as_stream(stream));
+  return gemm_status(tpk::launch_gemm(p, as_stream(stream), d.err, d.num_sms));
+}
+
+tp_status tp_row_linear(const uint16_t* X_shards, int64_t B, int64_t h_in,
+                        const uint16_t* W_shards, int64_t h_out, int n_shards, float* partials,
+                        void* stream) {
+  if (X_shards == nullptr || W_shards == nullptr || partials == nullptr) return TP_ERR_NULL;
+  if (B <= 0 || h_in <= 0 || h_out <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (h_in % n_shards) return TP_ERR_SHAPE;
+  const int64_t k = h_in / n_shards;
+  if (k % 8 || h_out % 8) return TP_ERR_SHAPE;
+  if (B > kIntMax || k > kIntMax || h_out > kIntMax) return TP_ERR_SHAPE;
+  if (!al16(X_shards) || !al16(W_shards) || !al16(partials)) return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  tpk::GemmProblem p;
+  p.A = X_shards;
+  p.B = W_shards;
+  p.D = partials;
+  p.bias = nullptr;
+  p.M = static_cast<int>(B);
+  p.Nc = static_cast<int>(h_out);
+  p.K = static_cast<int>(k);
+  p.G = n_shards;
+  p.a_batched = true;
+  p.out_f32 = true;
+  p.act = 0;
+  TraceScope ts(tpk::KID_GEMM_ROW, as_stream(stream));
+  return gemm_status(tpk::launch_gemm(p, as_stream(stream), d.err, d.num_sms));
+}
+
+tp_status tp_reduce_partials(const float* partials, int n_shards, int64_t B, int64_t h_out,
+                             const uint16_t* bias, const uint16_t* residual, uint16_t* Y,
+                             void* stream) {
+  if (partials == nullptr || Y == nullptr) return TP_ERR_NULL;
+  if (B <= 0 || h_out <= 0 || n_shards <= 0 || h_out % 8) return TP_ERR_SHAPE;
+  if (!al16(partials) || !al16(Y) || (bias && !al16(bias)) || (residual && !al16(residual)))
+    return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_REDUCE, as_stream(stream));
+  return tpk::launch_reduce(partials, n_shards, B, h_out, bias, residual, Y, as_stream(stream),
+                            d.num_sms) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_reduce_partials_layernorm(const float* partials, int n_shards, int64_t B,
+                                       int64_t h_out, const uint16_t* bias,
+                                       const uint16_t* residual, const uint16_t* gamma,
+                                       const uint16_t* beta, float eps, uint16_t* Y_sum,
+                                       uint16_t* Y_ln, void* stream) {
+  if (partials == nullptr || gamma == nullptr || beta == nullptr || Y_sum == nullptr ||
+      Y_ln == nullptr)
+    return TP_ERR_NULL;
+  if (B <= 0 || h_out <= 0 || n_shards <= 0 || h_out % 8 || h_out > 16384 || B > kIntMax)
+    return TP_ERR_SHAPE;
+  if (!(eps >= 0.f)) return TP_ERR_SHAPE;
+  if (!al16(partials) || !al16(gamma) || !al16(beta) || !al16(Y_sum) || !al16(Y_ln) ||
+      (bias && !al16(bias)) || (residual && !al16(residual)))
+    return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_REDUCE_LN, as_stream(stream));
+  return tpk::launch_rows_sum_ln(partials, n_shards, B, h_out, bias, residual, gamma, beta, eps,
+                                 Y_sum, Y_ln, as_stream(stream)) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_layernorm(const uint16_t* X, int64_t B, int64_t h, const uint16_t* gamma,
+                       const uint16_t* beta, float eps, uint16_t* Y, void* stream) {
+  if (X == nullptr || gamma == nullptr || beta == nullptr || Y == nullptr) return TP_ERR_NULL;
+  if (B <= 0 || h <= 0 || h % 8 || h > 16384 || B > kIntMax) return TP_ERR_SHAPE;
+  if (!(eps >= 0.f)) return TP_ERR_SHAPE;
+  if (!al16(X) || !al16(gamma) || !al16(beta) || !al16(Y)) return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_LAYERNORM, as_stream(stream));
+  return tpk::launch_rows_sum_ln(nullptr, 0, B, h, nullptr, X, gamma, beta, eps, nullptr, Y,
+                                 as_stream(stream)) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_attention(const uint16_t* QKV_shards, int64_t batch, int64_t seq, int64_t h,
+                       int64_t n_heads, int causal, int n_shards, uint16_t* O_shards,
+                       void* stream) {
+  if (QKV_shards == nullptr || O_shards == nullptr) return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || n_heads <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (h % n_heads || n_heads % n_shards) return TP_ERR_SHAPE;
+  if (h / n_heads != 128) return TP_ERR_UNSUPPORTED;
+  if (batch * seq > kIntMax || seq > kIntMax) return TP_ERR_SHAPE;
+  if (static_cast<int64_t>(n_shards) * batch * (n_heads / n_shards) > 65535) return TP_ERR_SHAPE;
+  if (!al16(QKV_shards) || !al16(O_shards)) return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
+  return tpk::launch_attention(QKV_shards, batch, seq, h, n_heads, n_shards, causal ? 1 : 0,
+                               O_shards, as_stream(stream), d.err) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int n_shards) {
+  if (tokens <= 0 || h <= 0 || n_shards <= 0) return 0;
+  const size_t M = static_cast<size_t>(tokens), H = static_cast<size_t>(h);
+  const size_t N = static_cast<size_t>(n_shards);
+  const size_t partials = round256(N * M * H * 4);
+  if (kind == TP_WS_MLP) {
+    if (ffn <= 0) return 0;
+    return round256(M * static_cast<size_t>(ffn) * 2) + partials;
+  }
+  if (kind == TP_WS_ATTN) {
+    return round256(M * 3 * H * 2) + round256(M * H * 2) + partials;
+  }
+  if (kind == TP_WS_LAYER) {
+    if (ffn <= 0) return 0;
+    return 3 * round256(M * H * 2) + round256(M * 3 * H * 2) + round256(M * H * 2) +
+           round256(M * static_cast<size_t>(ffn) * 2) + partials;
+  }
+  return 0;
+}
+
+tp_status tp_mlp_forward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, int n_shards,
+                         const uint16_t* A_shards, const uint16_t* b1_shards,
+                         const uint16_t* B_shards, const uint16_t* b2, const uint16_t* residual,
+                         void* ws, size_t ws_bytes, uint16_t* Y, void* stream) {
+  if (X == nullptr || A_shards == nullptr || B_shards == nullptr || Y == nullptr || ws == nullptr)
+    return TP_ERR_NULL;
+  if (B <= 0 || h <= 0 || ffn <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (ffn % n_shards || (ffn / n_shards) % 8 || h % 8) return TP_ERR_SHAPE;
+  const size_t need = tp_workspace_bytes(TP_WS_MLP, B, h, ffn, n_shards);
+  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  if (!al16(ws)) return TP_ERR_ALIGN;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* act = reinterpret_cast<uint16_t*>(w);
+  float* part = reinterpret_cast<float*>(w + round256(static_cast<size_t>(B) * ffn * 2));
+  tp_status st = tp_column_linear(X, B, h, A_shards, b1_shards, ffn, n_shards, TP_ACT_GELU_ERF,
+                                  act, stream);
+  if (st != TP_OK) return st;
+  st = tp_row_linear(act, B, ffn, B_shards, h, n_shards, part, stream);
+  if (st != TP_OK) return st;
+  return tp_reduce_partials(part, n_shards, B, h, b2, residual, Y, stream);
+}
+
+tp_status tp_attn_forward(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
+                          int64_t n_heads, int causal, int n_shards, const uint16_t* Wqkv_shards,
+                          const uint16_t* bqkv_shards, const uint16_t* Wo_shards,
+                          const uint16_t* bo, const uint16_t* residual, void* ws,
+                          size_t ws_bytes, uint16_t* Y, void* stream) {
+  if (X == nullptr || Wqkv_shards == nullptr || Wo_shards == nullptr || Y == nullptr ||
+      ws == nullptr)
+    return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || n_heads <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (h % n_heads || n_heads % n_shards) return TP_ERR_SHAPE;
+  if (h / n_heads != 128) return TP_ERR_UNSUPPORTED;
+  const int64_t M = batch * seq;
+  const size_t need = tp_workspace_bytes(TP_WS_ATTN, M, h, 0, n_shards);
+  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  if (!al16(ws)) return TP_ERR_ALIGN;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* qkv = reinterpret_cast<uint16_t*>(w);
+  w += round256(static_cast<size_t>(M) * 3 * h * 2);
+  uint16_t* o = reinterpret_cast<uint16_t*>(w);
+  w += round256(static_cast<size_t>(M) * h * 2);
+  float* part = reinterpret_cast<float*>(w);
+  tp_status st = tp_column_linear(X, M, h, Wqkv_shards, bqkv_shards, 3 * h, n_shards,
+                                  TP_ACT_NONE, qkv, stream);
+  if (st != TP_OK) return st;
+  st = tp_attention(qkv, batch, seq, h, n_heads, causal, n_shards, o, stream);
+  if (st != TP_OK) return st;
+  st = tp_row_linear(o, M, h, Wo_shards, h, n_shards, part, stream);
+  if (st != TP_OK) return st;
+  return tp_reduce_partials(part, n_shards, M, h, bo, residual, Y, stream);
+}
+
+tp_status tp_layer_forward(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
+                           int64_t n_heads, int64_t ffn, int n_shards, const tp_layer_weights* w,
+                           float ln_eps, void* ws, size_t ws_bytes, uint16_t* Y, void* stream) {
+  if (X == nullptr || w == nullptr || Y == nullptr || ws == nullptr) return TP_ERR_NULL;
+  if (w->ln1_gamma == nullptr || w->ln1_beta == nullptr || w->Wqkv_shards == nullptr ||
+      w->Wo_shards == nullptr || w->ln2_gamma == nullptr || w->ln2_beta == nullptr ||
+      w->A_shards == nullptr || w->B_shards == nullptr)
+    return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || n_heads <= 0 || ffn <= 0 || n_shards <= 0)
+    return TP_ERR_SHAPE;
+  if (h % n_heads || n_heads % n_shards || ffn % n_shards || (ffn / n_shards) % 8 || h % 8 ||
+      h > 16384)
+    return TP_ERR_SHAPE;
+  if (h / n_heads != 128) return TP_ERR_UNSUPPORTED;
+  const int64_t M = batch * seq;
+  const size_t need = tp_workspace_bytes(TP_WS_LAYER, M, h, ffn, n_shards);
+  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  if (!al16(ws)) return TP_ERR_ALIGN;
+  const size_t act_b = round256(static_cast<size_t>(M) * h * 2);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  uint16_t* x1 = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* h1 = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* x2 = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* qkv = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * 3 * h * 2);
+  uint16_t* o = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* a = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * ffn * 2);
+  float* part = reinterpret_cast<float*>(p);
+
+  tp_status st = tp_layernorm(X, M, h, w->ln1_gamma, w->ln1_beta, ln_eps, x1, stream);
+  if (st != TP_OK) return st;
+  st = tp_column_linear(x1, M, h, w->Wqkv_shards, w->bqkv_shards, 3 * h, n_shards, TP_ACT_NONE,
+                        qkv, stream);
+  if (st != TP_OK) return st;
+  st = tp_attention(qkv, batch, seq, h, n_heads, 1, n_shards, o, stream);
+  if (st != TP_OK) return st;
+  st = tp_row_linear(o, M, h, w->Wo_shards, h, n_shards, part, stream);
+  if (st != TP_OK) return st;
+  st = tp_reduce_partials_layernorm(part, n_shards, M, h, w->bo, X, w->ln2_gamma, w->ln2_beta,
+                                    ln_eps, h1, x2, stream);
+  if (st != TP_OK) return st;
+  st = tp_column_linear(x2, M, h, w->A_shards, w->b1_shards, ffn, n_shards, TP_ACT_GELU_ERF, a,
+                        stream);
+  if (st != TP_OK) return st;
+  st = tp_row_linear(a, M, ffn, w->B_shards, h, n_shards, part, stream);
+  if (st != TP_OK) return st;
+  return tp_reduce_partials(part, n_shards, M, h, w->b2, h1, Y, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// Host-side interface between the C-ABI layer (tp_api.cu) and the kernel
+// translation units. Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tpk {
+
+enum KernelId {
+  KID_SHARD = 0,
+  KID_GEMM_COLUMN = 1,
+  KID_GEMM_ROW = 2,
+  KID_REDUCE = 3,
+  KID_REDUCE_LN = 4,
+  KID_LAYERNORM = 5,
+  KID_ATTENTION = 6,
+  KID_COUNT = 7
+};
+
+// One batched GEMM over G shards: D[g] (M x Nc) = A[g] (M x K) . B[g]^T with
+// A [G_A][M][K] (G_A = G when a_batched, else 1: the replicated input) and
+// B [G][Nc][K], both K-major bf16. D [G][M][Nc] is either bf16 with an
+// optional bias [G][Nc] and activation, or fp32 (no bias, no activation).
+struct GemmProblem {
+  const void* A;
+  const void* B;
+  void* D;
+  const void* bias;
+  int M, Nc, K, G;
+  bool a_batched;
+  bool out_f32;
+  int act;  // 0 none, 1 GeLU (erf form)
+};
+
+// Returns 0 on success, 1 if a tensor map could not be encoded, 2 if the
+// launch failed (cudaGetLastError()).
+int launch_gemm(const GemmProblem& p, cudaStream_t s, unsigned* err, int num_sms);
+
+// Y = sum_{i<N} P_i + bias + residual (bf16 out). n_elems % 8 == 0, h % 8 == 0.
+int launch_reduce(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
+                  const void* residual, void* Y, cudaStream_t s, int num_sms);
+
+// Per row: S = bf16(sum_i P_i + bias + residual) -> Y_sum (if non-null);
+// Y_ln = LN(S) with gamma, beta, eps (if non-null). n_shards may be 0
+// (then S = residual, i.e. a plain LayerNorm of `residual`). h % 8 == 0,
+// h <= 16384.
+int launch_rows_sum_ln(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
+                       const void* residual, const void* gamma, const void* beta, float eps,
+                       void* Y_sum, void* Y_ln, cudaStream_t s);
+
+// Causal / full attention of every shard's heads, head_dim 128.
+int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t h, int64_t n_heads,
+                     int n_shards, int causal, void* O, cudaStream_t s, unsigned* err);
+
+// out[i][c][r] = W[row(i, r)][col(i, c)] for the three split kinds.
+int launch_shard(const void* W, int64_t h_in, int64_t h_out, int n_shards, int kind,
+                 int64_t head_dim, void* out, cudaStream_t s);
+
+}  // namespace tpk

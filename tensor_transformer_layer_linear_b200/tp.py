@@ -1,0 +1,221 @@
+"""Thin ctypes binding of libtp.so (the C ABI declared in include/tp.h).
+
+Argument marshalling only: tensors are passed as raw device pointers
+(``data_ptr()``), the stream as the raw ``cudaStream_t`` of torch's current
+stream unless one is given. Every step of the computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and importing
+this module fails loudly if the library has not been built.
+
+Function names are those of the C ABI. bf16 tensors may be given as
+``torch.bfloat16`` or ``torch.int16`` (bit patterns); fp32 partials as
+``torch.float32``. All tensors must be contiguous CUDA tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtp.so")
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "tp.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with "
+        "`python -m tensor_transformer_layer_linear_b200.build` (nvcc, sm_100a)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+# status codes and enums (include/tp.h)
+TP_OK, TP_ERR_NULL, TP_ERR_SHAPE, TP_ERR_ALIGN = 0, 1, 2, 3
+TP_ERR_WORKSPACE, TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_TIMEOUT = 4, 5, 6, 7
+TP_SPLIT_COLUMN, TP_SPLIT_ROW, TP_SPLIT_QKV_HEADS = 0, 1, 2
+TP_ACT_NONE, TP_ACT_GELU_ERF = 0, 1
+TP_WS_MLP, TP_WS_ATTN, TP_WS_LAYER = 0, 1, 2
+
+_vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+
+class tp_layer_weights(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in (
+        "ln1_gamma", "ln1_beta", "Wqkv_shards", "bqkv_shards", "Wo_shards", "bo",
+        "ln2_gamma", "ln2_beta", "A_shards", "b1_shards", "B_shards", "b2")]
+
+
+_SIGS = {
+    "tp_shard_weights": (_i32, [_vp, _i64, _i64, _i32, _i32, _i64, _vp, _vp]),
+    "tp_shard_index_map": (_i32, [_i32, _i64, _i64, _i32, _i64, _vp, _vp]),
+    "tp_column_linear": (_i32, [_vp, _i64, _i64, _vp, _vp, _i64, _i32, _i32, _vp, _vp]),
+    "tp_row_linear": (_i32, [_vp, _i64, _i64, _vp, _i64, _i32, _vp, _vp]),
+    "tp_reduce_partials": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "tp_reduce_partials_layernorm": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp, _f32,
+                                            _vp, _vp, _vp]),
+    "tp_layernorm": (_i32, [_vp, _i64, _i64, _vp, _vp, _f32, _vp, _vp]),
+    "tp_attention": (_i32, [_vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp]),
+    "tp_mlp_forward": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                              _vp, _vp]),
+    "tp_attn_forward": (_i32, [_vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp,
+                               _vp, _sz, _vp, _vp]),
+    "tp_layer_forward": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32,
+                                ctypes.POINTER(tp_layer_weights), _f32, _vp, _sz, _vp, _vp]),
+    "tp_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
+    "tp_get_last_error": (_i32, [_vp]),
+    "tp_status_string": (ctypes.c_char_p, [_i32]),
+    "tp_trace_begin": (_i32, [_i32]),
+    "tp_trace_end": (_i32, []),
+    "tp_trace_record": (_i32, [_i32, ctypes.POINTER(_i32), ctypes.POINTER(_f32)]),
+    "tp_kernel_name": (ctypes.c_char_p, [_i32]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+def header_functions() -> list:
+    """Names of every function include/tp.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(tp_[a-z_0-9]+)\s*\(",
+                                 text, flags=re.M)))
+
+
+class TPError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.tp_status_string(status).decode()}")
+
+
+def _check(st: int, where: str) -> None:
+    if st != TP_OK:
+        raise TPError(st, where)
+
+
+def _p(t) -> int:
+    """Raw pointer of a tensor (None -> NULL; ints pass through)."""
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    if t.device.type != "cuda":
+        raise ValueError("tensor must be on a CUDA device")
+    return t.data_ptr()
+
+
+def _s(stream) -> int:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def tp_status_string(status: int) -> str:
+    return lib.tp_status_string(status).decode()
+
+
+def tp_workspace_bytes(kind: int, tokens: int, h: int, ffn: int, n_shards: int) -> int:
+    return int(lib.tp_workspace_bytes(kind, tokens, h, ffn, n_shards))
+
+
+def tp_shard_index_map(kind: int, h_in: int, h_out: int, n_shards: int, head_dim: int = 0):
+    """Host-only index map -> (owner int32 array, local int64 array)."""
+    import numpy as np
+    n = h_in if kind == TP_SPLIT_ROW else h_out
+    owner = np.zeros(n, dtype=np.int32)
+    local = np.zeros(n, dtype=np.int64)
+    _check(lib.tp_shard_index_map(kind, h_in, h_out, n_shards, head_dim,
+                                  owner.ctypes.data, local.ctypes.data), "tp_shard_index_map")
+    return owner, local
+
+
+def tp_shard_weights(W, h_in, h_out, n_shards, kind, head_dim, W_shards, stream=None):
+    _check(lib.tp_shard_weights(_p(W), h_in, h_out, n_shards, kind, head_dim, _p(W_shards),
+                                _s(stream)), "tp_shard_weights")
+
+
+def tp_column_linear(X, B, h_in, W_shards, bias_shards, h_out, n_shards, act, Y_shards,
+                     stream=None):
+    _check(lib.tp_column_linear(_p(X), B, h_in, _p(W_shards), _p(bias_shards), h_out, n_shards,
+                                act, _p(Y_shards), _s(stream)), "tp_column_linear")
+
+
+def tp_row_linear(X_shards, B, h_in, W_shards, h_out, n_shards, partials, stream=None):
+    _check(lib.tp_row_linear(_p(X_shards), B, h_in, _p(W_shards), h_out, n_shards, _p(partials),
+                             _s(stream)), "tp_row_linear")
+
+
+def tp_reduce_partials(partials, n_shards, B, h_out, bias, residual, Y, stream=None):
+    _check(lib.tp_reduce_partials(_p(partials), n_shards, B, h_out, _p(bias), _p(residual), _p(Y),
+                                  _s(stream)), "tp_reduce_partials")
+
+
+def tp_reduce_partials_layernorm(partials, n_shards, B, h_out, bias, residual, gamma, beta, eps,
+                                 Y_sum, Y_ln, stream=None):
+    _check(lib.tp_reduce_partials_layernorm(_p(partials), n_shards, B, h_out, _p(bias),
+                                            _p(residual), _p(gamma), _p(beta), eps, _p(Y_sum),
+                                            _p(Y_ln), _s(stream)),
+           "tp_reduce_partials_layernorm")
+
+
+def tp_layernorm(X, B, h, gamma, beta, eps, Y, stream=None):
+    _check(lib.tp_layernorm(_p(X), B, h, _p(gamma), _p(beta), eps, _p(Y), _s(stream)),
+           "tp_layernorm")
+
+
+def tp_attention(QKV_shards, batch, seq, h, n_heads, causal, n_shards, O_shards, stream=None):
+    _check(lib.tp_attention(_p(QKV_shards), batch, seq, h, n_heads, int(bool(causal)), n_shards,
+                            _p(O_shards), _s(stream)), "tp_attention")
+
+
+def tp_mlp_forward(X, B, h, ffn, n_shards, A_shards, b1_shards, B_shards, b2, residual, ws,
+                   ws_bytes, Y, stream=None):
+    _check(lib.tp_mlp_forward(_p(X), B, h, ffn, n_shards, _p(A_shards), _p(b1_shards),
+                              _p(B_shards), _p(b2), _p(residual), _p(ws), ws_bytes, _p(Y),
+                              _s(stream)), "tp_mlp_forward")
+
+
+def tp_attn_forward(X, batch, seq, h, n_heads, causal, n_shards, Wqkv_shards, bqkv_shards,
+                    Wo_shards, bo, residual, ws, ws_bytes, Y, stream=None):
+    _check(lib.tp_attn_forward(_p(X), batch, seq, h, n_heads, int(bool(causal)), n_shards,
+                               _p(Wqkv_shards), _p(bqkv_shards), _p(Wo_shards), _p(bo),
+                               _p(residual), _p(ws), ws_bytes, _p(Y), _s(stream)),
+           "tp_attn_forward")
+
+
+def make_layer_weights(**tensors) -> tp_layer_weights:
+    """Build the tp_layer_weights struct from tensors named like its fields."""
+    w = tp_layer_weights()
+    for name, _ in tp_layer_weights._fields_:
+        setattr(w, name, _p(tensors.get(name)))
+    return w
+
+
+def tp_layer_forward(X, batch, seq, h, n_heads, ffn, n_shards, weights: tp_layer_weights,
+                     ln_eps, ws, ws_bytes, Y, stream=None):
+    _check(lib.tp_layer_forward(_p(X), batch, seq, h, n_heads, ffn, n_shards,
+                                ctypes.byref(weights), ln_eps, _p(ws), ws_bytes, _p(Y),
+                                _s(stream)), "tp_layer_forward")
+
+
+def tp_get_last_error(stream=None) -> int:
+    return int(lib.tp_get_last_error(_s(stream)))
+
+
+def tp_trace_begin(max_records: int) -> None:
+    _check(lib.tp_trace_begin(max_records), "tp_trace_begin")
+
+
+def tp_trace_end() -> list:
+    """Stop the trace; return [(kernel_name, ms), ...] for the timed launches
+    and, as a second value, the number of launches seen."""
+    seen = lib.tp_trace_end()
+    recs = []
+    k = 0
+    while True:
+        kid, ms = _i32(), _f32()
+        if lib.tp_trace_record(k, ctypes.byref(kid), ctypes.byref(ms)) != TP_OK:
+            break
+        recs.append((lib.tp_kernel_name(kid.value).decode(), float(ms.value)))
+        k += 1
+    return recs, int(seen)

@@ -1,0 +1,38 @@
+"""Shared test helpers: bf16 bit arrays <-> torch tensors, the parity gate."""
+import numpy as np
+
+from tensor_transformer_layer_linear_b200 import synth
+
+# Value tolerance of the parity gate: max|gpu - oracle| <= MAX_REL * max|oracle|
+# and ||gpu - oracle||_F / ||oracle||_F <= FRO_REL.
+MAX_REL = 2e-2
+FRO_REL = 5e-3
+
+
+def to_dev(bits: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda()
+
+
+def from_dev_bf16(t) -> np.ndarray:
+    """Device bf16 (int16 bits) -> float64 numpy."""
+    return synth.bf16_bits_to_f64(t.cpu().numpy().view(np.uint16))
+
+
+def f64(bits: np.ndarray) -> np.ndarray:
+    return synth.bf16_bits_to_f64(bits)
+
+
+def assert_parity(gpu: np.ndarray, ref: np.ndarray, what: str = "",
+                  max_rel: float = MAX_REL, fro_rel: float = FRO_REL) -> dict:
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite values"
+    err = np.abs(gpu - ref)
+    scale = np.max(np.abs(ref))
+    fro = np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-300)
+    stats = dict(max_abs=float(err.max()), max_ref=float(scale), fro_rel=float(fro))
+    assert err.max() <= max_rel * scale, f"{what}: max error {stats}"
+    assert fro <= fro_rel, f"{what}: Frobenius error {stats}"
+    return stats
