@@ -230,6 +230,35 @@ tp_status tp_layer_forward(const uint16_t* X, int64_t batch, int64_t seq,
                            float ln_eps, void* ws, size_t ws_bytes,
                            uint16_t* Y, void* stream);
 
+/* Size in bytes of the library-owned scratch array used by
+ * tp_mlp_forward_noalloc (32 MiB, reserved on every GPU that loads the
+ * library, until the process exits). */
+#define TP_NOALLOC_WS_BYTES (32u * 1024u * 1024u)
+
+/* tp_mlp_forward_noalloc - tp_mlp_forward for callers that cannot allocate
+ * device memory: the same arguments and result, but without the workspace
+ * pair; the intermediates live in a fixed library-owned device array of
+ * TP_NOALLOC_WS_BYTES. The pages have no counterpart to this call: it exists
+ * for callers that have no device allocator to hand (a C program embedding
+ * the library without a memory pool) or whose framework has already reserved
+ * all device memory, so they cannot ask for a workspace.
+ * - Rejects, with TP_ERR_WORKSPACE and before any launch, a problem whose
+ *   tp_workspace_bytes(TP_WS_MLP, B, h, ffn, N) exceeds TP_NOALLOC_WS_BYTES.
+ * - All calls on a device share the array; it keeps the last call's contents
+ *   (no part of it needs to start at zero). Calls that overlap on the GPU
+ *   (unordered streams or host threads) race on it: the caller must order
+ *   them.
+ * - The first call on a device looks up and caches the array's device
+ *   address; make it before any stream capture begins.
+ * - Calls no cudaMalloc, cudaFree or other allocating routine. */
+tp_status tp_mlp_forward_noalloc(const uint16_t* X, int64_t B, int64_t h,
+                                 int64_t ffn, int n_shards,
+                                 const uint16_t* A_shards,
+                                 const uint16_t* b1_shards,
+                                 const uint16_t* B_shards, const uint16_t* b2,
+                                 const uint16_t* residual, uint16_t* Y,
+                                 void* stream);
+
 /* Workspace bytes for tp_mlp_forward (kind TP_WS_MLP), tp_attn_forward
  * (TP_WS_ATTN, ffn ignored) or tp_layer_forward (TP_WS_LAYER). tokens =
  * batch * seq. Returns 0 for invalid arguments. */

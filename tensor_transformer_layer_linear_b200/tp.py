@@ -58,6 +58,8 @@ _SIGS = {
                                _vp, _sz, _vp, _vp]),
     "tp_layer_forward": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32,
                                 ctypes.POINTER(tp_layer_weights), _f32, _vp, _sz, _vp, _vp]),
+    "tp_mlp_forward_noalloc": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      _vp]),
     "tp_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "tp_get_last_error": (_i32, [_vp]),
     "tp_status_string": (ctypes.c_char_p, [_i32]),
@@ -173,6 +175,20 @@ def tp_mlp_forward(X, B, h, ffn, n_shards, A_shards, b1_shards, B_shards, b2, re
     _check(lib.tp_mlp_forward(_p(X), B, h, ffn, n_shards, _p(A_shards), _p(b1_shards),
                               _p(B_shards), _p(b2), _p(residual), _p(ws), ws_bytes, _p(Y),
                               _s(stream)), "tp_mlp_forward")
+
+
+TP_NOALLOC_WS_BYTES = 32 * 1024 * 1024
+
+
+def tp_mlp_forward_noalloc(X, B, h, ffn, n_shards, A_shards, b1_shards, B_shards, b2, residual,
+                           Y, stream=None):
+    """tp_mlp_forward without a workspace argument, for callers that cannot
+    allocate device memory: the intermediates live in the library's fixed
+    TP_NOALLOC_WS_BYTES device array (shared by all calls on a device; calls
+    that overlap on the GPU race on it)."""
+    _check(lib.tp_mlp_forward_noalloc(_p(X), B, h, ffn, n_shards, _p(A_shards), _p(b1_shards),
+                                      _p(B_shards), _p(b2), _p(residual), _p(Y), _s(stream)),
+           "tp_mlp_forward_noalloc")
 
 
 def tp_attn_forward(X, batch, seq, h, n_heads, causal, n_shards, Wqkv_shards, bqkv_shards,
