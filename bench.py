@@ -99,7 +99,7 @@ def work(cfg: dict) -> dict:
 # clocks during the timed region
 # --------------------------------------------------------------------------
 
-CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+CLOCK_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -114,12 +114,14 @@ class ClockSampler:
             gid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", gid, f"--query-gpu={CLOCK_FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
 
-    def stop(self) -> dict:
+    def stop(self, t0: float = None, t1: float = None) -> dict:
+        """Median SM clock and the throttle reasons seen in samples taken
+        between host wall-clock times t0 and t1 (all samples if none are)."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -128,23 +130,28 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             text, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
+        import datetime
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        samples = []
         for line in text.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                samples.append((ts, float(f[2]), float(f[3]), float(f[4]) if f[4] else 0.0,
+                                [nm for nm, v in zip(names, f[6:10]) if v.lower() == "active"]))
             except ValueError:
                 continue
-            for nm, val in zip(names, f[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
+        inside = [x for x in samples if t0 is not None and t0 <= x[0] <= t1]
+        use = inside or samples
+        sm = [x[1] for x in use]
+        reasons = sorted({r for x in use for r in x[4]})
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "sm_max_mhz": max(x[2] for x in use) if use else None,
+                "power_w_max": max(x[3] for x in use) if use else None,
+                "reasons": reasons, "samples": len(use),
+                "window": "timed region" if inside else "whole run"}
 
 
 # --------------------------------------------------------------------------
@@ -312,13 +319,15 @@ def run_ours(args, cfg) -> None:
     ev1 = torch.cuda.Event(enable_timing=True)
     tp.tp_trace_begin(64 * args.steps)
     barrier()
+    t_wall0 = time.time()
     ev0.record(stream)
     for _ in range(args.steps):
         model.step()
     ev1.record(stream)
     barrier()
+    t_wall1 = time.time()
     recs, launches = tp.tp_trace_end()
-    clocks = sampler.stop()
+    clocks = sampler.stop(t_wall0, t_wall1)
     ms = ev0.elapsed_time(ev1) / args.steps
     st = tp.tp_get_last_error()
     if st != tp.TP_OK:
@@ -429,7 +438,7 @@ def run_ours(args, cfg) -> None:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.CONFIGS))

@@ -38,8 +38,12 @@ struct GemmCfg {
   static constexpr int kBBytes = BN * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
+  // epilogue staging: 4 warps x 2 buffers x (32 rows x 128 bytes)
+  static constexpr int kStagingBytes = 4 * 2 * 4096;
   static constexpr int kNumBars = 2 * kStages + 5;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kNumBars * 8 + 16;
+  static constexpr int kSmemBytes =
+      1024 + kStages * kStageBytes + kStagingBytes + kNumBars * 8 + 16;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 struct GemmParams {
@@ -55,12 +59,14 @@ struct GemmParams {
 template <int BN, bool OUT_F32>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* tiles = smem_raw + pad;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(tiles + C::kStages * C::kStageBytes);
+  uint8_t* staging = tiles + C::kStages * C::kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + C::kStagingBytes);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -90,6 +96,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmD);
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
   tc_fence_before();
@@ -189,9 +196,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lanes [32 q, 32 q + 32) are this warp's
+    // Each warp owns TMEM lanes [32 q, 32 q + 32) = 32 output rows. Per chunk
+    // of columns (32 fp32 or 64 bf16 = 128 bytes per row) every thread
+    // writes its row into a 128-byte-swizzled staging buffer, then one lane
+    // issues a TMA tensor store of the 32-row box (rows/columns outside the
+    // output are clipped by the TMA unit). Two staging buffers per warp let
+    // the next chunk be written while the previous store drains.
+    const int q = warp & 3;
+    const uint32_t stage_base = smem_u32(staging) + static_cast<uint32_t>((warp - 2) * 2 * 4096);
+    constexpr int CW = OUT_F32 ? 32 : 64;  // columns per chunk
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t chunk_ctr = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int mb = tile % p.num_m;
@@ -203,61 +219,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row = mb * BM + q * 32 + lane;
-      const bool row_ok = row < p.M;
+      const int row0 = mb * BM + q * 32;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      const int64_t out_row = (static_cast<int64_t>(g) * p.M + row) * p.Nc;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tbase + c * 32, r);
+      for (int c = 0; c < BN / CW; ++c) {
+        uint32_t r[CW];
+        tmem_ld_32x32b_x32(tbase + c * CW, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        if constexpr (!OUT_F32)
+          tmem_ld_32x32b_x32(tbase + c * CW + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_ld_wait();
-        const int col0 = nb * BN + c * 32;
-        if (row_ok && col0 < p.Nc) {
-          if constexpr (OUT_F32) {
-            float* out = static_cast<float*>(p.out) + out_row;
+        const int col0 = nb * BN + c * CW;
+        if (col0 >= p.Nc) continue;  // warp-uniform: the whole chunk is past the edge
+        uint32_t w[32];              // this thread's 128-byte row of the chunk
+        if constexpr (OUT_F32) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int col = col0 + 4 * j;
-              if (col < p.Nc) {
-                float4 v = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                       __uint_as_float(r[4 * j + 2]),
-                                       __uint_as_float(r[4 * j + 3]));
-                *reinterpret_cast<float4*>(out + col) = v;
-              }
+          for (int e = 0; e < 32; ++e) w[e] = r[e];
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * j + e]);
+            const int col = col0 + 8 * j;
+            if (p.bias != nullptr && col < p.Nc) {
+              const uint4 b = *reinterpret_cast<const uint4*>(
+                  p.bias + static_cast<int64_t>(g) * p.Nc + col);
+              v[0] += bf16_lo(b.x); v[1] += bf16_hi(b.x);
+              v[2] += bf16_lo(b.y); v[3] += bf16_hi(b.y);
+              v[4] += bf16_lo(b.z); v[5] += bf16_hi(b.z);
+              v[6] += bf16_lo(b.w); v[7] += bf16_hi(b.w);
             }
-          } else {
-            uint16_t* out = static_cast<uint16_t*>(p.out) + out_row;
+            if (p.act == 1) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int col = col0 + 8 * j;
-              if (col < p.Nc) {
-                float v[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * j + e]);
-                if (p.bias != nullptr) {
-                  const uint4 b = *reinterpret_cast<const uint4*>(
-                      p.bias + static_cast<int64_t>(g) * p.Nc + col);
-                  v[0] += bf16_lo(b.x); v[1] += bf16_hi(b.x);
-                  v[2] += bf16_lo(b.y); v[3] += bf16_hi(b.y);
-                  v[4] += bf16_lo(b.z); v[5] += bf16_hi(b.z);
-                  v[6] += bf16_lo(b.w); v[7] += bf16_hi(b.w);
-                }
-                if (p.act == 1) {
-#pragma unroll
-                  for (int e = 0; e < 8; ++e) v[e] = gelu_erf(v[e]);
-                }
-                uint4 o;
-                o.x = pack_bf16x2(v[0], v[1]);
-                o.y = pack_bf16x2(v[2], v[3]);
-                o.z = pack_bf16x2(v[4], v[5]);
-                o.w = pack_bf16x2(v[6], v[7]);
-                *reinterpret_cast<uint4*>(out + col) = o;
-              }
+              for (int e = 0; e < 8; ++e) v[e] = gelu_erf(v[e]);
             }
+            w[4 * j + 0] = pack_bf16x2(v[0], v[1]);
+            w[4 * j + 1] = pack_bf16x2(v[2], v[3]);
+            w[4 * j + 2] = pack_bf16x2(v[4], v[5]);
+            w[4 * j + 3] = pack_bf16x2(v[6], v[7]);
           }
         }
+        const uint32_t sbuf = stage_base + (chunk_ctr & 1u) * 4096u;
+        if (lane == 0) bulk_wait_read<1>();  // the store that last used sbuf has read it
+        __syncwarp();
+        const uint32_t row_addr = sbuf + static_cast<uint32_t>(lane) * 128u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4), w[4 * j],
+                       w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tmD, sbuf, col0, row0, g);
+          bulk_commit();
+        }
+        ++chunk_ctr;
       }
       tc_fence_before();
       __syncwarp();
@@ -267,6 +284,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    if (lane == 0) bulk_wait<0>();  // every store of this warp has completed
     if (!ok) {
       if (lane == 0) atomicOr(p.err, ERR_WAIT_EPILOGUE);
       *abort_flag = 1;
@@ -297,17 +315,19 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [d2][d1][d0] bf16 tensor, boxes of box0 x box1 x 1 with the 128-byte swizzle;
-// out-of-range elements read as zero.
+// [d2][d1][d0] tensor (bf16 or fp32), boxes of box0 x box1 x 1 with the
+// 128-byte swizzle; loads read out-of-range elements as zero, stores skip them.
 static bool encode_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                      uint32_t box0, uint32_t box1) {
+                      uint32_t box0, uint32_t box1, bool f32 = false) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return false;
+  const uint64_t es = f32 ? 4 : 2;
   cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint64_t strides[2] = {d0 * es, d0 * d1 * es};
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+  CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -316,9 +336,10 @@ static bool encode_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1
 template <int BN, bool OUT_F32>
 static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, int num_sms) {
   using C = GemmCfg<BN>;
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmD;
   if (!encode_3d(&tmA, pr.A, pr.K, pr.M, pr.a_batched ? pr.G : 1, BK, BM)) return 1;
   if (!encode_3d(&tmB, pr.B, pr.K, pr.Nc, pr.G, BK, BN)) return 1;
+  if (!encode_3d(&tmD, pr.D, pr.Nc, pr.M, pr.G, OUT_F32 ? 32 : 64, 32, OUT_F32)) return 1;
   GemmParams p;
   p.M = pr.M;
   p.Nc = pr.Nc;
@@ -336,7 +357,7 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
   auto kern = gemm_tcgen05_kernel<BN, OUT_F32>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  kern<<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmA, tmB, p);
+  kern<<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmA, tmB, tmD, p);
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
 
