@@ -7,17 +7,27 @@
 //
 //   warp 0      TMA producer: 128-byte-swizzled A and B tiles (BK = 64) into
 //               a ring of shared-memory stages, completion on mbarriers.
-//   warp 1      owns TMEM (two BM x BN fp32 accumulators) and one thread
-//               issues tcgen05.mma (M = 128, N = BN, K = 16) per stage,
-//               releasing the stage with tcgen05.commit.
+//   warp 1      owns TMEM (two fp32 accumulators of BN columns); one thread
+//               issues tcgen05.mma per stage and releases the stage with
+//               tcgen05.commit.
 //   warps 2-5   epilogue: tcgen05.ld of the finished accumulator, then the
 //               column-parallel bias + GeLU (bf16 out) or the row-parallel
-//               fp32 partial store, overlapping the next tile's mainloop.
+//               fp32 partials, staged in swizzled shared memory and written
+//               with TMA tensor stores, overlapping the next tile's
+//               mainloop.
 //
-// Tiles are (shard g, m-block, n-block), m fastest, strided over the
-// CTAs. Every barrier wait is bounded; on expiry the CTA records an error
+// CTAS = 1: one CTA per tile of 128 x BN (tcgen05 cta_group::1).
+// CTAS = 2: a cluster of two CTAs per tile of 256 x 256 (cta_group::2). Each
+// CTA loads its own 128 rows of A and its own 128 rows of B^T (half of the
+// tile's columns) with plain (non-multicast) TMA; the leader CTA issues the
+// M = 256 MMAs, which read both CTAs' shared memory and write each CTA's 128
+// rows of D into that CTA's TMEM. Per SM this halves the B panel traffic
+// from L2 and lets 6 pipeline stages fit beside the epilogue staging.
+//
+// Tiles are (shard g, m-block, n-block), m fastest, strided over the CTAs
+// (pairs). Every barrier wait is bounded; on expiry the CTA records an error
 // bit, stops all roles, waits for its own copies and MMAs in flight, frees
-// TMEM and returns.
+// TMEM and returns through the same exit path.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -27,16 +37,18 @@
 
 namespace tpk {
 
-constexpr int BM = 128;
+constexpr int BM = 128;            // accumulator rows per CTA (TMEM lanes)
 constexpr int BK = 64;             // 64 bf16 = 128 bytes = one swizzle row
 constexpr int kGemmThreads = 192;  // 6 warps
 
-template <int BN>
+template <int BN, int CTAS>
 struct GemmCfg {
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kTileM = BM * CTAS;       // rows of a tile
+  static constexpr int kBRows = BN / CTAS;       // B^T rows held per CTA
   static constexpr int kABytes = BM * BK * 2;
-  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kBBytes = kBRows * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (CTAS == 2) ? 6 : ((BN == 256) ? 4 : 6);
   static constexpr int kTmemCols = 2 * BN;
   // epilogue staging: 4 warps x 2 buffers x (32 rows x 128 bytes)
   static constexpr int kStagingBytes = 4 * 2 * 4096;
@@ -44,6 +56,7 @@ struct GemmCfg {
   static constexpr int kSmemBytes =
       1024 + kStages * kStageBytes + kStagingBytes + kNumBars * 8 + 16;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(CTAS == 1 || BN == 256, "pairs use 256 x 256 tiles");
 };
 
 struct GemmParams {
@@ -51,17 +64,16 @@ struct GemmParams {
   int num_m, num_n, num_k, num_tiles;
   int a_batched;
   int act;
-  void* out;
   const uint16_t* bias;
   unsigned* err;
 };
 
-template <int BN, bool OUT_F32>
+template <int BN, bool OUT_F32, int CTAS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, CTAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* tiles = smem_raw + pad;
@@ -79,6 +91,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = (CTAS == 2) ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int first_tile = blockIdx.x / CTAS;
+  const int tile_step = gridDim.x / CTAS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -87,7 +103,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 4);  // one arrival per epilogue warp
+      mbar_init(tempty_bar(b), 4 * CTAS);  // one arrival per epilogue warp of the pair
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -98,9 +114,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmD);
   }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+  if (warp == 1) {
+    if constexpr (CTAS == 2)
+      tmem_alloc_pair(smem_u32(tmem_holder), C::kTmemCols);
+    else
+      tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+  }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CTAS == 2) cluster_sync_all();  // peer barriers initialised before use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -111,20 +133,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = first_tile; ok && tile < p.num_tiles; tile += tile_step) {
         const int mb = tile % p.num_m;
         const int rest = tile / p.num_m;
         const int nb = rest % p.num_n;
         const int g = rest / p.num_n;
+        const int arow = mb * C::kTileM + static_cast<int>(rank) * BM;
+        const int brow = nb * BN + static_cast<int>(rank) * C::kBRows;
         for (int kb = 0; kb < p.num_k; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           const uint32_t sa = smem_u32(tiles + stage * C::kStageBytes);
-          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
-          tma_load_3d(sa, &tmA, full_bar(stage), kb * BK, mb * BM, p.a_batched ? g : 0);
-          tma_load_3d(sa + C::kABytes, &tmB, full_bar(stage), kb * BK, nb * BN, g);
+          if constexpr (CTAS == 2) {
+            // both CTAs' bytes are counted on the leader's full barrier
+            const uint32_t fb = mapa_shared(full_bar(stage), 0);
+            if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * C::kStageBytes);
+            tma_load_3d_pair(sa, &tmA, fb, kb * BK, arow, p.a_batched ? g : 0);
+            tma_load_3d_pair(sa + C::kABytes, &tmB, fb, kb * BK, brow, g);
+          } else {
+            mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+            tma_load_3d(sa, &tmA, full_bar(stage), kb * BK, arow, p.a_batched ? g : 0);
+            tma_load_3d(sa + C::kABytes, &tmB, full_bar(stage), kb * BK, brow, g);
+          }
           ++issued;
           if (++stage == C::kStages) {
             stage = 0;
@@ -136,23 +168,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         atomicOr(p.err, ERR_WAIT_PRODUCER);
         *abort_flag = 1;
       }
-      // Every armed stage must have landed before the CTA may exit.
-      for (int s = 0; s < C::kStages && s < issued; ++s) {
-        const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
-        int never = 0;
-        if (!mbar_wait(full_bar(s), par, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
+      // Every armed stage must have landed before the CTA may exit (for a
+      // pair the leader's full barriers count both CTAs' bytes).
+      if (leader) {
+        for (int s = 0; s < C::kStages && s < issued; ++s) {
+          const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+          int never = 0;
+          if (!mbar_wait(full_bar(s), par, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(BM, BN);
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(C::kTileM, BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = first_tile; ok && tile < p.num_tiles; tile += tile_step) {
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -169,17 +204,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t sb = sa + C::kABytes;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            umma_bf16(d_tmem, umma_desc_sw128(sa + kk * 32), umma_desc_sw128(sb + kk * 32), idesc,
-                      (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t ad = umma_desc_sw128(sa + kk * 32);
+            const uint64_t bd = umma_desc_sw128(sb + kk * 32);
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            if constexpr (CTAS == 2)
+              umma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+            else
+              umma_bf16(d_tmem, ad, bd, idesc, accum);
           }
-          umma_commit(empty_bar(stage));
+          if constexpr (CTAS == 2)
+            umma_commit_pair_mc(empty_bar(stage), 0x3);
+          else
+            umma_commit(empty_bar(stage));
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(tfull_bar(acc));
+        if constexpr (CTAS == 2)
+          umma_commit_pair_mc(tfull_bar(acc), 0x3);
+        else
+          umma_commit(tfull_bar(acc));
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
@@ -190,7 +236,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         *abort_flag = 1;
       }
       // All MMAs issued by this thread must be complete before TMEM is freed.
-      umma_commit(drain_bar);
+      if constexpr (CTAS == 2)
+        umma_commit_pair(drain_bar);
+      else
+        umma_commit(drain_bar);
       int never = 0;
       if (!mbar_wait(drain_bar, 0, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
     }
@@ -209,7 +258,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     uint32_t chunk_ctr = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    for (int tile = first_tile; tile < p.num_tiles; tile += tile_step) {
       const int mb = tile % p.num_m;
       const int rest = tile / p.num_m;
       const int nb = rest % p.num_n;
@@ -219,7 +268,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row0 = mb * BM + q * 32;
+      const int row0 = mb * C::kTileM + static_cast<int>(rank) * BM + q * 32;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
@@ -278,7 +327,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (lane == 0) {
+        if constexpr (CTAS == 2)
+          mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));  // the leader's barrier
+        else
+          mbar_arrive(tempty_bar(acc));
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -293,9 +347,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // A pair leaves together: the leader's MMAs read the peer's shared memory
+  // and the peer's epilogue arrives on the leader's barriers.
+  if constexpr (CTAS == 2) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if constexpr (CTAS == 2)
+      tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else
+      tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -327,47 +387,77 @@ static bool encode_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                   const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool OUT_F32>
+template <int BN, bool OUT_F32, int CTAS>
 static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, int num_sms) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, CTAS>;
   CUtensorMap tmA, tmB, tmD;
   if (!encode_3d(&tmA, pr.A, pr.K, pr.M, pr.a_batched ? pr.G : 1, BK, BM)) return 1;
-  if (!encode_3d(&tmB, pr.B, pr.K, pr.Nc, pr.G, BK, BN)) return 1;
+  if (!encode_3d(&tmB, pr.B, pr.K, pr.Nc, pr.G, BK, C::kBRows)) return 1;
   if (!encode_3d(&tmD, pr.D, pr.Nc, pr.M, pr.G, OUT_F32 ? 32 : 64, 32, OUT_F32)) return 1;
   GemmParams p;
   p.M = pr.M;
   p.Nc = pr.Nc;
   p.K = pr.K;
   p.G = pr.G;
-  p.num_m = (pr.M + BM - 1) / BM;
+  p.num_m = (pr.M + C::kTileM - 1) / C::kTileM;
   p.num_n = (pr.Nc + BN - 1) / BN;
   p.num_k = (pr.K + BK - 1) / BK;
   p.num_tiles = p.num_m * p.num_n * pr.G;
   p.a_batched = pr.a_batched ? 1 : 0;
   p.act = pr.act;
-  p.out = pr.D;
   p.bias = static_cast<const uint16_t*>(pr.bias);
   p.err = err;
-  auto kern = gemm_tcgen05_kernel<BN, OUT_F32>;
+  auto kern = gemm_tcgen05_kernel<BN, OUT_F32, CTAS>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  kern<<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmA, tmB, tmD, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CTAS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // Persistent grid: as many CTAs (pairs) as can be resident at once; pairs
+  // need two free SMs of one GPC, which the occupancy query accounts for.
+  static int resident_units = 0;
+  if (resident_units == 0) {
+    int n = num_sms / CTAS;
+    if (CTAS > 1) {
+      cfg.gridDim = dim3(static_cast<unsigned>(num_sms));
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0 &&
+          clusters < n)
+        n = clusters;
+      cudaGetLastError();
+    }
+    resident_units = n;
+  }
+  const int units = p.num_tiles < resident_units ? p.num_tiles : resident_units;
+  cfg.gridDim = dim3(static_cast<unsigned>(units * CTAS));
+  if (cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, p) != cudaSuccess) return 2;
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
 
 int launch_gemm(const GemmProblem& p, cudaStream_t s, unsigned* err, int num_sms) {
   const bool wide = p.Nc > 128;
-  if (p.out_f32)
-    return wide ? launch_gemm_t<256, true>(p, s, err, num_sms)
-                : launch_gemm_t<128, true>(p, s, err, num_sms);
-  return wide ? launch_gemm_t<256, false>(p, s, err, num_sms)
-              : launch_gemm_t<128, false>(p, s, err, num_sms);
+  const bool pair = wide && p.M > BM;  // 256-row tiles only when there are rows to fill them
+  if (p.out_f32) {
+    if (pair) return launch_gemm_t<256, true, 2>(p, s, err, num_sms);
+    return wide ? launch_gemm_t<256, true, 1>(p, s, err, num_sms)
+                : launch_gemm_t<128, true, 1>(p, s, err, num_sms);
+  }
+  if (pair) return launch_gemm_t<256, false, 2>(p, s, err, num_sms);
+  return wide ? launch_gemm_t<256, false, 1>(p, s, err, num_sms)
+              : launch_gemm_t<128, false, 1>(p, s, err, num_sms);
 }
 
 }  // namespace tpk
