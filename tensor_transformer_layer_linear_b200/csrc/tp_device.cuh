@@ -215,6 +215,44 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 
+
+// Shared-memory descriptor for an MN-major operand written by TMA with the
+// 128-byte swizzle: 64-element (128-byte) rows along MN, 8-row atoms along
+// K 1024 bytes apart (stride byte offset), successive 64-element MN blocks
+// `mn_block_bytes` apart (leading byte offset).
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t mn_block_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((mn_block_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16, bf16 in, fp32 accumulate, A K-major and
+// B MN-major (bit 16).
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32_bmn(int M, int N) {
+  return umma_idesc_bf16_f32(M, N) | (1u << 16);
+}
+
+// 32 lanes x 32 fp32 columns from registers into TMEM (thread t -> lane t).
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- CTA pairs
 // Two CTAs of a cluster running one tcgen05 MMA together (cta_group::2):
 // the leader (rank 0) issues the MMAs; each CTA holds half of A (rows) and
