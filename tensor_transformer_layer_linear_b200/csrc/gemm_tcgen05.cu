@@ -274,9 +274,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < BN / CW; ++c) {
         uint32_t r[CW];
-        tmem_ld_32x32b_x32(tbase + c * CW, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld_32x32b_x32(tbase + c * CW, &r[0]);
         if constexpr (!OUT_F32)
-          tmem_ld_32x32b_x32(tbase + c * CW + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          tmem_ld_32x32b_x32(tbase + c * CW + 32, &r[32]);
         tmem_ld_wait();
         const int col0 = nb * BN + c * CW;
         if (col0 >= p.Nc) continue;  // warp-uniform: the whole chunk is past the edge
