@@ -393,6 +393,13 @@ def run_ours(args, cfg) -> None:
     roof["kernel"] = dom
     roof["peak_source"] = f"{pk['source']} (burst bf16 {pk['bf16']} TFLOP/s, HBM {pk['hbm']} GB/s)"
     kernels = {k: kernel_fig(k) for k in per}
+    # launches of one step in order, with their mean device time over the timed steps
+    per_step = len(recs) // args.steps if args.steps else 0
+    step_breakdown = []
+    if per_step and len(recs) == per_step * args.steps:
+        for pos in range(per_step):
+            times = [recs[s * per_step + pos][1] for s in range(args.steps)]
+            step_breakdown.append([recs[pos][0], round(sum(times) / len(times), 5)])
     reduce_fig = kernels.get("reduce_partials")
 
     value = w["total_flops"] * world / (ms * 1e-3) / 1e12
@@ -427,12 +434,62 @@ def run_ours(args, cfg) -> None:
         "clocks": clocks,
         "gpu_launches": launches,
         "gflop_per_step": w["total_flops"] / 1e9,
+        "step_breakdown_ms": step_breakdown,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_sweep(args, cfg) -> None:
+    """Shard-count sweep of one MLP workload (the large-MLP sweep by default):
+    the same inputs run with N = 1, 2, 4, 8, 16 shards; reports TFLOP/s per N
+    and the N-overhead t(N) / t(1) - 1 (one JSON line)."""
+    import torch
+    from tensor_transformer_layer_linear_b200 import tp
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    inp = synth.make_inputs(cfg)
+    res = {}
+    pk = peaks()
+    for n in cfg.get("sweep", (1, 2, 4, 8, 16)):
+        c = dict(cfg, n_shards=n)
+        model = Model(tp, torch, c, inp)
+        for _ in range(args.warmup):
+            model.step()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        tp.tp_trace_begin(8 * args.steps)
+        e0.record()
+        for _ in range(args.steps):
+            model.step()
+        e1.record()
+        torch.cuda.synchronize()
+        recs, _ = tp.tp_trace_end()
+        assert tp.tp_get_last_error() == tp.TP_OK
+        ms = e0.elapsed_time(e1) / args.steps
+        kern = {}
+        for name, kms in recs:
+            kern[name] = kern.get(name, 0.0) + kms / args.steps
+        w = work(c)
+        red_bytes = w["bytes"]["reduce_partials"]
+        res[n] = {"ms_per_step": ms, "tflops": w["total_flops"] / ms / 1e9,
+                  "frac_of_bf16_peak": w["total_flops"] / ms / 1e9 / pk["bf16"],
+                  "kernel_ms": {k: round(v, 4) for k, v in kern.items()},
+                  "reduce_gbs": red_bytes / (kern["reduce_partials"] * 1e-3) / 1e9}
+        del model
+        torch.cuda.empty_cache()
+    t1 = res[min(res)]["ms_per_step"]
+    for n in res:
+        res[n]["overhead_vs_n1"] = res[n]["ms_per_step"] / t1 - 1.0
+    line = {"metric": "large-MLP shard sweep: TFLOP/s and N-overhead", "unit": "TFLOP/s",
+            "value": res[max(res)]["tflops"], "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": cfg["name"]},
+            "sweep": {str(k): v for k, v in res.items()}}
+    print(json.dumps(line), flush=True)
 
 
 def main():
@@ -444,13 +501,17 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.CONFIGS))
     ap.add_argument("--shards", type=int, default=0, help="override the shard count N")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="run the workload at every shard count of its sweep (one JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = synth.config(args.workload)
     if args.shards:
         cfg["n_shards"] = args.shards
-    if args.impl == "reference":
+    if args.sweep:
+        run_sweep(args, cfg)
+    elif args.impl == "reference":
         run_reference(args, cfg)
     else:
         run_ours(args, cfg)
