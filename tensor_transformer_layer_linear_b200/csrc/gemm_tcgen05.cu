@@ -10,7 +10,7 @@
 //   warp 1      owns TMEM (two fp32 accumulators of BN columns); one thread
 //               issues tcgen05.mma per stage and releases the stage with
 //               tcgen05.commit.
-//   warps 2-5   epilogue: tcgen05.ld of the finished accumulator, then the
+//   warps 2-9   epilogue: tcgen05.ld of the finished accumulator, then the
 //               column-parallel bias + GeLU (bf16 out) or the row-parallel
 //               fp32 partials, staged in swizzled shared memory and written
 //               with TMA tensor stores, overlapping the next tile's
@@ -39,7 +39,8 @@ namespace tpk {
 
 constexpr int BM = 128;            // accumulator rows per CTA (TMEM lanes)
 constexpr int BK = 64;             // 64 bf16 = 128 bytes = one swizzle row
-constexpr int kGemmThreads = 192;  // 6 warps
+constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, each half the columns
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 
 template <int BN, int CTAS>
 struct GemmCfg {
@@ -50,8 +51,9 @@ struct GemmCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (CTAS == 2) ? 6 : ((BN == 256) ? 4 : 6);
   static constexpr int kTmemCols = 2 * BN;
-  // epilogue staging: 4 warps x 2 buffers x (32 rows x 128 bytes)
-  static constexpr int kStagingBytes = 4 * 2 * 4096;
+  // epilogue staging: per epilogue warp, kStagingBufs buffers of 32 rows x 128 bytes
+  static constexpr int kStagingBufs = 1;
+  static constexpr int kStagingBytes = kEpiWarps * kStagingBufs * 4096;
   static constexpr int kNumBars = 2 * kStages + 5;
   static constexpr int kSmemBytes =
       1024 + kStages * kStageBytes + kStagingBytes + kNumBars * 8 + 16;
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 4 * CTAS);  // one arrival per epilogue warp of the pair
+      mbar_init(tempty_bar(b), kEpiWarps * CTAS);  // one arrival per epilogue warp of the pair
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -245,18 +247,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Each warp owns TMEM lanes [32 q, 32 q + 32) = 32 output rows. Per chunk
-    // of columns (32 fp32 or 64 bf16 = 128 bytes per row) every thread
-    // writes its row into a 128-byte-swizzled staging buffer, then one lane
+    // Warp e (0..7) owns TMEM lanes [32 q, 32 q + 32) (q = warp % 4) = 32
+    // output rows, and half h = e / 4 of the tile's columns. Per chunk of
+    // columns (32 fp32 or 64 bf16 = 128 bytes per row) every thread writes
+    // its row into the warp's 128-byte-swizzled staging buffer, then one lane
     // issues a TMA tensor store of the 32-row box (rows/columns outside the
-    // output are clipped by the TMA unit). Two staging buffers per warp let
-    // the next chunk be written while the previous store drains.
+    // output are clipped by the TMA unit). The next chunk's TMEM load is in
+    // flight while the current chunk is converted and stored.
     const int q = warp & 3;
-    const uint32_t stage_base = smem_u32(staging) + static_cast<uint32_t>((warp - 2) * 2 * 4096);
-    constexpr int CW = OUT_F32 ? 32 : 64;  // columns per chunk
+    const int half = (warp - 2) >> 2;
+    const uint32_t sbase =
+        smem_u32(staging) + static_cast<uint32_t>((warp - 2) * C::kStagingBufs * 4096);
+    uint32_t chunk_ctr = 0;
+    constexpr int CW = OUT_F32 ? 32 : 64;     // columns per chunk
+    constexpr int NCH = (BN / 2) / CW;        // chunks per warp per tile
     int acc = 0;
     uint32_t acc_phase = 0;
-    uint32_t chunk_ctr = 0;
     bool ok = true;
     for (int tile = first_tile; tile < p.num_tiles; tile += tile_step) {
       const int mb = tile % p.num_m;
@@ -269,35 +275,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const int row0 = mb * C::kTileM + static_cast<int>(rank) * BM + q * 32;
-      const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-#pragma unroll 1
-      for (int c = 0; c < BN / CW; ++c) {
-        uint32_t r[CW];
-        tmem_ld_32x32b_x32(tbase + c * CW, &r[0]);
-        if constexpr (!OUT_F32)
-          tmem_ld_32x32b_x32(tbase + c * CW + 32, &r[32]);
-        tmem_ld_wait();
-        const int col0 = nb * BN + c * CW;
+      const int colh = nb * BN + half * (BN / 2);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN + half * (BN / 2));
+      uint32_t r[2][CW];
+      tmem_ld_32x32b_x32(tbase, &r[0][0]);
+      if constexpr (!OUT_F32) tmem_ld_32x32b_x32(tbase + 32, &r[0][32]);
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        tmem_ld_wait();  // chunk c has arrived
+        if (c + 1 < NCH) {
+          tmem_ld_32x32b_x32(tbase + (c + 1) * CW, &r[(c + 1) & 1][0]);
+          if constexpr (!OUT_F32) tmem_ld_32x32b_x32(tbase + (c + 1) * CW + 32, &r[(c + 1) & 1][32]);
+        }
+        const int col0 = colh + c * CW;
         if (col0 >= p.Nc) continue;  // warp-uniform: the whole chunk is past the edge
-        uint32_t w[32];              // this thread's 128-byte row of the chunk
+        const uint32_t* rc = r[c & 1];
+        uint32_t w[32];  // this thread's 128-byte row of the chunk
         if constexpr (OUT_F32) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) w[e] = r[e];
+          for (int e = 0; e < 32; ++e) w[e] = rc[e];
         } else {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             float v[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * j + e]);
+            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(rc[8 * j + e]);
             const int col = col0 + 8 * j;
             if (p.bias != nullptr && col < p.Nc) {
-              const uint4 b = *reinterpret_cast<const uint4*>(
+              const uint4 bv = *reinterpret_cast<const uint4*>(
                   p.bias + static_cast<int64_t>(g) * p.Nc + col);
-              v[0] += bf16_lo(b.x); v[1] += bf16_hi(b.x);
-              v[2] += bf16_lo(b.y); v[3] += bf16_hi(b.y);
-              v[4] += bf16_lo(b.z); v[5] += bf16_hi(b.z);
-              v[6] += bf16_lo(b.w); v[7] += bf16_hi(b.w);
+              v[0] += bf16_lo(bv.x); v[1] += bf16_hi(bv.x);
+              v[2] += bf16_lo(bv.y); v[3] += bf16_hi(bv.y);
+              v[4] += bf16_lo(bv.z); v[5] += bf16_hi(bv.z);
+              v[6] += bf16_lo(bv.w); v[7] += bf16_hi(bv.w);
             }
             if (p.act == 1) {
 #pragma unroll
@@ -309,8 +320,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             w[4 * j + 3] = pack_bf16x2(v[6], v[7]);
           }
         }
-        const uint32_t sbuf = stage_base + (chunk_ctr & 1u) * 4096u;
-        if (lane == 0) bulk_wait_read<1>();  // the store that last used sbuf has read it
+        const uint32_t sbuf = sbase + (chunk_ctr % C::kStagingBufs) * 4096u;
+        ++chunk_ctr;
+        if (lane == 0) bulk_wait_read<C::kStagingBufs - 1>();  // the store that last used sbuf read it
         __syncwarp();
         const uint32_t row_addr = sbuf + static_cast<uint32_t>(lane) * 128u;
 #pragma unroll
@@ -323,7 +335,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_store_3d(&tmD, sbuf, col0, row0, g);
           bulk_commit();
         }
-        ++chunk_ctr;
       }
       tc_fence_before();
       __syncwarp();

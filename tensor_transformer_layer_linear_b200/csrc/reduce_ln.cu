@@ -82,8 +82,7 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(
   }
 }
 
-constexpr int kRowThreads = 256;
-
+template <int THREADS>
 __device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -92,13 +91,15 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   __syncthreads();
   float t = 0.f;
 #pragma unroll
-  for (int i = 0; i < kRowThreads / 32; ++i) t += red[i];
+  for (int i = 0; i < THREADS / 32; ++i) t += red[i];
   __syncthreads();
   return t;
 }
 
-// One CTA per row. CH = 8-element chunks per thread (h <= CH * 8 * 256).
-template <int CH, int NS>
+// One CTA of kRowThreads threads per row; CH = 8-element chunks per thread
+// (h <= CH * 8 * kRowThreads). The plain LayerNorm (no partials) uses 128
+// threads per row so that more rows, and more loads, are in flight per SM.
+template <int CH, int NS, int kRowThreads>
 __global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
     const float* __restrict__ P, int n_shards, int64_t stride, int h,
     const uint16_t* __restrict__ bias, const uint16_t* __restrict__ res,
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
     }
   }
   if (Yln == nullptr) return;
-  const float mean = block_sum(s, red) / static_cast<float>(h);
+  const float mean = block_sum<kRowThreads>(s, red) / static_cast<float>(h);
   float q = 0.f;
 #pragma unroll
   for (int c = 0; c < CH; ++c) {
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
       }
     }
   }
-  const float var = block_sum(q, red) / static_cast<float>(h);
+  const float var = block_sum<kRowThreads>(q, red) / static_cast<float>(h);
   const float rstd = rsqrtf(var + eps);
 #pragma unroll
   for (int c = 0; c < CH; ++c) {
@@ -190,7 +191,7 @@ int launch_reduce(const float* P, int n_shards, int64_t rows, int64_t h, const v
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
 
-template <int CH>
+template <int CH, int THREADS>
 static void launch_rows_ch(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
                            const void* residual, const void* gamma, const void* beta, float eps,
                            void* Y_sum, void* Y_ln, cudaStream_t s) {
@@ -204,21 +205,32 @@ static void launch_rows_ch(const float* P, int n_shards, int64_t rows, int64_t h
   const int hh = static_cast<int>(h);
   const dim3 grid(static_cast<unsigned>(rows));
   switch (n_shards) {
-    case 4: rows_sum_ln_kernel<CH, 4><<<grid, kRowThreads, 0, s>>>(P, 4, stride, hh, b, r, g, be, eps, ys, yl); break;
-    case 8: rows_sum_ln_kernel<CH, 8><<<grid, kRowThreads, 0, s>>>(P, 8, stride, hh, b, r, g, be, eps, ys, yl); break;
-    default: rows_sum_ln_kernel<CH, 0><<<grid, kRowThreads, 0, s>>>(P, n_shards, stride, hh, b, r, g, be, eps, ys, yl); break;
+    case 4: rows_sum_ln_kernel<CH, 4, THREADS><<<grid, THREADS, 0, s>>>(P, 4, stride, hh, b, r, g, be, eps, ys, yl); break;
+    case 8: rows_sum_ln_kernel<CH, 8, THREADS><<<grid, THREADS, 0, s>>>(P, 8, stride, hh, b, r, g, be, eps, ys, yl); break;
+    default: rows_sum_ln_kernel<CH, 0, THREADS><<<grid, THREADS, 0, s>>>(P, n_shards, stride, hh, b, r, g, be, eps, ys, yl); break;
   }
+}
+
+template <int THREADS>
+static void launch_rows(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
+                        const void* residual, const void* gamma, const void* beta, float eps,
+                        void* Y_sum, void* Y_ln, cudaStream_t s) {
+  const int64_t nch = h / 8;
+  if (nch <= THREADS) launch_rows_ch<1, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  else if (nch <= 2 * THREADS) launch_rows_ch<2, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  else if (nch <= 4 * THREADS) launch_rows_ch<4, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  else if (nch <= 8 * THREADS) launch_rows_ch<8, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  else launch_rows_ch<16, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
 }
 
 int launch_rows_sum_ln(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
                        const void* residual, const void* gamma, const void* beta, float eps,
                        void* Y_sum, void* Y_ln, cudaStream_t s) {
   if (rows <= 0) return 0;
-  const int64_t nch = h / 8;
-  if (nch <= kRowThreads) launch_rows_ch<1>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
-  else if (nch <= 2 * kRowThreads) launch_rows_ch<2>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
-  else if (nch <= 4 * kRowThreads) launch_rows_ch<4>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
-  else launch_rows_ch<8>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  if (n_shards == 0)
+    launch_rows<128>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  else
+    launch_rows<256>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
 
