@@ -48,7 +48,12 @@ L2_BYTES = 126 * 1024 * 1024
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # committed ncu captures under profiles/, keyed by (workload, kernel). None
 # until a capture of the current kernel exists.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/gemm_tcgen05_layer_ncu_full.md: QKV 244.1 MB and MLP-up 321.7 MB -> mean per launch
+    (DEFAULT_WORKLOAD, "gemm_column_parallel"): 282.9e6,
+    # same capture: W_O 545.1 MB and MLP-down 769.9 MB -> mean per launch
+    (DEFAULT_WORKLOAD, "gemm_row_parallel"): 657.5e6,
+}
 
 
 def peaks() -> dict:
