@@ -323,6 +323,67 @@ def transformer_layer(X, p: dict, batch: int, seq: int, n_heads: int,
 
 
 # --------------------------------------------------------------------------
+# sequence parallelism ([TP-LLM] "Sequence Parallelism")
+# --------------------------------------------------------------------------
+#
+# Activations outside the blocks are split along the sequence: shard i owns
+# positions [i S/N, (i+1) S/N) of every sequence of the batch. A shard's
+# slice is stored [batch][S/N][h]; the N slices stacked make [N][b][S/N][h].
+
+def sequence_shard(X: np.ndarray, batch: int, seq: int, n_shards: int) -> list:
+    """Split token rows (batch-major [b*S, h]) into the N sequence slices,
+    each [b, S/N, h]."""
+    _check_div("seq", seq, n_shards)
+    ss = seq // n_shards
+    X3 = X.reshape(batch, seq, -1)
+    return [X3[:, i * ss:(i + 1) * ss, :] for i in range(n_shards)]
+
+
+def all_gather_sequence(slices: list, batch: int, seq: int) -> np.ndarray:
+    """The all-gather before a column-parallel layer: the N sequence slices
+    concatenated along the sequence, back to [b*S, h] token rows."""
+    return np.concatenate(slices, axis=1).reshape(batch * seq, -1)
+
+
+def reduce_scatter_partials(partials: list, batch: int, seq: int, n_shards: int,
+                            bias=None, residual_slices=None) -> list:
+    """The reduce-scatter after a row-parallel layer: the sum of the N
+    partials, scattered along the sequence (shard i keeps its slice), with the
+    output bias and that shard's residual slice added once."""
+    Y = reduce_partials(partials, bias)
+    out = sequence_shard(Y, batch, seq, n_shards)
+    if residual_slices is not None:
+        out = [o + r for o, r in zip(out, residual_slices)]
+    return out
+
+
+def transformer_layer_sp(X_slices: list, p: dict, batch: int, seq: int,
+                         n_heads: int, n_shards: int, eps: float = 1e-5,
+                         causal: bool = True) -> list:
+    """Pre-LN layer with sequence parallelism: LayerNorm on each shard's
+    slice, all-gather before each column-parallel layer, reduce-scatter
+    after each row-parallel layer, residual adds on the slices.
+    Returns the N output slices [b, S/N, h]."""
+    h = X_slices[0].shape[-1]
+    d = h // n_heads
+    hs = h // n_shards
+    x1 = [layernorm(x, p["ln1_g"], p["ln1_b"], eps) for x in X_slices]
+    X1 = all_gather_sequence(x1, batch, seq)
+    QKV_i = column_parallel_linear(X1, p["Wqkv"], p["bqkv"], n_shards,
+                                   kind=SPLIT_QKV_HEADS, head_dim=d)
+    O_i = [attention_heads(q[:, :hs], q[:, hs:2 * hs], q[:, 2 * hs:],
+                           batch, seq, n_heads // n_shards, causal)
+           for q in QKV_i]
+    P_i = row_parallel_linear(O_i, p["Wo"], n_shards)
+    h1 = reduce_scatter_partials(P_i, batch, seq, n_shards, p["bo"], X_slices)
+    x2 = [layernorm(x, p["ln2_g"], p["ln2_b"], eps) for x in h1]
+    X2 = all_gather_sequence(x2, batch, seq)
+    A_i = column_parallel_linear(X2, p["A"], p["b1"], n_shards, act=gelu)
+    P_i = row_parallel_linear(A_i, p["B"], n_shards)
+    return reduce_scatter_partials(P_i, batch, seq, n_shards, p["b2"], h1)
+
+
+# --------------------------------------------------------------------------
 # the same definitions restricted to a subset of output token rows
 # (used to check full-size workloads on sampled rows)
 # --------------------------------------------------------------------------

@@ -420,3 +420,39 @@ def test_planted_mistakes_are_caught(monkeypatch):
         m.setattr(O, "reduce_partials", per_partial)
         with pytest.raises(AssertionError):
             test_mlp_brute_force(2)
+
+
+# ---------------------------------------------------------------- sequence parallelism
+
+@pytest.mark.parametrize("n", [1, 2, 4])
+def test_reduce_scatter_then_all_gather_is_all_reduce(n):
+    """[TP-LLM] "Sequence Parallelism": an all-reduce is a reduce-scatter
+    followed by an all-gather; exact for integer-valued partials."""
+    rng = np.random.default_rng(12)
+    batch, seq, h = 3, 8, 5
+    P = [_int_matrix(rng, (batch * seq, h)) for _ in range(n)]
+    b = _int_matrix(rng, (h,))
+    rs = O.reduce_scatter_partials(P, batch, seq, n, b)
+    assert all(r.shape == (batch, seq // n, h) for r in rs)
+    assert np.array_equal(O.all_gather_sequence(rs, batch, seq), O.reduce_partials(P, b))
+    # shard i holds positions [i S/N, (i+1) S/N) of every sequence
+    full = O.reduce_partials(P, b).reshape(batch, seq, h)
+    for i, r in enumerate(rs):
+        for bb in range(batch):
+            for s_ in range(seq // n):
+                assert np.array_equal(r[bb, s_], full[bb, i * (seq // n) + s_])
+
+
+@pytest.mark.parametrize("n", [1, 2, 4])
+def test_sequence_parallel_layer_equals_standard_layer(n):
+    """Sharding LayerNorm, dropout and the residual along the sequence does
+    not change the layer's output ([TP-LLM] "Sequence Parallelism": the same
+    math with reduce-scatter + all-gather in place of all-reduce)."""
+    rng = np.random.default_rng(13)
+    batch, seq, n_heads, d, F = 2, 8, 4, 2, 16
+    h = n_heads * d
+    p = _layer_params(rng, h, F)
+    X = rng.standard_normal((batch * seq, h))
+    ref = O.transformer_layer(X, p, batch, seq, n_heads)
+    out = O.transformer_layer_sp(O.sequence_shard(X, batch, seq, n), p, batch, seq, n_heads, n)
+    np.testing.assert_allclose(O.all_gather_sequence(out, batch, seq), ref, rtol=1e-11, atol=1e-11)
