@@ -273,7 +273,11 @@ class Model:
         X = self.X if X is None else X
         Y = self.Y if Y is None else Y
         n, h = cfg["n_shards"], cfg["h"]
-        if cfg["kind"] == "layer":
+        if cfg["kind"] == "layer" and cfg.get("sequence_parallel"):
+            # X and Y hold the N sequence slices [N][b][S/N][h]
+            tp.tp_layer_forward_sp(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"], cfg["ffn"], n,
+                                   self.w, cfg.get("ln_eps", 1e-5), self.ws, self.ws_bytes, Y)
+        elif cfg["kind"] == "layer":
             tp.tp_layer_forward(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"], cfg["ffn"], n,
                                 self.w, cfg.get("ln_eps", 1e-5), self.ws, self.ws_bytes, Y)
         elif cfg["kind"] == "attn":
@@ -423,7 +427,9 @@ def run_ours(args, cfg) -> None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": cfg["name"], "tokens": M, "h": h, "n_shards": cfg["n_shards"],
+        "config": {"workload": cfg["name"] + ("+sequence_parallel" if cfg.get("sequence_parallel")
+                                              else ""),
+                   "tokens": M, "h": h, "n_shards": cfg["n_shards"],
                    "heads": cfg.get("n_heads"), "ffn": cfg.get("ffn"),
                    "l2": "inputs larger than L2 (per-step working set "
                          f"{(w['bytes'].get('reduce_partials', 0) + 4 * h * h * 2) / 1e6:.0f}+ MB "
@@ -506,6 +512,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.CONFIGS))
     ap.add_argument("--shards", type=int, default=0, help="override the shard count N")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sequence-parallel", action="store_true",
+                    help="layer workload: run tp_layer_forward_sp on sequence-sharded input")
     ap.add_argument("--sweep", action="store_true",
                     help="run the workload at every shard count of its sweep (one JSON line)")
     args = ap.parse_args()
@@ -514,6 +522,10 @@ def main():
     cfg = synth.config(args.workload)
     if args.shards:
         cfg["n_shards"] = args.shards
+    if args.sequence_parallel:
+        if cfg["kind"] != "layer":
+            ap.error("--sequence-parallel applies to the layer workload")
+        cfg["sequence_parallel"] = True
     if args.sweep:
         run_sweep(args, cfg)
     elif args.impl == "reference":

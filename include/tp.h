@@ -84,7 +84,7 @@ typedef enum {
     TP_ACT_GELU_ERF = 1
 } tp_act;
 
-typedef enum { TP_WS_MLP = 0, TP_WS_ATTN = 1, TP_WS_LAYER = 2 } tp_ws_kind;
+typedef enum { TP_WS_MLP = 0, TP_WS_ATTN = 1, TP_WS_LAYER = 2, TP_WS_LAYER_SP = 3 } tp_ws_kind;
 
 /* Weights of one pre-LN layer, all device pointers in the packed shard
    layouts below. h = hidden, F = FFN width, N = shards. */
@@ -230,6 +230,45 @@ tp_status tp_layer_forward(const uint16_t* X, int64_t batch, int64_t seq,
                            float ln_eps, void* ws, size_t ws_bytes,
                            uint16_t* Y, void* stream);
 
+/* ---- Sequence parallelism ([TP-LLM] "Sequence Parallelism") ----------
+ * Outside the tensor-parallel blocks, activations are split along the
+ * sequence: shard i owns positions [i S/N, (i+1) S/N) of every sequence.
+ * Sequence-sharded layout: [N][batch][S/N][h], i.e. token (b, s) of a
+ * token-ordered [batch*S][h] tensor lives at
+ * [s / (S/N)][b][s % (S/N)][:]. seq % N must be 0. */
+
+/* tp_reduce_scatter_partials - the reduce-scatter after a row-parallel layer:
+ * Y_shards (sequence-sharded) = slices of (sum_{i<N} P_i + bias), plus the
+ * residual given in the same sharded layout (NULL ok). partials
+ * [N][batch*seq][h] fp32 in token order; bias [h] or NULL. An all-reduce is
+ * this followed by tp_all_gather_sequence. h % 8 == 0. */
+tp_status tp_reduce_scatter_partials(const float* partials, int n_shards,
+                                     int64_t batch, int64_t seq, int64_t h,
+                                     const uint16_t* bias,
+                                     const uint16_t* residual_shards,
+                                     uint16_t* Y_shards, void* stream);
+
+/* tp_all_gather_sequence - the all-gather before a column-parallel layer:
+ * X [batch*seq][h] (token order) from X_shards (sequence-sharded). A pure
+ * permutation copy. h % 8 == 0. */
+tp_status tp_all_gather_sequence(const uint16_t* X_shards, int n_shards,
+                                 int64_t batch, int64_t seq, int64_t h,
+                                 uint16_t* X, void* stream);
+
+/* tp_layer_forward_sp - the pre-LN layer of tp_layer_forward with sequence
+ * parallelism: X_shards and Y_shards in the sequence-sharded layout;
+ * LayerNorm on each shard's slice followed by the all-gather (one fused
+ * kernel), reduce-scatter after each row-parallel layer (fused with the
+ * bias, the sharded residual and, after attention, LN2 + all-gather).
+ * Same result as tp_layer_forward up to the row order.
+ * ws >= tp_workspace_bytes(TP_WS_LAYER_SP, batch*seq, h, F, N). */
+tp_status tp_layer_forward_sp(const uint16_t* X_shards, int64_t batch,
+                              int64_t seq, int64_t h, int64_t n_heads,
+                              int64_t ffn, int n_shards,
+                              const tp_layer_weights* w, float ln_eps,
+                              void* ws, size_t ws_bytes, uint16_t* Y_shards,
+                              void* stream);
+
 /* Size in bytes of the library-owned scratch array used by
  * tp_mlp_forward_noalloc (32 MiB, reserved on every GPU that loads the
  * library, until the process exits). */
@@ -260,7 +299,8 @@ tp_status tp_mlp_forward_noalloc(const uint16_t* X, int64_t B, int64_t h,
                                  void* stream);
 
 /* Workspace bytes for tp_mlp_forward (kind TP_WS_MLP), tp_attn_forward
- * (TP_WS_ATTN, ffn ignored) or tp_layer_forward (TP_WS_LAYER). tokens =
+ * (TP_WS_ATTN, ffn ignored), tp_layer_forward (TP_WS_LAYER) or
+ * tp_layer_forward_sp (TP_WS_LAYER_SP). tokens =
  * batch * seq. Returns 0 for invalid arguments. */
 size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn,
                           int n_shards);

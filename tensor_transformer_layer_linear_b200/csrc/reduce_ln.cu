@@ -65,20 +65,59 @@ __device__ __forceinline__ void sum_partials8(const float* __restrict__ P, int n
   }
 }
 
+// Row m = b S + s of the token-ordered [batch][S] rows, stored in the
+// sequence-sharded layout [N][batch][S/N]: shard s / (S/N) keeps positions
+// [i S/N, (i+1) S/N) of every sequence ("Sequence Parallelism"). sp.n == 0
+// means the identity.
+struct SeqShard {
+  int n;      // shards (0: no permutation)
+  int batch;
+  int seq;
+};
+__device__ __forceinline__ int64_t seq_shard_row(const SeqShard& sp, int64_t m) {
+  if (sp.n == 0) return m;
+  const int ss = sp.seq / sp.n;
+  const int64_t b = m / sp.seq;
+  const int s = static_cast<int>(m - b * sp.seq);
+  const int i = s / ss;
+  return (static_cast<int64_t>(i) * sp.batch + b) * ss + (s - i * ss);
+}
+
+// Y = sum_i P_i + bias + residual. With sp.n > 0 the residual is read from,
+// and Y written to, the sequence-sharded layout (the reduce-scatter).
 template <int NS>
 __global__ void __launch_bounds__(256) reduce_partials_kernel(
     const float* __restrict__ P, int n_shards, int64_t n_elems, int h,
     const uint16_t* __restrict__ bias, const uint16_t* __restrict__ res,
-    uint16_t* __restrict__ Y) {
+    uint16_t* __restrict__ Y, SeqShard sp) {
   const int64_t n8 = n_elems >> 3;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t e = i << 3;
     float acc[8];
     sum_partials8<NS>(P, n_shards, n_elems, e, acc);
-    if (bias != nullptr) add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(bias + e % h)));
-    if (res != nullptr) add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(res + e)));
-    *reinterpret_cast<uint4*>(Y + e) = to_bf16x8(acc);
+    const int64_t m = e / h;
+    const int64_t col = e - m * h;
+    const int64_t d = seq_shard_row(sp, m) * h + col;
+    if (bias != nullptr) add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(bias + col)));
+    if (res != nullptr) add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(res + d)));
+    *reinterpret_cast<uint4*>(Y + d) = to_bf16x8(acc);
+  }
+}
+
+// X[b S + s] = X_shards[s / (S/N)][b][s % (S/N)]: the all-gather along the
+// sequence before a column-parallel layer (16-byte copies).
+__global__ void __launch_bounds__(256) all_gather_sequence_kernel(
+    const uint16_t* __restrict__ Xs, uint16_t* __restrict__ X, int64_t n_elems, int h,
+    SeqShard sp) {
+  const int64_t n8 = n_elems >> 3;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t e = i << 3;
+    const int64_t m = e / h;
+    const int64_t col = e - m * h;
+    *reinterpret_cast<uint4*>(X + e) =
+        __ldcs(reinterpret_cast<const uint4*>(Xs + seq_shard_row(sp, m) * h + col));
   }
 }
 
@@ -99,14 +138,19 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 // One CTA of kRowThreads threads per row; CH = 8-element chunks per thread
 // (h <= CH * 8 * kRowThreads). The plain LayerNorm (no partials) uses 128
 // threads per row so that more rows, and more loads, are in flight per SM.
+// With sp.n > 0 the residual is read from and Y_sum written to the
+// sequence-sharded layout, and Y_ln is written in token order when ln_natural
+// (the sharded LayerNorm followed by the all-gather) or sharded otherwise.
 template <int CH, int NS, int kRowThreads>
 __global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
     const float* __restrict__ P, int n_shards, int64_t stride, int h,
     const uint16_t* __restrict__ bias, const uint16_t* __restrict__ res,
     const uint16_t* __restrict__ gamma, const uint16_t* __restrict__ beta, float eps,
-    uint16_t* __restrict__ Ysum, uint16_t* __restrict__ Yln) {
+    uint16_t* __restrict__ Ysum, uint16_t* __restrict__ Yln, SeqShard sp, int ln_natural) {
   __shared__ float red[kRowThreads / 32];
   const int64_t row_off = static_cast<int64_t>(blockIdx.x) * h;
+  const int64_t sh_off = seq_shard_row(sp, blockIdx.x) * h;  // same row, sharded layout
+  const int64_t ln_off = ln_natural ? row_off : sh_off;
   const int nch = h >> 3;
   float v[CH][8];
   float s = 0.f;
@@ -121,10 +165,11 @@ __global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[c][j] = 0.f;
       }
+      const int64_t es = sh_off + (ch << 3);
       if (bias != nullptr) add_bf16x8(v[c], __ldg(reinterpret_cast<const uint4*>(bias + (ch << 3))));
-      if (res != nullptr) add_bf16x8(v[c], __ldg(reinterpret_cast<const uint4*>(res + e)));
+      if (res != nullptr) add_bf16x8(v[c], __ldg(reinterpret_cast<const uint4*>(res + es)));
       const uint4 o = to_bf16x8(v[c]);
-      if (Ysum != nullptr) *reinterpret_cast<uint4*>(Ysum + e) = o;
+      if (Ysum != nullptr) *reinterpret_cast<uint4*>(Ysum + es) = o;
       // statistics of the rounded values, as a separate LayerNorm would see them
       v[c][0] = bf16_lo(o.x); v[c][1] = bf16_hi(o.x);
       v[c][2] = bf16_lo(o.y); v[c][3] = bf16_hi(o.y);
@@ -163,13 +208,15 @@ __global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
       float y[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) y[j] = (v[c][j] - mean) * rstd * gv[j] + bv[j];
-      *reinterpret_cast<uint4*>(Yln + row_off + (ch << 3)) = to_bf16x8(y);
+      *reinterpret_cast<uint4*>(Yln + ln_off + (ch << 3)) = to_bf16x8(y);
     }
   }
 }
 
 int launch_reduce(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
-                  const void* residual, void* Y, cudaStream_t s, int num_sms) {
+                  const void* residual, void* Y, cudaStream_t s, int num_sms, int sp_n,
+                  int sp_batch, int sp_seq) {
+  const SeqShard sp{sp_n, sp_batch, sp_seq};
   const int64_t n = rows * h;
   const int64_t n8 = n / 8;
   int64_t blocks = (n8 + 255) / 256;
@@ -181,12 +228,12 @@ int launch_reduce(const float* P, int n_shards, int64_t rows, int64_t h, const v
   auto y = static_cast<uint16_t*>(Y);
   const int hh = static_cast<int>(h);
   switch (n_shards) {
-    case 1: reduce_partials_kernel<1><<<blocks, 256, 0, s>>>(P, 1, n, hh, b, r, y); break;
-    case 2: reduce_partials_kernel<2><<<blocks, 256, 0, s>>>(P, 2, n, hh, b, r, y); break;
-    case 4: reduce_partials_kernel<4><<<blocks, 256, 0, s>>>(P, 4, n, hh, b, r, y); break;
-    case 8: reduce_partials_kernel<8><<<blocks, 256, 0, s>>>(P, 8, n, hh, b, r, y); break;
-    case 16: reduce_partials_kernel<16><<<blocks, 256, 0, s>>>(P, 16, n, hh, b, r, y); break;
-    default: reduce_partials_kernel<0><<<blocks, 256, 0, s>>>(P, n_shards, n, hh, b, r, y); break;
+    case 1: reduce_partials_kernel<1><<<blocks, 256, 0, s>>>(P, 1, n, hh, b, r, y, sp); break;
+    case 2: reduce_partials_kernel<2><<<blocks, 256, 0, s>>>(P, 2, n, hh, b, r, y, sp); break;
+    case 4: reduce_partials_kernel<4><<<blocks, 256, 0, s>>>(P, 4, n, hh, b, r, y, sp); break;
+    case 8: reduce_partials_kernel<8><<<blocks, 256, 0, s>>>(P, 8, n, hh, b, r, y, sp); break;
+    case 16: reduce_partials_kernel<16><<<blocks, 256, 0, s>>>(P, 16, n, hh, b, r, y, sp); break;
+    default: reduce_partials_kernel<0><<<blocks, 256, 0, s>>>(P, n_shards, n, hh, b, r, y, sp); break;
   }
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
@@ -194,7 +241,7 @@ int launch_reduce(const float* P, int n_shards, int64_t rows, int64_t h, const v
 template <int CH, int THREADS>
 static void launch_rows_ch(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
                            const void* residual, const void* gamma, const void* beta, float eps,
-                           void* Y_sum, void* Y_ln, cudaStream_t s) {
+                           void* Y_sum, void* Y_ln, cudaStream_t s, SeqShard sp, int ln_nat) {
   auto b = static_cast<const uint16_t*>(bias);
   auto r = static_cast<const uint16_t*>(residual);
   auto g = static_cast<const uint16_t*>(gamma);
@@ -205,32 +252,50 @@ static void launch_rows_ch(const float* P, int n_shards, int64_t rows, int64_t h
   const int hh = static_cast<int>(h);
   const dim3 grid(static_cast<unsigned>(rows));
   switch (n_shards) {
-    case 4: rows_sum_ln_kernel<CH, 4, THREADS><<<grid, THREADS, 0, s>>>(P, 4, stride, hh, b, r, g, be, eps, ys, yl); break;
-    case 8: rows_sum_ln_kernel<CH, 8, THREADS><<<grid, THREADS, 0, s>>>(P, 8, stride, hh, b, r, g, be, eps, ys, yl); break;
-    default: rows_sum_ln_kernel<CH, 0, THREADS><<<grid, THREADS, 0, s>>>(P, n_shards, stride, hh, b, r, g, be, eps, ys, yl); break;
+    case 4: rows_sum_ln_kernel<CH, 4, THREADS><<<grid, THREADS, 0, s>>>(P, 4, stride, hh, b, r, g, be, eps, ys, yl, sp, ln_nat); break;
+    case 8: rows_sum_ln_kernel<CH, 8, THREADS><<<grid, THREADS, 0, s>>>(P, 8, stride, hh, b, r, g, be, eps, ys, yl, sp, ln_nat); break;
+    default: rows_sum_ln_kernel<CH, 0, THREADS><<<grid, THREADS, 0, s>>>(P, n_shards, stride, hh, b, r, g, be, eps, ys, yl, sp, ln_nat); break;
   }
 }
 
 template <int THREADS>
 static void launch_rows(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
                         const void* residual, const void* gamma, const void* beta, float eps,
-                        void* Y_sum, void* Y_ln, cudaStream_t s) {
+                        void* Y_sum, void* Y_ln, cudaStream_t s, SeqShard sp, int ln_nat) {
   const int64_t nch = h / 8;
-  if (nch <= THREADS) launch_rows_ch<1, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
-  else if (nch <= 2 * THREADS) launch_rows_ch<2, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
-  else if (nch <= 4 * THREADS) launch_rows_ch<4, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
-  else if (nch <= 8 * THREADS) launch_rows_ch<8, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
-  else launch_rows_ch<16, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+  if (nch <= THREADS) launch_rows_ch<1, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_nat);
+  else if (nch <= 2 * THREADS) launch_rows_ch<2, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_nat);
+  else if (nch <= 4 * THREADS) launch_rows_ch<4, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_nat);
+  else if (nch <= 8 * THREADS) launch_rows_ch<8, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_nat);
+  else launch_rows_ch<16, THREADS>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_nat);
 }
 
 int launch_rows_sum_ln(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
                        const void* residual, const void* gamma, const void* beta, float eps,
-                       void* Y_sum, void* Y_ln, cudaStream_t s) {
+                       void* Y_sum, void* Y_ln, cudaStream_t s, int sp_n, int sp_batch,
+                       int sp_seq, int ln_natural) {
   if (rows <= 0) return 0;
+  const SeqShard sp{sp_n, sp_batch, sp_seq};
   if (n_shards == 0)
-    launch_rows<128>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+    launch_rows<128>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp,
+                     ln_natural);
   else
-    launch_rows<256>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s);
+    launch_rows<256>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp,
+                     ln_natural);
+  return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
+
+int launch_all_gather_sequence(const void* Xs, int sp_n, int sp_batch, int sp_seq, int64_t h,
+                               void* X, cudaStream_t s, int num_sms) {
+  const SeqShard sp{sp_n, sp_batch, sp_seq};
+  const int64_t n = static_cast<int64_t>(sp_batch) * sp_seq * h;
+  int64_t blocks = (n / 8 + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  all_gather_sequence_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(Xs),
+                                                     static_cast<uint16_t*>(X), n,
+                                                     static_cast<int>(h), sp);
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
 

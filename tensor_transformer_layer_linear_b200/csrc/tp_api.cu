@@ -130,6 +130,7 @@ const char* tp_kernel_name(int kid) {
     case tpk::KID_REDUCE_LN: return "reduce_partials_layernorm";
     case tpk::KID_LAYERNORM: return "layernorm";
     case tpk::KID_ATTENTION: return "attention";
+    case tpk::KID_ALL_GATHER: return "all_gather_sequence";
     default: return "unknown";
   }
 }
@@ -401,7 +402,7 @@ size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int 
   if (kind == TP_WS_ATTN) {
     return round256(M * 3 * H * 2) + round256(M * H * 2) + partials;
   }
-  if (kind == TP_WS_LAYER) {
+  if (kind == TP_WS_LAYER || kind == TP_WS_LAYER_SP) {
     if (ffn <= 0) return 0;
     return 3 * round256(M * H * 2) + round256(M * 3 * H * 2) + round256(M * H * 2) +
            round256(M * static_cast<size_t>(ffn) * 2) + partials;
@@ -510,4 +511,107 @@ tp_status tp_layer_forward(const uint16_t* X, int64_t batch, int64_t seq, int64_
   return tp_reduce_partials(part, n_shards, M, h, w->b2, h1, Y, stream);
 }
 
+
+tp_status tp_reduce_scatter_partials(const float* partials, int n_shards, int64_t batch,
+                                     int64_t seq, int64_t h, const uint16_t* bias,
+                                     const uint16_t* residual_shards, uint16_t* Y_shards,
+                                     void* stream) {
+  if (partials == nullptr || Y_shards == nullptr) return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || n_shards <= 0 || h % 8 || seq % n_shards)
+    return TP_ERR_SHAPE;
+  if (batch * seq > kIntMax || seq > kIntMax) return TP_ERR_SHAPE;
+  if (!al16(partials) || !al16(Y_shards) || (bias && !al16(bias)) ||
+      (residual_shards && !al16(residual_shards)))
+    return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_REDUCE, as_stream(stream));
+  return tpk::launch_reduce(partials, n_shards, batch * seq, h, bias, residual_shards, Y_shards,
+                            as_stream(stream), d.num_sms, n_shards, static_cast<int>(batch),
+                            static_cast<int>(seq)) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_all_gather_sequence(const uint16_t* X_shards, int n_shards, int64_t batch,
+                                 int64_t seq, int64_t h, uint16_t* X, void* stream) {
+  if (X_shards == nullptr || X == nullptr) return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || n_shards <= 0 || h % 8 || seq % n_shards)
+    return TP_ERR_SHAPE;
+  if (batch * seq > kIntMax || seq > kIntMax || h > kIntMax) return TP_ERR_SHAPE;
+  if (!al16(X_shards) || !al16(X)) return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_ALL_GATHER, as_stream(stream));
+  return tpk::launch_all_gather_sequence(X_shards, n_shards, static_cast<int>(batch),
+                                         static_cast<int>(seq), h, X, as_stream(stream),
+                                         d.num_sms) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_layer_forward_sp(const uint16_t* X_shards, int64_t batch, int64_t seq, int64_t h,
+                              int64_t n_heads, int64_t ffn, int n_shards,
+                              const tp_layer_weights* w, float ln_eps, void* ws, size_t ws_bytes,
+                              uint16_t* Y_shards, void* stream) {
+  if (X_shards == nullptr || w == nullptr || Y_shards == nullptr || ws == nullptr)
+    return TP_ERR_NULL;
+  if (w->ln1_gamma == nullptr || w->ln1_beta == nullptr || w->Wqkv_shards == nullptr ||
+      w->Wo_shards == nullptr || w->ln2_gamma == nullptr || w->ln2_beta == nullptr ||
+      w->A_shards == nullptr || w->B_shards == nullptr)
+    return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || n_heads <= 0 || ffn <= 0 || n_shards <= 0)
+    return TP_ERR_SHAPE;
+  if (h % n_heads || n_heads % n_shards || ffn % n_shards || (ffn / n_shards) % 8 || h % 8 ||
+      h > 16384 || seq % n_shards)
+    return TP_ERR_SHAPE;
+  if (h / n_heads != 128) return TP_ERR_UNSUPPORTED;
+  const int64_t M = batch * seq;
+  if (M > kIntMax) return TP_ERR_SHAPE;
+  const size_t need = tp_workspace_bytes(TP_WS_LAYER_SP, M, h, ffn, n_shards);
+  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  if (!al16(ws) || !al16(X_shards) || !al16(Y_shards)) return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  const size_t act_b = round256(static_cast<size_t>(M) * h * 2);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  uint16_t* x1 = reinterpret_cast<uint16_t*>(p); p += act_b;  // token order (gathered)
+  uint16_t* h1 = reinterpret_cast<uint16_t*>(p); p += act_b;  // sequence-sharded
+  uint16_t* x2 = reinterpret_cast<uint16_t*>(p); p += act_b;  // token order (gathered)
+  uint16_t* qkv = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * 3 * h * 2);
+  uint16_t* o = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* a = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * ffn * 2);
+  float* part = reinterpret_cast<float*>(p);
+  cudaStream_t s = as_stream(stream);
+  const int sb = static_cast<int>(batch), sq = static_cast<int>(seq);
+
+  {  // LN1 on each shard's slice, written gathered (token order)
+    TraceScope ts(tpk::KID_LAYERNORM, s);
+    if (tpk::launch_rows_sum_ln(nullptr, 0, M, h, nullptr, X_shards, w->ln1_gamma, w->ln1_beta,
+                                ln_eps, nullptr, x1, s, n_shards, sb, sq, 1) != 0)
+      return TP_ERR_CUDA;
+  }
+  st = tp_column_linear(x1, M, h, w->Wqkv_shards, w->bqkv_shards, 3 * h, n_shards, TP_ACT_NONE,
+                        qkv, stream);
+  if (st != TP_OK) return st;
+  st = tp_attention(qkv, batch, seq, h, n_heads, 1, n_shards, o, stream);
+  if (st != TP_OK) return st;
+  st = tp_row_linear(o, M, h, w->Wo_shards, h, n_shards, part, stream);
+  if (st != TP_OK) return st;
+  {  // reduce-scatter (+ b_O + sharded residual) -> h1 sharded; LN2 -> x2 gathered
+    TraceScope ts(tpk::KID_REDUCE_LN, s);
+    if (tpk::launch_rows_sum_ln(part, n_shards, M, h, w->bo, X_shards, w->ln2_gamma, w->ln2_beta,
+                                ln_eps, h1, x2, s, n_shards, sb, sq, 1) != 0)
+      return TP_ERR_CUDA;
+  }
+  st = tp_column_linear(x2, M, h, w->A_shards, w->b1_shards, ffn, n_shards, TP_ACT_GELU_ERF, a,
+                        stream);
+  if (st != TP_OK) return st;
+  st = tp_row_linear(a, M, ffn, w->B_shards, h, n_shards, part, stream);
+  if (st != TP_OK) return st;
+  return tp_reduce_scatter_partials(part, n_shards, batch, seq, h, w->b2, h1, Y_shards, stream);
+}
 }  // extern "C"

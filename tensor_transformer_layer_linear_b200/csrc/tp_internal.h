@@ -15,7 +15,8 @@ enum KernelId {
   KID_REDUCE_LN = 4,
   KID_LAYERNORM = 5,
   KID_ATTENTION = 6,
-  KID_COUNT = 7
+  KID_ALL_GATHER = 7,
+  KID_COUNT = 8
 };
 
 // One batched GEMM over G shards: D[g] (M x Nc) = A[g] (M x K) . B[g]^T with
@@ -37,17 +38,29 @@ struct GemmProblem {
 // launch failed (cudaGetLastError()).
 int launch_gemm(const GemmProblem& p, cudaStream_t s, unsigned* err, int num_sms);
 
+// Sequence-sharded layout of token rows (sp_n > 0): row b*S + s lives at
+// [s / (S/N)][b][s % (S/N)] of [N][batch][S/N]; sp_n == 0 means token order.
+
 // Y = sum_{i<N} P_i + bias + residual (bf16 out). n_elems % 8 == 0, h % 8 == 0.
+// With sp_n > 0 the residual and Y use the sequence-sharded layout.
 int launch_reduce(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
-                  const void* residual, void* Y, cudaStream_t s, int num_sms);
+                  const void* residual, void* Y, cudaStream_t s, int num_sms, int sp_n = 0,
+                  int sp_batch = 0, int sp_seq = 0);
+
+// X (token order) from X_shards (sequence-sharded layout).
+int launch_all_gather_sequence(const void* Xs, int sp_n, int sp_batch, int sp_seq, int64_t h,
+                               void* X, cudaStream_t s, int num_sms);
 
 // Per row: S = bf16(sum_i P_i + bias + residual) -> Y_sum (if non-null);
 // Y_ln = LN(S) with gamma, beta, eps (if non-null). n_shards may be 0
 // (then S = residual, i.e. a plain LayerNorm of `residual`). h % 8 == 0,
 // h <= 16384.
+// With sp_n > 0 the residual and Y_sum use the sequence-sharded layout and
+// Y_ln is written in token order if ln_natural, else sharded.
 int launch_rows_sum_ln(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
                        const void* residual, const void* gamma, const void* beta, float eps,
-                       void* Y_sum, void* Y_ln, cudaStream_t s);
+                       void* Y_sum, void* Y_ln, cudaStream_t s, int sp_n = 0, int sp_batch = 0,
+                       int sp_seq = 0, int ln_natural = 1);
 
 // Causal / full attention of every shard's heads, head_dim 128.
 int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t h, int64_t n_heads,

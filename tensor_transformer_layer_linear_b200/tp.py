@@ -31,7 +31,7 @@ TP_OK, TP_ERR_NULL, TP_ERR_SHAPE, TP_ERR_ALIGN = 0, 1, 2, 3
 TP_ERR_WORKSPACE, TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_TIMEOUT = 4, 5, 6, 7
 TP_SPLIT_COLUMN, TP_SPLIT_ROW, TP_SPLIT_QKV_HEADS = 0, 1, 2
 TP_ACT_NONE, TP_ACT_GELU_ERF = 0, 1
-TP_WS_MLP, TP_WS_ATTN, TP_WS_LAYER = 0, 1, 2
+TP_WS_MLP, TP_WS_ATTN, TP_WS_LAYER, TP_WS_LAYER_SP = 0, 1, 2, 3
 
 _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
@@ -60,6 +60,10 @@ _SIGS = {
                                 ctypes.POINTER(tp_layer_weights), _f32, _vp, _sz, _vp, _vp]),
     "tp_mlp_forward_noalloc": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                       _vp]),
+    "tp_reduce_scatter_partials": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "tp_all_gather_sequence": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _vp]),
+    "tp_layer_forward_sp": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32,
+                                   ctypes.POINTER(tp_layer_weights), _f32, _vp, _sz, _vp, _vp]),
     "tp_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "tp_get_last_error": (_i32, [_vp]),
     "tp_status_string": (ctypes.c_char_p, [_i32]),
@@ -212,6 +216,25 @@ def tp_layer_forward(X, batch, seq, h, n_heads, ffn, n_shards, weights: tp_layer
     _check(lib.tp_layer_forward(_p(X), batch, seq, h, n_heads, ffn, n_shards,
                                 ctypes.byref(weights), ln_eps, _p(ws), ws_bytes, _p(Y),
                                 _s(stream)), "tp_layer_forward")
+
+
+def tp_reduce_scatter_partials(partials, n_shards, batch, seq, h, bias, residual_shards,
+                               Y_shards, stream=None):
+    _check(lib.tp_reduce_scatter_partials(_p(partials), n_shards, batch, seq, h, _p(bias),
+                                          _p(residual_shards), _p(Y_shards), _s(stream)),
+           "tp_reduce_scatter_partials")
+
+
+def tp_all_gather_sequence(X_shards, n_shards, batch, seq, h, X, stream=None):
+    _check(lib.tp_all_gather_sequence(_p(X_shards), n_shards, batch, seq, h, _p(X), _s(stream)),
+           "tp_all_gather_sequence")
+
+
+def tp_layer_forward_sp(X_shards, batch, seq, h, n_heads, ffn, n_shards,
+                        weights: tp_layer_weights, ln_eps, ws, ws_bytes, Y_shards, stream=None):
+    _check(lib.tp_layer_forward_sp(_p(X_shards), batch, seq, h, n_heads, ffn, n_shards,
+                                   ctypes.byref(weights), ln_eps, _p(ws), ws_bytes, _p(Y_shards),
+                                   _s(stream)), "tp_layer_forward_sp")
 
 
 def tp_get_last_error(stream=None) -> int:
