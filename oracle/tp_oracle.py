@@ -46,6 +46,10 @@ from scipy.special import erf as _erf
 SPLIT_COLUMN = 0
 SPLIT_ROW = 1
 SPLIT_QKV_HEADS = 2
+SPLIT_GATE_UP = 3
+
+# gate / up columns are packed in blocks of this many output features
+GATE_UP_BLOCK = 128
 
 
 # --------------------------------------------------------------------------
@@ -320,6 +324,53 @@ def transformer_layer(X, p: dict, batch: int, seq: int, n_heads: int,
                         batch, seq, n_heads, causal)
     x2 = layernorm(h1, p["ln2_g"], p["ln2_b"], eps)
     return mlp(x2, p["A"], p["b1"], p["B"], p["b2"], h1)
+
+
+# --------------------------------------------------------------------------
+# gated MLP (SwiGLU) ([TP-LLM] MLP block, gated architectures)
+# --------------------------------------------------------------------------
+
+def silu(x: np.ndarray) -> np.ndarray:
+    """SiLU(x) = x * sigmoid(x) = x / (1 + exp(-x))."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / (1.0 + np.exp(-x))
+
+
+def swiglu_mlp(X, W_gate, W_up, B, b2=None, residual=None) -> np.ndarray:
+    """(SiLU(X W_gate) * (X W_up)) B + b2 (+ R), unsharded. [TP-LLM] "For
+    gated architectures like SwiGLU ... SiLU(X W_gate,i) (.) (X W_up,i)"."""
+    return reduce_partials([linear(silu(linear(X, W_gate)) * linear(X, W_up), B)],
+                           b2, residual)
+
+
+def swiglu_mlp_sharded(X, W_gate, W_up, B, b2, residual, n_shards: int) -> np.ndarray:
+    """Gate and up both column-parallel, the gated product local to each
+    shard, B row-parallel, one sum of the partials."""
+    G_i = column_parallel_linear(X, W_gate, None, n_shards)
+    U_i = column_parallel_linear(X, W_up, None, n_shards)
+    A_i = [silu(g) * u for g, u in zip(G_i, U_i)]
+    return reduce_partials(row_parallel_linear(A_i, B, n_shards), b2, residual)
+
+
+def packed_gate_up(W_gate: np.ndarray, W_up: np.ndarray, n_shards: int) -> np.ndarray:
+    """Byte layout of the fused gate/up column-parallel weights: for shard i
+    the column shards W_gate,i and W_up,i (F/N columns each), interleaved in
+    blocks of GATE_UP_BLOCK output features - block k holds gate features
+    [k b, (k+1) b) then the same up features - and stored transposed:
+    shape [N, 2 F/N, h]."""
+    G = shard_matrices(W_gate, SPLIT_COLUMN, n_shards)
+    U = shard_matrices(W_up, SPLIT_COLUMN, n_shards)
+    fs = G[0].shape[1]
+    if fs % GATE_UP_BLOCK:
+        raise ValueError("F/N must be a multiple of the gate/up block")
+    out = []
+    for g, u in zip(G, U):
+        cols = []
+        for k in range(fs // GATE_UP_BLOCK):
+            sl = slice(k * GATE_UP_BLOCK, (k + 1) * GATE_UP_BLOCK)
+            cols += [g[:, sl], u[:, sl]]
+        out.append(np.ascontiguousarray(np.concatenate(cols, axis=1).T))
+    return np.stack(out)
 
 
 # --------------------------------------------------------------------------

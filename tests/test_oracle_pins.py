@@ -456,3 +456,60 @@ def test_sequence_parallel_layer_equals_standard_layer(n):
     ref = O.transformer_layer(X, p, batch, seq, n_heads)
     out = O.transformer_layer_sp(O.sequence_shard(X, batch, seq, n), p, batch, seq, n_heads, n)
     np.testing.assert_allclose(O.all_gather_sequence(out, batch, seq), ref, rtol=1e-11, atol=1e-11)
+
+
+# ---------------------------------------------------------------- SwiGLU
+
+def test_silu_textbook_values():
+    e = math.e
+    for x, ref in [(0.0, 0.0), (1.0, 1.0 / (1.0 + 1.0 / e)), (-1.0, -1.0 / (1.0 + e)),
+                   (2.0, 2.0 / (1.0 + e ** -2))]:
+        assert O.silu(np.array([x]))[0] == pytest.approx(ref, rel=1e-15, abs=1e-300)
+    # SiLU(x) -> x from below for large x (x e^{-x} ~ 2.8e-12 at x = 30)
+    assert 0.0 < 30.0 - O.silu(np.array([30.0]))[0] < 1e-11
+    assert O.silu(np.array([1.0]))[0] == pytest.approx(0.7310585786300049, abs=1e-15)
+    assert abs(O.silu(np.array([-40.0]))[0]) < 1e-15
+
+
+def _brute_swiglu(X, Wg, Wu, B, b2, R):
+    M, h = X.shape
+    F = Wg.shape[1]
+    Y = np.zeros((M, B.shape[1]))
+    for r in range(M):
+        a = []
+        for f in range(F):
+            g = sum(X[r][k] * Wg[k][f] for k in range(h))
+            u = sum(X[r][k] * Wu[k][f] for k in range(h))
+            a.append(g / (1.0 + math.exp(-g)) * u)
+        for c in range(B.shape[1]):
+            Y[r][c] = b2[c] + R[r][c] + sum(a[f] * B[f][c] for f in range(F))
+    return Y
+
+
+@pytest.mark.parametrize("n", [1, 2, 4])
+def test_swiglu_brute_force_and_sharded(n):
+    rng = np.random.default_rng(14)
+    M, h, F = 3, 4, 8
+    X = rng.standard_normal((M, h))
+    Wg, Wu, B = rng.standard_normal((h, F)), rng.standard_normal((h, F)), rng.standard_normal((F, h))
+    b2 = rng.standard_normal(h)
+    ref = _brute_swiglu(X, Wg, Wu, B, b2, X)
+    np.testing.assert_allclose(O.swiglu_mlp(X, Wg, Wu, B, b2, X), ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(O.swiglu_mlp_sharded(X, Wg, Wu, B, b2, X, n), ref,
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_packed_gate_up_layout():
+    rng = np.random.default_rng(15)
+    h, F, n = 3, 2 * 256, 2
+    Wg, Wu = rng.standard_normal((h, F)), rng.standard_normal((h, F))
+    P = O.packed_gate_up(Wg, Wu, n)
+    assert P.shape == (n, 2 * F // n, h)
+    b = O.GATE_UP_BLOCK
+    fs = F // n
+    for i in range(n):
+        for k in range(fs // b):
+            for j in range(b):
+                f = i * fs + k * b + j              # global output feature
+                assert np.array_equal(P[i, 2 * k * b + j], Wg[:, f])
+                assert np.array_equal(P[i, 2 * k * b + b + j], Wu[:, f])
