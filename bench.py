@@ -88,6 +88,10 @@ def work(cfg: dict) -> dict:
         F = cfg["ffn"]
         fl["gemm_column_parallel"] += 2.0 * M * h * F
         fl["gemm_row_parallel"] += 2.0 * M * F * h
+    if kind == "swiglu":
+        F = cfg["ffn"]
+        fl["gemm_column_parallel"] += 2.0 * M * h * 2 * F   # gate and up
+        fl["gemm_row_parallel"] += 2.0 * M * F * h
     partial_read = n * M * h * 4
     act = M * h * 2
     if kind == "layer":
@@ -177,6 +181,9 @@ def oracle_sample(cfg: dict, inp: dict, tokens: int):
     if cfg["kind"] == "layer":
         p = {k: f64(v) for k, v in inp.items() if k != "X"}
         O.transformer_layer(x, p, 1, T, cfg["n_heads"], cfg.get("ln_eps", 1e-5))
+    elif cfg["kind"] == "swiglu":
+        R = x if cfg.get("residual") else None
+        O.swiglu_mlp(x, f64(inp["Wg"]), f64(inp["Wu"]), f64(inp["B"]), f64(inp["b2"]), R)
     elif cfg["kind"] == "attn":
         R = x if cfg.get("residual") else None
         O.self_attention(x, f64(inp["Wqkv"]), f64(inp["bqkv"]), f64(inp["Wo"]), f64(inp["bo"]),
@@ -255,6 +262,12 @@ class Model:
             self.A = shard("A", h, F, 0)
             self.B = shard("B", F, h, 1)
             self.b1, self.b2 = dev["b1"], dev["b2"]
+        if kind == "swiglu":
+            F = cfg["ffn"]
+            dev["GU"] = torch.cat([dev["Wg"].view(h, F), dev["Wu"].view(h, F)], dim=1).contiguous()
+            self.GU = shard("GU", h, 2 * F, 3)
+            self.B = shard("B", F, h, 1)
+            self.b2 = dev["b2"]
         if kind == "layer":
             self.w = tp.make_layer_weights(
                 ln1_gamma=dev["ln1_g"], ln1_beta=dev["ln1_b"], Wqkv_shards=self.Wqkv,
@@ -262,7 +275,8 @@ class Model:
                 ln2_beta=dev["ln2_b"], A_shards=self.A, b1_shards=self.b1, B_shards=self.B,
                 b2=self.b2)
             self.dev_keep = dev
-        wsk = {"mlp": tp.TP_WS_MLP, "attn": tp.TP_WS_ATTN, "layer": tp.TP_WS_LAYER}[kind]
+        wsk = {"mlp": tp.TP_WS_MLP, "swiglu": tp.TP_WS_MLP, "attn": tp.TP_WS_ATTN,
+               "layer": tp.TP_WS_LAYER}[kind]
         self.ws_bytes = tp.tp_workspace_bytes(wsk, self.M, h, cfg.get("ffn", 0), n)
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
         self.Y = torch.empty((self.M, h), dtype=torch.int16, device="cuda")
@@ -280,6 +294,10 @@ class Model:
         elif cfg["kind"] == "layer":
             tp.tp_layer_forward(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"], cfg["ffn"], n,
                                 self.w, cfg.get("ln_eps", 1e-5), self.ws, self.ws_bytes, Y)
+        elif cfg["kind"] == "swiglu":
+            tp.tp_mlp_forward_swiglu(X, self.M, h, cfg["ffn"], n, self.GU, self.B, self.b2,
+                                     X if cfg.get("residual") else None, self.ws, self.ws_bytes,
+                                     Y)
         elif cfg["kind"] == "attn":
             tp.tp_attn_forward(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"],
                                cfg.get("causal", True), n, self.Wqkv, self.bqkv, self.Wo,

@@ -73,7 +73,13 @@ typedef enum {
        heads [i n_h/N, (i+1) n_h/N), head k being columns [k d, (k+1) d) of
        each projection. Packed shard i = [Q_i | K_i | V_i]^T, shape
        [3h/N][H_in]. */
-    TP_SPLIT_QKV_HEADS = 2
+    TP_SPLIT_QKV_HEADS = 2,
+    /* [TP-LLM] MLP block, gated architectures: W = [W_gate | W_up]
+       (H_out = 2F), both projections column-parallel. Shard i's columns
+       alternate 128 gate features and the same 128 up features (block k =
+       gate features [k 128, (k+1) 128) of the shard, then the same up
+       features). Packed shard i shape [2F/N][H_in]; F/N % 128 == 0. */
+    TP_SPLIT_GATE_UP = 3
 } tp_split;
 
 typedef enum {
@@ -81,7 +87,12 @@ typedef enum {
     /* GeLU(x) = 0.5 x (1 + erf(x / sqrt 2)), applied per column shard
        ([TP-LLM] "Column-Parallel Linear Layer": an element-wise function is
        applied to the local slice; [M-LM] step 1). */
-    TP_ACT_GELU_ERF = 1
+    TP_ACT_GELU_ERF = 1,
+    /* Gated: with TP_SPLIT_GATE_UP weights, Y_i = SiLU(X W_gate,i) *
+       (X W_up,i), SiLU(x) = x / (1 + e^-x) ([TP-LLM] MLP block: the gated
+       product is local to each shard). Y_shards then has F/N = H_out/(2N)
+       columns per shard; no bias. */
+    TP_ACT_SWIGLU = 2
 } tp_act;
 
 typedef enum { TP_WS_MLP = 0, TP_WS_ATTN = 1, TP_WS_LAYER = 2, TP_WS_LAYER_SP = 3 } tp_ws_kind;
@@ -129,12 +140,29 @@ tp_status tp_shard_index_map(int kind, int64_t h_in, int64_t h_out,
  * communication; element-wise activation on the local slice).
  * X [B][H_in]; W_shards [N][H_out/N][H_in] (packed); bias_shards [N][H_out/N]
  * or NULL; Y_shards [N][B][H_out/N] (shard-major: the column gather of
- * [INTRO] is a view, not a copy). H_in and H_out/N must be multiples of 8. */
+ * [INTRO] is a view, not a copy). H_in and H_out/N must be multiples of 8.
+ * With act = TP_ACT_SWIGLU: W_shards is TP_SPLIT_GATE_UP-packed, H_out = 2F
+ * counts gate and up columns, (H_out/N) % 256 == 0, bias_shards must be NULL
+ * and Y_shards is [N][B][H_out/(2N)]. */
 tp_status tp_column_linear(const uint16_t* X, int64_t B, int64_t h_in,
                            const uint16_t* W_shards,
                            const uint16_t* bias_shards, int64_t h_out,
                            int n_shards, int act, uint16_t* Y_shards,
                            void* stream);
+
+/* tp_mlp_forward_swiglu - Y = (SiLU(X W_gate) * (X W_up)) B + b2 + residual
+ * by the tensor-parallel route: gate and up column-parallel with the gated
+ * product fused into the GEMM epilogue, B row-parallel into N partials, one
+ * sum ([TP-LLM] MLP block, gated architectures). X [B][h]; GU_shards
+ * TP_SPLIT_GATE_UP of [h][2F]: [N][2F/N][h]; B_shards [N][h][F/N]; b2 [h] or
+ * NULL; residual [B][h] or NULL; Y [B][h]. F/N % 128 == 0.
+ * ws >= tp_workspace_bytes(TP_WS_MLP, B, h, F, N). */
+tp_status tp_mlp_forward_swiglu(const uint16_t* X, int64_t B, int64_t h,
+                                int64_t ffn, int n_shards,
+                                const uint16_t* GU_shards,
+                                const uint16_t* B_shards, const uint16_t* b2,
+                                const uint16_t* residual, void* ws,
+                                size_t ws_bytes, uint16_t* Y, void* stream);
 
 /* tp_row_linear - partials P_i = X_i W_i (each B x H_out, fp32), one launch.
  * [TP-LLM] "Row-Parallel Linear Layer" (X = [X_1 ... X_N] along channels,

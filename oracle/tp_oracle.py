@@ -136,6 +136,23 @@ def shard_index_map(kind: int, h_in: int, h_out: int, n_shards: int,
         owner = head // (n_heads // n_shards)
         local = part * hs + (within_part - owner * hs)
         return owner, local
+    if kind == SPLIT_GATE_UP:
+        # W = [W_gate | W_up] (h_out = 2F): both column-parallel; a shard's
+        # columns alternate GATE_UP_BLOCK gate features and the same up ones
+        if h_out % 2 != 0:
+            raise ValueError("gate/up weight must have 2F columns")
+        F = h_out // 2
+        _check_div("F", F, n_shards)
+        fs = F // n_shards
+        if fs % GATE_UP_BLOCK != 0:
+            raise ValueError("F/N must be a multiple of the gate/up block")
+        j = np.arange(h_out, dtype=np.int64)
+        part, f = j // F, j % F                # part 0 = gate, 1 = up
+        owner = f // fs
+        within = f % fs
+        local = (within // GATE_UP_BLOCK) * 2 * GATE_UP_BLOCK + part * GATE_UP_BLOCK + \
+            within % GATE_UP_BLOCK
+        return owner, local
     raise ValueError(f"unknown split kind {kind}")
 
 

@@ -70,7 +70,13 @@ struct GemmParams {
   unsigned* err;
 };
 
-template <int BN, bool OUT_F32, int CTAS>
+// Epilogue kinds: bf16 + bias + activation (column-parallel), fp32 partials
+// (row-parallel), gated SiLU(gate) * up over interleaved 128-column blocks.
+enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU = 2 };
+
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + __expf(-x)); }
+
+template <int BN, int EPI, int CTAS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -254,6 +260,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // issues a TMA tensor store of the 32-row box (rows/columns outside the
     // output are clipped by the TMA unit). The next chunk's TMEM load is in
     // flight while the current chunk is converted and stored.
+    constexpr bool OUT_F32 = EPI == EPI_F32;
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const uint32_t sbase =
@@ -278,6 +285,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int colh = nb * BN + half * (BN / 2);
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + half * (BN / 2));
+      if constexpr (EPI == EPI_SWIGLU) {
+        // tile columns [0, 128) are gate features, [128, 256) the same up
+        // features; this warp forms output features [64 half, 64 half + 64)
+        // of the tile's 128, i.e. columns (nb * 128 + 64 half) of the output.
+        const int ocol0 = nb * (BN / 2) + half * 64;
+        const uint32_t gbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(acc * BN + half * 64);
+        uint32_t w[32];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          uint32_t gv[32], uv[32];
+          tmem_ld_32x32b_x32(gbase + part * 32, gv);
+          tmem_ld_32x32b_x32(gbase + BN / 2 + part * 32, uv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float a = silu(__uint_as_float(gv[e])) * __uint_as_float(uv[e]);
+            const float b = silu(__uint_as_float(gv[e + 1])) * __uint_as_float(uv[e + 1]);
+            w[part * 16 + (e >> 1)] = pack_bf16x2(a, b);
+          }
+        }
+        if (ocol0 < p.Nc / 2) {
+          const uint32_t sbuf = sbase + (chunk_ctr % C::kStagingBufs) * 4096u;
+          ++chunk_ctr;
+          if (lane == 0) bulk_wait_read<C::kStagingBufs - 1>();
+          __syncwarp();
+          const uint32_t row_addr = sbuf + static_cast<uint32_t>(lane) * 128u;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4), w[4 * j],
+                         w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmD, sbuf, ocol0, row0, g);
+            bulk_commit();
+          }
+        }
+      } else {
       uint32_t r[2][CW];
       tmem_ld_32x32b_x32(tbase, &r[0][0]);
       if constexpr (!OUT_F32) tmem_ld_32x32b_x32(tbase + 32, &r[0][32]);
@@ -336,6 +382,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           bulk_commit();
         }
       }
+      }  // EPI
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -404,13 +451,15 @@ static bool encode_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool OUT_F32, int CTAS>
+template <int BN, int EPI, int CTAS>
 static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, int num_sms) {
   using C = GemmCfg<BN, CTAS>;
+  constexpr bool OUT_F32 = EPI == EPI_F32;
   CUtensorMap tmA, tmB, tmD;
   if (!encode_3d(&tmA, pr.A, pr.K, pr.M, pr.a_batched ? pr.G : 1, BK, BM)) return 1;
   if (!encode_3d(&tmB, pr.B, pr.K, pr.Nc, pr.G, BK, C::kBRows)) return 1;
-  if (!encode_3d(&tmD, pr.D, pr.Nc, pr.M, pr.G, OUT_F32 ? 32 : 64, 32, OUT_F32)) return 1;
+  const uint64_t out_cols = (EPI == EPI_SWIGLU) ? pr.Nc / 2 : pr.Nc;
+  if (!encode_3d(&tmD, pr.D, out_cols, pr.M, pr.G, OUT_F32 ? 32 : 64, 32, OUT_F32)) return 1;
   GemmParams p;
   p.M = pr.M;
   p.Nc = pr.Nc;
@@ -424,7 +473,7 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
   p.act = pr.act;
   p.bias = static_cast<const uint16_t*>(pr.bias);
   p.err = err;
-  auto kern = gemm_tcgen05_kernel<BN, OUT_F32, CTAS>;
+  auto kern = gemm_tcgen05_kernel<BN, EPI, CTAS>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kGemmThreads);
@@ -461,14 +510,18 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
 int launch_gemm(const GemmProblem& p, cudaStream_t s, unsigned* err, int num_sms) {
   const bool wide = p.Nc > 128;
   const bool pair = wide && p.M > BM;  // 256-row tiles only when there are rows to fill them
-  if (p.out_f32) {
-    if (pair) return launch_gemm_t<256, true, 2>(p, s, err, num_sms);
-    return wide ? launch_gemm_t<256, true, 1>(p, s, err, num_sms)
-                : launch_gemm_t<128, true, 1>(p, s, err, num_sms);
+  if (p.act == 2) {  // gated: 256-wide tiles always (128 gate + 128 up columns)
+    return p.M > BM ? launch_gemm_t<256, EPI_SWIGLU, 2>(p, s, err, num_sms)
+                    : launch_gemm_t<256, EPI_SWIGLU, 1>(p, s, err, num_sms);
   }
-  if (pair) return launch_gemm_t<256, false, 2>(p, s, err, num_sms);
-  return wide ? launch_gemm_t<256, false, 1>(p, s, err, num_sms)
-              : launch_gemm_t<128, false, 1>(p, s, err, num_sms);
+  if (p.out_f32) {
+    if (pair) return launch_gemm_t<256, EPI_F32, 2>(p, s, err, num_sms);
+    return wide ? launch_gemm_t<256, EPI_F32, 1>(p, s, err, num_sms)
+                : launch_gemm_t<128, EPI_F32, 1>(p, s, err, num_sms);
+  }
+  if (pair) return launch_gemm_t<256, EPI_BF16, 2>(p, s, err, num_sms);
+  return wide ? launch_gemm_t<256, EPI_BF16, 1>(p, s, err, num_sms)
+              : launch_gemm_t<128, EPI_BF16, 1>(p, s, err, num_sms);
 }
 
 }  // namespace tpk

@@ -4,6 +4,11 @@
 // attention "Q, K, V Projections": W_Q, W_K, W_V sliced by whole heads),
 // each shard stored transposed (K-major) as the GEMM kernels read it.
 //
+// A fourth kind packs the gate and up projections of a gated MLP (given as
+// one [h][2F] matrix [W_gate | W_up]) so that each shard's columns alternate
+// 128 gate features and the same 128 up features ("Partitioning the
+// Multi-Layer Perceptron (MLP) Block": gate and up are both column-parallel).
+//
 // out[i][c][r] = W[row(i, r)][col(i, c)], an exact copy done as a 32 x 32
 // shared-memory tiled transpose (coalesced reads along W's columns,
 // coalesced writes along the shard's rows). One-time setup, HBM-bound.
@@ -15,10 +20,12 @@ namespace tpk {
 struct ShardMap {
   int64_t h_in, h_out;
   int64_t C, R;  // shard shape [C][R]
-  int kind;      // 0 column, 1 row, 2 qkv heads
-  int64_t hs;    // QKV: columns of one projection per shard (h / N)
-  int64_t h3;    // QKV: h (columns of one projection)
+  int kind;      // 0 column, 1 row, 2 qkv heads, 3 gate/up interleaved
+  int64_t hs;    // QKV: columns of one projection per shard (h / N); gate/up: F / N
+  int64_t h3;    // QKV: h (columns of one projection); gate/up: F
 };
+
+constexpr int kGateUpBlock = 128;  // output features per gate (or up) block
 
 __device__ __forceinline__ int64_t src_row(const ShardMap& m, int i, int64_t r) {
   return m.kind == 1 ? static_cast<int64_t>(i) * m.R + r : r;
@@ -26,6 +33,12 @@ __device__ __forceinline__ int64_t src_row(const ShardMap& m, int i, int64_t r) 
 __device__ __forceinline__ int64_t src_col(const ShardMap& m, int i, int64_t c) {
   if (m.kind == 0) return static_cast<int64_t>(i) * m.C + c;
   if (m.kind == 1) return c;
+  if (m.kind == 3) {
+    // block k of 2 x 128 shard columns: gate features k*128.., then up features
+    const int64_t k = c / (2 * kGateUpBlock), w = c - k * 2 * kGateUpBlock;
+    const int64_t f = static_cast<int64_t>(i) * m.hs + k * kGateUpBlock + (w % kGateUpBlock);
+    return (w < kGateUpBlock) ? f : m.h3 + f;
+  }
   const int64_t part = c / m.hs, within = c - part * m.hs;
   return part * m.h3 + static_cast<int64_t>(i) * m.hs + within;
 }
@@ -67,10 +80,15 @@ int launch_shard(const void* W, int64_t h_in, int64_t h_out, int n_shards, int k
   } else if (kind == 1) {
     m.C = h_out;
     m.R = h_in / n_shards;
-  } else {
+  } else if (kind == 2) {
     m.h3 = h_out / 3;
     m.hs = m.h3 / n_shards;
     m.C = 3 * m.hs;
+    m.R = h_in;
+  } else {
+    m.h3 = h_out / 2;          // F
+    m.hs = m.h3 / n_shards;    // F / N
+    m.C = 2 * m.hs;
     m.R = h_in;
   }
   const dim3 grid(static_cast<unsigned>((m.R + 31) / 32), static_cast<unsigned>((m.C + 31) / 32),

@@ -209,6 +209,18 @@ tp_status tp_shard_index_map(int kind, int64_t h_in, int64_t h_out, int n_shards
     }
     return TP_OK;
   }
+  if (kind == TP_SPLIT_GATE_UP) {
+    if (h_out % 2) return TP_ERR_SHAPE;
+    const int64_t F = h_out / 2;
+    if (F % n_shards || (F / n_shards) % 128) return TP_ERR_SHAPE;
+    const int64_t fs = F / n_shards;
+    for (int64_t j = 0; j < h_out; ++j) {
+      const int64_t part = j / F, f = j % F, within = f % fs;
+      host_owner[j] = static_cast<int32_t>(f / fs);
+      host_local[j] = (within / 128) * 256 + part * 128 + within % 128;
+    }
+    return TP_OK;
+  }
   if (kind == TP_SPLIT_QKV_HEADS) {
     if (h_out % 3 || head_dim <= 0) return TP_ERR_SHAPE;
     const int64_t h = h_out / 3;
@@ -238,6 +250,8 @@ tp_status tp_shard_weights(const uint16_t* W, int64_t h_in, int64_t h_out, int n
   } else if (kind == TP_SPLIT_QKV_HEADS) {
     if (h_out % 3 || head_dim <= 0 || (h_out / 3) % head_dim || ((h_out / 3) / head_dim) % n_shards)
       return TP_ERR_SHAPE;
+  } else if (kind == TP_SPLIT_GATE_UP) {
+    if (h_out % 2 || (h_out / 2) % n_shards || ((h_out / 2) / n_shards) % 128) return TP_ERR_SHAPE;
   } else {
     return TP_ERR_SHAPE;
   }
@@ -262,7 +276,9 @@ tp_status tp_column_linear(const uint16_t* X, int64_t B, int64_t h_in, const uin
   const int64_t nc = h_out / n_shards;
   if (h_in % 8 || nc % 8) return TP_ERR_SHAPE;
   if (B > kIntMax || h_in > kIntMax || nc > kIntMax) return TP_ERR_SHAPE;
-  if (act != TP_ACT_NONE && act != TP_ACT_GELU_ERF) return TP_ERR_UNSUPPORTED;
+  if (act != TP_ACT_NONE && act != TP_ACT_GELU_ERF && act != TP_ACT_SWIGLU)
+    return TP_ERR_UNSUPPORTED;
+  if (act == TP_ACT_SWIGLU && (nc % 256 || bias_shards != nullptr)) return TP_ERR_UNSUPPORTED;
   if (!al16(X) || !al16(W_shards) || !al16(Y_shards) || (bias_shards && !al16(bias_shards)))
     return TP_ERR_ALIGN;
   DevInfo d;
@@ -425,6 +441,29 @@ tp_status tp_mlp_forward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, i
   uint16_t* act = reinterpret_cast<uint16_t*>(w);
   float* part = reinterpret_cast<float*>(w + round256(static_cast<size_t>(B) * ffn * 2));
   tp_status st = tp_column_linear(X, B, h, A_shards, b1_shards, ffn, n_shards, TP_ACT_GELU_ERF,
+                                  act, stream);
+  if (st != TP_OK) return st;
+  st = tp_row_linear(act, B, ffn, B_shards, h, n_shards, part, stream);
+  if (st != TP_OK) return st;
+  return tp_reduce_partials(part, n_shards, B, h, b2, residual, Y, stream);
+}
+
+tp_status tp_mlp_forward_swiglu(const uint16_t* X, int64_t B, int64_t h, int64_t ffn,
+                                int n_shards, const uint16_t* GU_shards,
+                                const uint16_t* B_shards, const uint16_t* b2,
+                                const uint16_t* residual, void* ws, size_t ws_bytes, uint16_t* Y,
+                                void* stream) {
+  if (X == nullptr || GU_shards == nullptr || B_shards == nullptr || Y == nullptr || ws == nullptr)
+    return TP_ERR_NULL;
+  if (B <= 0 || h <= 0 || ffn <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (ffn % n_shards || (ffn / n_shards) % 128 || h % 8) return TP_ERR_SHAPE;
+  const size_t need = tp_workspace_bytes(TP_WS_MLP, B, h, ffn, n_shards);
+  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  if (!al16(ws)) return TP_ERR_ALIGN;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* act = reinterpret_cast<uint16_t*>(w);
+  float* part = reinterpret_cast<float*>(w + round256(static_cast<size_t>(B) * ffn * 2));
+  tp_status st = tp_column_linear(X, B, h, GU_shards, nullptr, 2 * ffn, n_shards, TP_ACT_SWIGLU,
                                   act, stream);
   if (st != TP_OK) return st;
   st = tp_row_linear(act, B, ffn, B_shards, h, n_shards, part, stream);

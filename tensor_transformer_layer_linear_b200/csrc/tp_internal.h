@@ -31,7 +31,7 @@ struct GemmProblem {
   int M, Nc, K, G;
   bool a_batched;
   bool out_f32;
-  int act;  // 0 none, 1 GeLU (erf form)
+  int act;  // 0 none, 1 GeLU (erf form), 2 gated SiLU(gate) * up (D has Nc / 2 columns)
 };
 
 // Returns 0 on success, 1 if a tensor map could not be encoded, 2 if the

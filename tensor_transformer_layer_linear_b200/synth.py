@@ -18,7 +18,8 @@ The five workloads are the shapes of the Megatron-LM tensor-parallel MLP,
 attention and layer examples: the page-1 worked example
 (Linear(1024 -> 4096) on 32 tokens, tensor_model_parallel_size = 2), a
 4 x 2048-token MLP, a 16-head causal attention block, a full pre-LN layer,
-and a large MLP swept over shard counts.
+and a large MLP swept over shard counts. A gated (SwiGLU) MLP of the
+4 x 2048-token MLP's shape is added for the gated variant.
 """
 from __future__ import annotations
 
@@ -39,6 +40,9 @@ CONFIGS = {
         kind="layer", batch=2, seq=2048, h=4096, n_heads=32, ffn=16384,
         n_shards=8, causal=True, x_std=1.0, w_std=0.02, b_std=0.01,
         ln_eps=1e-5),
+    "swiglu_8192x1024_f4096_n4": dict(
+        kind="swiglu", batch=4, seq=2048, h=1024, ffn=4096, n_shards=4,
+        x_std=1.0, w_std=0.02, b_std=0.01, residual=True),
     "mlp_2048x12288_f49152_sweep": dict(
         kind="mlp", batch=1, seq=2048, h=12288, ffn=49152, n_shards=1,
         sweep=(1, 2, 4, 8, 16), x_std=0.02, w_std=0.02, b_std=0.0,
@@ -85,7 +89,8 @@ def make_inputs(cfg: dict, seed: int = 0) -> dict:
     Returns a dict of uint16 arrays (bf16 bits), row-major:
       X [M, h]; MLP: A [h, F], b1 [F], B [F, h], b2 [h];
       attention: Wqkv [h, 3h] (= [W_Q | W_K | W_V]), bqkv [3h], Wo [h, h], bo [h];
-      layer: both sets plus ln1_g, ln1_b, ln2_g, ln2_b [h].
+      layer: both sets plus ln1_g, ln1_b, ln2_g, ln2_b [h];
+      swiglu (gated MLP): Wg, Wu [h, F], B [F, h], b2 [h].
     """
     rng = np.random.Generator(np.random.Philox(seed))
     kind = cfg["kind"]
@@ -100,6 +105,12 @@ def make_inputs(cfg: dict, seed: int = 0) -> dict:
         F = cfg["ffn"]
         out["A"] = _draw(rng, (h, F), w)
         out["B"] = _draw(rng, (F, h), w)
+    if kind == "swiglu":
+        F = cfg["ffn"]
+        out["Wg"] = _draw(rng, (h, F), w)
+        out["Wu"] = _draw(rng, (h, F), w)
+        out["B"] = _draw(rng, (F, h), w)
+        out["b2"] = _draw(rng, (h,), b)
     if kind in ("attn", "layer"):
         out["bqkv"] = _draw(rng, (3 * h,), b)
         out["bo"] = _draw(rng, (h,), b)

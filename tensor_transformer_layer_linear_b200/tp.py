@@ -29,8 +29,8 @@ lib = ctypes.CDLL(LIB_PATH)
 # status codes and enums (include/tp.h)
 TP_OK, TP_ERR_NULL, TP_ERR_SHAPE, TP_ERR_ALIGN = 0, 1, 2, 3
 TP_ERR_WORKSPACE, TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_TIMEOUT = 4, 5, 6, 7
-TP_SPLIT_COLUMN, TP_SPLIT_ROW, TP_SPLIT_QKV_HEADS = 0, 1, 2
-TP_ACT_NONE, TP_ACT_GELU_ERF = 0, 1
+TP_SPLIT_COLUMN, TP_SPLIT_ROW, TP_SPLIT_QKV_HEADS, TP_SPLIT_GATE_UP = 0, 1, 2, 3
+TP_ACT_NONE, TP_ACT_GELU_ERF, TP_ACT_SWIGLU = 0, 1, 2
 TP_WS_MLP, TP_WS_ATTN, TP_WS_LAYER, TP_WS_LAYER_SP = 0, 1, 2, 3
 
 _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -58,6 +58,8 @@ _SIGS = {
                                _vp, _sz, _vp, _vp]),
     "tp_layer_forward": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32,
                                 ctypes.POINTER(tp_layer_weights), _f32, _vp, _sz, _vp, _vp]),
+    "tp_mlp_forward_swiglu": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _sz,
+                                     _vp, _vp]),
     "tp_mlp_forward_noalloc": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                       _vp]),
     "tp_reduce_scatter_partials": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
@@ -179,6 +181,13 @@ def tp_mlp_forward(X, B, h, ffn, n_shards, A_shards, b1_shards, B_shards, b2, re
     _check(lib.tp_mlp_forward(_p(X), B, h, ffn, n_shards, _p(A_shards), _p(b1_shards),
                               _p(B_shards), _p(b2), _p(residual), _p(ws), ws_bytes, _p(Y),
                               _s(stream)), "tp_mlp_forward")
+
+
+def tp_mlp_forward_swiglu(X, B, h, ffn, n_shards, GU_shards, B_shards, b2, residual, ws,
+                          ws_bytes, Y, stream=None):
+    _check(lib.tp_mlp_forward_swiglu(_p(X), B, h, ffn, n_shards, _p(GU_shards), _p(B_shards),
+                                     _p(b2), _p(residual), _p(ws), ws_bytes, _p(Y), _s(stream)),
+           "tp_mlp_forward_swiglu")
 
 
 TP_NOALLOC_WS_BYTES = 32 * 1024 * 1024

@@ -28,7 +28,8 @@ def test_status_strings():
     assert "unknown" in tp.tp_status_string(99)
 
 
-@pytest.mark.parametrize("kind", [tp.TP_SPLIT_COLUMN, tp.TP_SPLIT_ROW, tp.TP_SPLIT_QKV_HEADS])
+@pytest.mark.parametrize("kind", [tp.TP_SPLIT_COLUMN, tp.TP_SPLIT_ROW, tp.TP_SPLIT_QKV_HEADS,
+                                  tp.TP_SPLIT_GATE_UP])
 @pytest.mark.parametrize("n", [1, 2, 4, 8, 16])
 def test_index_map_matches_oracle(kind, n):
     h, d = 2048, 128

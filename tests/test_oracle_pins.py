@@ -513,3 +513,13 @@ def test_packed_gate_up_layout():
                 f = i * fs + k * b + j              # global output feature
                 assert np.array_equal(P[i, 2 * k * b + j], Wg[:, f])
                 assert np.array_equal(P[i, 2 * k * b + b + j], Wu[:, f])
+
+
+def test_gate_up_index_map_matches_packing():
+    rng = np.random.default_rng(16)
+    h, F, n = 3, 2 * 256, 2
+    Wg, Wu = rng.standard_normal((h, F)), rng.standard_normal((h, F))
+    W = np.concatenate([Wg, Wu], axis=1)
+    assert np.array_equal(O.packed_shards(W, O.SPLIT_GATE_UP, n), O.packed_gate_up(Wg, Wu, n))
+    with pytest.raises(ValueError):
+        O.shard_index_map(O.SPLIT_GATE_UP, h, 2 * 192, 2)   # F/N = 96 not a block multiple
