@@ -391,6 +391,97 @@ def packed_gate_up(W_gate: np.ndarray, W_up: np.ndarray, n_shards: int) -> np.nd
 
 
 # --------------------------------------------------------------------------
+# grouped-query attention ([TP-LLM] "Grouped-Query Attention (GQA)
+# Constraints")
+# --------------------------------------------------------------------------
+#
+# W_QKV = [W_Q | W_K | W_V] with n_q query heads and n_kv key/value heads of
+# dimension d (W_Q: h x n_q d, W_K, W_V: h x n_kv d); query head j uses
+# key/value head j // (n_q / n_kv). Sharding keeps whole groups local: with
+# n_kv % N == 0 shard i owns query heads [i n_q/N, (i+1) n_q/N) and kv heads
+# [i n_kv/N, (i+1) n_kv/N); with N > n_kv (N % n_kv == 0) each shard owns
+# n_q/N query heads, all in one group, and a copy of that group's kv head
+# (the duplication the page allows). Shard i's columns: [Q_i | K_i | V_i].
+
+def gqa_kv_local(n_kv: int, n_shards: int) -> int:
+    if n_shards <= n_kv:
+        _check_div("n_kv", n_kv, n_shards)
+        return n_kv // n_shards
+    _check_div("N", n_shards, n_kv)
+    return 1
+
+
+def gqa_shard_columns(n_q: int, n_kv: int, d: int, n_shards: int) -> list:
+    """For each shard, the W_QKV column indices of [Q_i | K_i | V_i]."""
+    _check_div("n_q", n_q, n_shards)
+    if n_q % n_kv:
+        raise ValueError("n_q must be a multiple of n_kv")
+    qs, kvl = n_q // n_shards, gqa_kv_local(n_kv, n_shards)
+    kv0 = n_q * d                      # first K column
+    v0 = kv0 + n_kv * d                # first V column
+    out = []
+    for i in range(n_shards):
+        q_heads = range(i * qs, (i + 1) * qs)
+        first_kv = (i * qs) // (n_q // n_kv)
+        kv_heads = range(first_kv, first_kv + kvl)
+        cols = [k * d + e for k in q_heads for e in range(d)]
+        cols += [kv0 + k * d + e for k in kv_heads for e in range(d)]
+        cols += [v0 + k * d + e for k in kv_heads for e in range(d)]
+        out.append(np.asarray(cols, dtype=np.int64))
+    return out
+
+
+def packed_gqa_shards(Wqkv: np.ndarray, n_q: int, n_kv: int, d: int,
+                      n_shards: int) -> np.ndarray:
+    """Byte layout of GQA QKV shards: [N, (n_q/N + 2 kv_local) d, h_in]."""
+    return np.stack([np.ascontiguousarray(Wqkv[:, c].T)
+                     for c in gqa_shard_columns(n_q, n_kv, d, n_shards)])
+
+
+def gqa_attention_heads(Q, K, V, batch: int, seq: int, n_q: int, n_kv: int,
+                        causal: bool) -> np.ndarray:
+    """Query head j attends with key/value head j // (n_q / n_kv)."""
+    d = Q.shape[1] // n_q
+    g = n_q // n_kv
+    O = np.zeros((Q.shape[0], n_q * d))
+    for s in range(batch):
+        r = slice(s * seq, (s + 1) * seq)
+        for j in range(n_q):
+            c = slice(j * d, (j + 1) * d)
+            kc = slice((j // g) * d, (j // g + 1) * d)
+            O[r, c] = attention_head(Q[r, c], K[r, kc], V[r, kc], causal)
+    return O
+
+
+def gqa_self_attention(X, Wqkv, bqkv, Wo, bo, residual, batch: int, seq: int,
+                       n_q: int, n_kv: int, causal: bool = True) -> np.ndarray:
+    """Unsharded GQA block: Y = concat_j head_j W_O + b_O (+ R)."""
+    d = Wo.shape[0] // n_q
+    QKV = linear(X, Wqkv, bqkv)
+    Q = QKV[:, :n_q * d]
+    K = QKV[:, n_q * d:(n_q + n_kv) * d]
+    V = QKV[:, (n_q + n_kv) * d:]
+    O = gqa_attention_heads(Q, K, V, batch, seq, n_q, n_kv, causal)
+    return reduce_partials([linear(O, Wo)], bo, residual)
+
+
+def gqa_self_attention_sharded(X, Wqkv, bqkv, Wo, bo, residual, batch: int,
+                               seq: int, n_q: int, n_kv: int, n_shards: int,
+                               causal: bool = True) -> np.ndarray:
+    """The tensor-parallel route for GQA: each shard projects its query heads
+    and its (possibly duplicated) kv heads, attends locally, and W_O is
+    row-parallel over the query heads; one sum of the partials."""
+    d = Wo.shape[0] // n_q
+    qs, kvl = n_q // n_shards, gqa_kv_local(n_kv, n_shards)
+    O_i = []
+    for cols in gqa_shard_columns(n_q, n_kv, d, n_shards):
+        q = linear(X, Wqkv[:, cols], None if bqkv is None else bqkv[cols])
+        O_i.append(gqa_attention_heads(q[:, :qs * d], q[:, qs * d:(qs + kvl) * d],
+                                       q[:, (qs + kvl) * d:], batch, seq, qs, kvl, causal))
+    return reduce_partials(row_parallel_linear(O_i, Wo, n_shards), bo, residual)
+
+
+# --------------------------------------------------------------------------
 # sequence parallelism ([TP-LLM] "Sequence Parallelism")
 # --------------------------------------------------------------------------
 #

@@ -523,3 +523,70 @@ def test_gate_up_index_map_matches_packing():
     assert np.array_equal(O.packed_shards(W, O.SPLIT_GATE_UP, n), O.packed_gate_up(Wg, Wu, n))
     with pytest.raises(ValueError):
         O.shard_index_map(O.SPLIT_GATE_UP, h, 2 * 192, 2)   # F/N = 96 not a block multiple
+
+
+
+# ---------------------------------------------------------------- grouped-query attention
+
+def _gqa_params(rng, h, n_q, n_kv, d):
+    cols = (n_q + 2 * n_kv) * d
+    return (rng.standard_normal((h, cols)) * .3, rng.standard_normal(cols) * .1,
+            rng.standard_normal((n_q * d, h)) * .3, rng.standard_normal(h) * .1)
+
+
+def test_gqa_with_all_kv_heads_is_multi_head_attention():
+    rng = np.random.default_rng(17)
+    batch, seq, n, d = 2, 6, 4, 3
+    h = n * d
+    X = rng.standard_normal((batch * seq, h))
+    Wqkv, bqkv, Wo, bo = _gqa_params(rng, h, n, n, d)
+    np.testing.assert_allclose(
+        O.gqa_self_attention(X, Wqkv, bqkv, Wo, bo, X, batch, seq, n, n),
+        O.self_attention(X, Wqkv, bqkv, Wo, bo, X, batch, seq, n), rtol=1e-12, atol=1e-12)
+
+
+def test_gqa_brute_force_shared_kv():
+    """Every query head of a group sees the same K, V: a brute-force loop
+    that uses head j // g explicitly."""
+    rng = np.random.default_rng(18)
+    batch, seq, n_q, n_kv, d = 1, 5, 4, 2, 2
+    Q = rng.standard_normal((seq, n_q * d))
+    K = rng.standard_normal((seq, n_kv * d))
+    V = rng.standard_normal((seq, n_kv * d))
+    out = O.gqa_attention_heads(Q, K, V, batch, seq, n_q, n_kv, True)
+    for j in range(n_q):
+        kv = j // (n_q // n_kv)
+        for t in range(seq):
+            sc = [sum(Q[t, j * d + e] * K[u, kv * d + e] for e in range(d)) / math.sqrt(d)
+                  for u in range(t + 1)]
+            m = max(sc)
+            w = [math.exp(x - m) for x in sc]
+            for e in range(d):
+                ref = sum(w[u] * V[u, kv * d + e] for u in range(t + 1)) / sum(w)
+                assert abs(out[t, j * d + e] - ref) < 1e-12
+
+
+@pytest.mark.parametrize("n_q,n_kv,n", [(8, 2, 1), (8, 2, 2), (8, 4, 4), (8, 2, 4), (8, 1, 8),
+                                        (8, 2, 8)])
+def test_gqa_sharded_equals_unsharded(n_q, n_kv, n):
+    """Including N > n_kv, where kv heads are duplicated across shards."""
+    rng = np.random.default_rng(19)
+    batch, seq, d = 2, 5, 2
+    h = n_q * d
+    X = rng.standard_normal((batch * seq, h))
+    Wqkv, bqkv, Wo, bo = _gqa_params(rng, h, n_q, n_kv, d)
+    np.testing.assert_allclose(
+        O.gqa_self_attention_sharded(X, Wqkv, bqkv, Wo, bo, X, batch, seq, n_q, n_kv, n),
+        O.gqa_self_attention(X, Wqkv, bqkv, Wo, bo, X, batch, seq, n_q, n_kv),
+        rtol=1e-12, atol=1e-12)
+
+
+def test_gqa_shard_columns_and_constraints():
+    cols = O.gqa_shard_columns(8, 2, 1, 4)      # N = 4 > n_kv = 2: duplication
+    # shard 0, 1 use kv head 0; shards 2, 3 kv head 1 (K at 8 + kv, V at 10 + kv)
+    assert [c.tolist() for c in cols] == [[0, 1, 8, 10], [2, 3, 8, 10], [4, 5, 9, 11],
+                                         [6, 7, 9, 11]]
+    with pytest.raises(ValueError):
+        O.gqa_shard_columns(8, 4, 1, 3)          # 8 % 3
+    with pytest.raises(ValueError):
+        O.gqa_kv_local(4, 6)                     # N = 6 neither divides nor is divided by 4
