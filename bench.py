@@ -88,6 +88,12 @@ def work(cfg: dict) -> dict:
         F = cfg["ffn"]
         fl["gemm_column_parallel"] += 2.0 * M * h * F
         fl["gemm_row_parallel"] += 2.0 * M * F * h
+    if kind == "attn_gqa":
+        d = h // cfg["n_heads"]
+        fl["gemm_column_parallel"] += 2.0 * M * h * (cfg["n_heads"] + 2 * cfg["n_kv_heads"]) * d
+        fl["attention"] += 4.0 * cfg["seq"] ** 2 * d * cfg["n_heads"] * cfg["batch"] / (
+            2 if cfg.get("causal", True) else 1)
+        fl["gemm_row_parallel"] += 2.0 * M * h * h
     if kind == "swiglu":
         F = cfg["ffn"]
         fl["gemm_column_parallel"] += 2.0 * M * h * 2 * F   # gate and up
@@ -181,6 +187,11 @@ def oracle_sample(cfg: dict, inp: dict, tokens: int):
     if cfg["kind"] == "layer":
         p = {k: f64(v) for k, v in inp.items() if k != "X"}
         O.transformer_layer(x, p, 1, T, cfg["n_heads"], cfg.get("ln_eps", 1e-5))
+    elif cfg["kind"] == "attn_gqa":
+        R = x if cfg.get("residual") else None
+        O.gqa_self_attention(x, f64(inp["Wqkv"]), f64(inp["bqkv"]), f64(inp["Wo"]),
+                             f64(inp["bo"]), R, 1, T, cfg["n_heads"], cfg["n_kv_heads"],
+                             cfg.get("causal", True))
     elif cfg["kind"] == "swiglu":
         R = x if cfg.get("residual") else None
         O.swiglu_mlp(x, f64(inp["Wg"]), f64(inp["Wu"]), f64(inp["B"]), f64(inp["b2"]), R)
@@ -262,6 +273,18 @@ class Model:
             self.A = shard("A", h, F, 0)
             self.B = shard("B", F, h, 1)
             self.b1, self.b2 = dev["b1"], dev["b2"]
+        if kind == "attn_gqa":
+            nq, nkv = cfg["n_heads"], cfg["n_kv_heads"]
+            d = h // nq
+            kvl = nkv // n if n <= nkv else 1
+            cols = (nq // n + 2 * kvl) * d
+            self.qkv_cols = n * cols
+            self.Wqkv = torch.empty(n * cols * h, dtype=torch.int16, device="cuda")
+            tp.tp_shard_qkv_gqa(dev["Wqkv"], h, nq, nkv, d, n, self.Wqkv)
+            self.bqkv = torch.empty(n * cols, dtype=torch.int16, device="cuda")
+            tp.tp_shard_qkv_gqa(dev["bqkv"], 1, nq, nkv, d, n, self.bqkv)
+            self.Wo = shard("Wo", h, h, 1)
+            self.bo = dev["bo"]
         if kind == "swiglu":
             F = cfg["ffn"]
             dev["GU"] = torch.cat([dev["Wg"].view(h, F), dev["Wu"].view(h, F)], dim=1).contiguous()
@@ -276,7 +299,7 @@ class Model:
                 b2=self.b2)
             self.dev_keep = dev
         wsk = {"mlp": tp.TP_WS_MLP, "swiglu": tp.TP_WS_MLP, "attn": tp.TP_WS_ATTN,
-               "layer": tp.TP_WS_LAYER}[kind]
+               "attn_gqa": tp.TP_WS_ATTN, "layer": tp.TP_WS_LAYER}[kind]
         self.ws_bytes = tp.tp_workspace_bytes(wsk, self.M, h, cfg.get("ffn", 0), n)
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
         self.Y = torch.empty((self.M, h), dtype=torch.int16, device="cuda")
@@ -294,6 +317,11 @@ class Model:
         elif cfg["kind"] == "layer":
             tp.tp_layer_forward(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"], cfg["ffn"], n,
                                 self.w, cfg.get("ln_eps", 1e-5), self.ws, self.ws_bytes, Y)
+        elif cfg["kind"] == "attn_gqa":
+            tp.tp_attn_forward_gqa(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"],
+                                   cfg["n_kv_heads"], cfg.get("causal", True), n, self.Wqkv,
+                                   self.bqkv, self.Wo, self.bo,
+                                   X if cfg.get("residual") else None, self.ws, self.ws_bytes, Y)
         elif cfg["kind"] == "swiglu":
             tp.tp_mlp_forward_swiglu(X, self.M, h, cfg["ffn"], n, self.GU, self.B, self.b2,
                                      X if cfg.get("residual") else None, self.ws, self.ws_bytes,

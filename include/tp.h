@@ -258,6 +258,42 @@ tp_status tp_layer_forward(const uint16_t* X, int64_t batch, int64_t seq,
                            float ln_eps, void* ws, size_t ws_bytes,
                            uint16_t* Y, void* stream);
 
+/* ---- Grouped-query attention ([TP-LLM] "Grouped-Query Attention (GQA)
+ * Constraints") ------------------------------------------------------------
+ * W_QKV = [W_Q | W_K | W_V] with n_q query heads and n_kv key/value heads of
+ * head_dim d (W_Q h x n_q d; W_K, W_V h x n_kv d); query head j uses kv head
+ * j / (n_q / n_kv). Requires n_q % N == 0, n_q % n_kv == 0 and either
+ * n_kv % N == 0 (shard i owns n_kv/N whole groups) or N % n_kv == 0 (N >
+ * n_kv: each shard holds a duplicate of its group's kv head). Shard i's
+ * columns: [Q_i (n_q/N heads) | K_i | V_i (kv_local heads each)], kv_local =
+ * n_kv/N or 1. Errors: TP_ERR_SHAPE for any other (n_q, n_kv, N). */
+
+/* Pack W_QKV [h_in][(n_q + 2 n_kv) d] into [N][(n_q/N + 2 kv_local) d][h_in]
+ * (a bias is packed as a 1-row matrix). Exact copy. */
+tp_status tp_shard_qkv_gqa(const uint16_t* W, int64_t h_in, int64_t n_q,
+                           int64_t n_kv, int64_t head_dim, int n_shards,
+                           uint16_t* W_shards, void* stream);
+
+/* Local attention of every shard's query heads with their group's kv head.
+ * QKV_shards [N][batch*seq][(n_q/N + 2 kv_local) d]; O_shards
+ * [N][batch*seq][n_q d / N]. head_dim must be 128. */
+tp_status tp_attention_gqa(const uint16_t* QKV_shards, int64_t batch,
+                           int64_t seq, int64_t n_q, int64_t n_kv,
+                           int64_t head_dim, int causal, int n_shards,
+                           uint16_t* O_shards, void* stream);
+
+/* GQA attention block by the tensor-parallel route (h = n_q x 128):
+ * Wqkv_shards from tp_shard_qkv_gqa, bqkv_shards likewise or NULL,
+ * Wo_shards TP_SPLIT_ROW of [h][h], bo [h] or NULL, residual [M][h] or NULL.
+ * ws >= tp_workspace_bytes(TP_WS_ATTN, batch*seq, h, 0, N). */
+tp_status tp_attn_forward_gqa(const uint16_t* X, int64_t batch, int64_t seq,
+                              int64_t h, int64_t n_q, int64_t n_kv, int causal,
+                              int n_shards, const uint16_t* Wqkv_shards,
+                              const uint16_t* bqkv_shards,
+                              const uint16_t* Wo_shards, const uint16_t* bo,
+                              const uint16_t* residual, void* ws,
+                              size_t ws_bytes, uint16_t* Y, void* stream);
+
 /* ---- Sequence parallelism ([TP-LLM] "Sequence Parallelism") ----------
  * Outside the tensor-parallel blocks, activations are split along the
  * sequence: shard i owns positions [i S/N, (i+1) S/N) of every sequence.

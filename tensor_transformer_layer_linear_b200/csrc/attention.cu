@@ -75,7 +75,10 @@ constexpr int B_Q = 0, B_KFULL = 1, B_VFULL = 3, B_KEMPTY = 5, B_VEMPTY = 7, B_S
               B_PFULL = 11, B_ODONE = 13;
 
 struct AttnParams {
-  int seq, batch, hps, hs, causal, nq;
+  int seq, batch, hps, causal, nq;
+  int q_w;    // query columns per shard (query heads per shard x 128)
+  int kv_w;   // key (= value) columns per shard
+  int group;  // local query heads per local kv head
   long long M;  // tokens per shard
   float scale_log2;
   unsigned* err;
@@ -141,6 +144,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         tma_load_3d(s0 + OFF_Q + T * FA_TILE, &tm, bar(B_Q), head * FA_D, qrow, g);
         tma_load_3d(s0 + OFF_Q + T * FA_TILE + FA_SUB, &tm, bar(B_Q), head * FA_D + 64, qrow, g);
       }
+      const int kvh = head / p.group;  // this query head's local kv head
+      const int kcol = p.q_w + kvh * FA_D, vcol = p.q_w + p.kv_w + kvh * FA_D;
       int kj = 0, vj = 0;  // K and V blocks issued
       for (int j = 0; j < nb; ++j) {
         const int b = j & 1;
@@ -152,8 +157,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
         const uint32_t kd = s0 + OFF_K + b * FA_TILE;
         mbar_arrive_expect_tx(bar(B_KFULL + b), FA_TILE);
-        tma_load_3d(kd, &tm, bar(B_KFULL + b), p.hs + head * FA_D, krow, g);
-        tma_load_3d(kd + FA_SUB, &tm, bar(B_KFULL + b), p.hs + head * FA_D + 64, krow, g);
+        tma_load_3d(kd, &tm, bar(B_KFULL + b), kcol, krow, g);
+        tma_load_3d(kd + FA_SUB, &tm, bar(B_KFULL + b), kcol + 64, krow, g);
         ++kj;
         if (!mbar_wait(bar(B_VEMPTY + b), ph ^ 1u, abort_flag)) {
           ok = false;
@@ -161,8 +166,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
         const uint32_t vd = s0 + OFF_V + b * FA_TILE;
         mbar_arrive_expect_tx(bar(B_VFULL + b), FA_TILE);
-        tma_load_3d(vd, &tm, bar(B_VFULL + b), 2 * p.hs + head * FA_D, krow, g);
-        tma_load_3d(vd + FA_SUB, &tm, bar(B_VFULL + b), 2 * p.hs + head * FA_D + 64, krow, g);
+        tma_load_3d(vd, &tm, bar(B_VFULL + b), vcol, krow, g);
+        tma_load_3d(vd + FA_SUB, &tm, bar(B_VFULL + b), vcol + 64, krow, g);
         ++vj;
       }
       if (!ok) {
@@ -334,7 +339,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     } else if (mbar_wait(bar(B_ODONE), 0, abort_flag)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint16_t* orow = O + (static_cast<int64_t>(g) * p.M + row_base + t) * p.hs + head * FA_D;
+      uint16_t* orow = O + (static_cast<int64_t>(g) * p.M + row_base + t) * p.q_w + head * FA_D;
 #pragma unroll 1
       for (int c = 0; c < FA_D / 32; ++c) {
         uint32_t o[32];
@@ -382,18 +387,18 @@ static PFN_cuTensorMapEncodeTiled_v12000 attn_map_encoder() {
   return fn;
 }
 
-int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t h, int64_t n_heads,
+int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, int64_t kv_local,
                      int n_shards, int causal, void* O, cudaStream_t s, unsigned* err) {
-  const int hps = static_cast<int>(n_heads / n_shards);
-  const int64_t hs = h / n_shards;
+  const int hps = static_cast<int>(n_q / n_shards);
+  const int64_t q_w = hps * FA_D, kv_w = kv_local * FA_D;
+  const int64_t ld = q_w + 2 * kv_w;  // QKV row width per shard
   const int64_t M = batch * seq;
   auto enc = attn_map_encoder();
   if (enc == nullptr) return 1;
   CUtensorMap tm;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(3 * hs), static_cast<cuuint64_t>(M),
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(M),
                         static_cast<cuuint64_t>(n_shards)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(3 * hs * 2),
-                           static_cast<cuuint64_t>(M * 3 * hs * 2)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld * 2), static_cast<cuuint64_t>(M * ld * 2)};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(QKV), dims, strides, box,
@@ -404,11 +409,13 @@ int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t h, int
   p.seq = static_cast<int>(seq);
   p.batch = static_cast<int>(batch);
   p.hps = hps;
-  p.hs = static_cast<int>(hs);
+  p.q_w = static_cast<int>(q_w);
+  p.kv_w = static_cast<int>(kv_w);
+  p.group = static_cast<int>(hps / kv_local);
   p.causal = causal;
   p.nq = static_cast<int>((seq + FA_BM * FA_TILES - 1) / (FA_BM * FA_TILES));
   p.M = M;
-  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(h / n_heads));
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(FA_D));
   p.err = err;
   cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM);
   const dim3 grid(p.nq, static_cast<unsigned>(n_shards * batch * hps));

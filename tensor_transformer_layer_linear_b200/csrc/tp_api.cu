@@ -400,7 +400,8 @@ tp_status tp_attention(const uint16_t* QKV_shards, int64_t batch, int64_t seq, i
   tp_status st = device_info(&d);
   if (st != TP_OK) return st;
   TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
-  return tpk::launch_attention(QKV_shards, batch, seq, h, n_heads, n_shards, causal ? 1 : 0,
+  return tpk::launch_attention(QKV_shards, batch, seq, n_heads, n_heads / n_shards, n_shards,
+                               causal ? 1 : 0,
                                O_shards, as_stream(stream), d.err) == 0
              ? TP_OK
              : TP_ERR_CUDA;
@@ -652,5 +653,88 @@ tp_status tp_layer_forward_sp(const uint16_t* X_shards, int64_t batch, int64_t s
   st = tp_row_linear(a, M, ffn, w->B_shards, h, n_shards, part, stream);
   if (st != TP_OK) return st;
   return tp_reduce_scatter_partials(part, n_shards, batch, seq, h, w->b2, h1, Y_shards, stream);
+}
+
+// ---------------------------------------------------------------- grouped-query attention
+// Valid GQA sharding: n_q % N == 0, n_q % n_kv == 0, and either n_kv % N == 0
+// (each shard owns n_kv/N whole groups) or N % n_kv == 0 (N > n_kv: one
+// duplicated kv head per shard).
+static bool gqa_ok(int64_t n_q, int64_t n_kv, int n_shards) {
+  if (n_q <= 0 || n_kv <= 0 || n_shards <= 0) return false;
+  if (n_q % n_shards || n_q % n_kv) return false;
+  return (n_shards <= n_kv) ? (n_kv % n_shards == 0) : (n_shards % n_kv == 0);
+}
+static int64_t gqa_kv_local(int64_t n_kv, int n_shards) {
+  return n_shards <= n_kv ? n_kv / n_shards : 1;
+}
+
+tp_status tp_shard_qkv_gqa(const uint16_t* W, int64_t h_in, int64_t n_q, int64_t n_kv,
+                           int64_t head_dim, int n_shards, uint16_t* W_shards, void* stream) {
+  if (W == nullptr || W_shards == nullptr) return TP_ERR_NULL;
+  if (h_in <= 0 || head_dim <= 0 || n_shards > 65535 || !gqa_ok(n_q, n_kv, n_shards))
+    return TP_ERR_SHAPE;
+  const int64_t cols = (n_q / n_shards + 2 * gqa_kv_local(n_kv, n_shards)) * head_dim;
+  if ((h_in + 31) / 32 > kIntMax || (cols + 31) / 32 > 65535) return TP_ERR_SHAPE;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_SHARD, as_stream(stream));
+  return tpk::launch_shard(W, h_in, (n_q + 2 * n_kv) * head_dim, n_shards, 4, head_dim, W_shards,
+                           as_stream(stream), n_q, n_kv) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_attention_gqa(const uint16_t* QKV_shards, int64_t batch, int64_t seq, int64_t n_q,
+                           int64_t n_kv, int64_t head_dim, int causal, int n_shards,
+                           uint16_t* O_shards, void* stream) {
+  if (QKV_shards == nullptr || O_shards == nullptr) return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || !gqa_ok(n_q, n_kv, n_shards)) return TP_ERR_SHAPE;
+  if (head_dim != 128) return TP_ERR_UNSUPPORTED;
+  if (batch * seq > kIntMax || seq > kIntMax) return TP_ERR_SHAPE;
+  if (static_cast<int64_t>(n_shards) * batch * (n_q / n_shards) > 65535) return TP_ERR_SHAPE;
+  if (!al16(QKV_shards) || !al16(O_shards)) return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
+  return tpk::launch_attention(QKV_shards, batch, seq, n_q, gqa_kv_local(n_kv, n_shards),
+                               n_shards, causal ? 1 : 0, O_shards, as_stream(stream), d.err) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_attn_forward_gqa(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
+                              int64_t n_q, int64_t n_kv, int causal, int n_shards,
+                              const uint16_t* Wqkv_shards, const uint16_t* bqkv_shards,
+                              const uint16_t* Wo_shards, const uint16_t* bo,
+                              const uint16_t* residual, void* ws, size_t ws_bytes, uint16_t* Y,
+                              void* stream) {
+  if (X == nullptr || Wqkv_shards == nullptr || Wo_shards == nullptr || Y == nullptr ||
+      ws == nullptr)
+    return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || !gqa_ok(n_q, n_kv, n_shards)) return TP_ERR_SHAPE;
+  if (h % n_q || h / n_q != 128) return TP_ERR_UNSUPPORTED;
+  const int64_t M = batch * seq;
+  const int64_t qkv_cols = n_shards * (n_q / n_shards + 2 * gqa_kv_local(n_kv, n_shards)) * 128;
+  // the attention workspace holds 3h QKV columns, which covers GQA (duplicated
+  // kv heads included: N <= n_q)
+  const size_t need = tp_workspace_bytes(TP_WS_ATTN, M, h, 0, n_shards);
+  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  if (!al16(ws)) return TP_ERR_ALIGN;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* qkv = reinterpret_cast<uint16_t*>(w);
+  w += round256(static_cast<size_t>(M) * 3 * h * 2);
+  uint16_t* o = reinterpret_cast<uint16_t*>(w);
+  w += round256(static_cast<size_t>(M) * h * 2);
+  float* part = reinterpret_cast<float*>(w);
+  tp_status st = tp_column_linear(X, M, h, Wqkv_shards, bqkv_shards, qkv_cols, n_shards,
+                                  TP_ACT_NONE, qkv, stream);
+  if (st != TP_OK) return st;
+  st = tp_attention_gqa(qkv, batch, seq, n_q, n_kv, 128, causal, n_shards, o, stream);
+  if (st != TP_OK) return st;
+  st = tp_row_linear(o, M, h, Wo_shards, h, n_shards, part, stream);
+  if (st != TP_OK) return st;
+  return tp_reduce_partials(part, n_shards, M, h, bo, residual, Y, stream);
 }
 }  // extern "C"

@@ -62,12 +62,15 @@ int launch_rows_sum_ln(const float* P, int n_shards, int64_t rows, int64_t h, co
                        void* Y_sum, void* Y_ln, cudaStream_t s, int sp_n = 0, int sp_batch = 0,
                        int sp_seq = 0, int ln_natural = 1);
 
-// Causal / full attention of every shard's heads, head_dim 128.
-int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t h, int64_t n_heads,
+// Causal / full attention of every shard's heads, head_dim 128. Shard rows
+// of QKV are [Q (n_q/N heads) | K (kv_local heads) | V (kv_local heads)];
+// local query head k uses local kv head k / (n_q/N / kv_local).
+int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, int64_t kv_local,
                      int n_shards, int causal, void* O, cudaStream_t s, unsigned* err);
 
-// out[i][c][r] = W[row(i, r)][col(i, c)] for the three split kinds.
+// out[i][c][r] = W[row(i, r)][col(i, c)] for the split kinds (kind 4: GQA
+// QKV with n_q query and n_kv key/value heads of head_dim).
 int launch_shard(const void* W, int64_t h_in, int64_t h_out, int n_shards, int kind,
-                 int64_t head_dim, void* out, cudaStream_t s);
+                 int64_t head_dim, void* out, cudaStream_t s, int64_t n_q = 0, int64_t n_kv = 0);
 
 }  // namespace tpk

@@ -19,7 +19,9 @@ attention and layer examples: the page-1 worked example
 (Linear(1024 -> 4096) on 32 tokens, tensor_model_parallel_size = 2), a
 4 x 2048-token MLP, a 16-head causal attention block, a full pre-LN layer,
 and a large MLP swept over shard counts. A gated (SwiGLU) MLP of the
-4 x 2048-token MLP's shape is added for the gated variant.
+4 x 2048-token MLP's shape is added for the gated variant, and a
+grouped-query attention block of the attention block's shape (16 query
+heads, 4 key/value heads, 8 shards: key/value heads duplicated).
 """
 from __future__ import annotations
 
@@ -40,6 +42,9 @@ CONFIGS = {
         kind="layer", batch=2, seq=2048, h=4096, n_heads=32, ffn=16384,
         n_shards=8, causal=True, x_std=1.0, w_std=0.02, b_std=0.01,
         ln_eps=1e-5),
+    "attn_gqa_4x2048_h2048_16q4kv_n8": dict(
+        kind="attn_gqa", batch=4, seq=2048, h=2048, n_heads=16, n_kv_heads=4,
+        n_shards=8, causal=True, x_std=1.0, w_std=0.02, b_std=0.01, residual=True),
     "swiglu_8192x1024_f4096_n4": dict(
         kind="swiglu", batch=4, seq=2048, h=1024, ffn=4096, n_shards=4,
         x_std=1.0, w_std=0.02, b_std=0.01, residual=True),
@@ -90,7 +95,8 @@ def make_inputs(cfg: dict, seed: int = 0) -> dict:
       X [M, h]; MLP: A [h, F], b1 [F], B [F, h], b2 [h];
       attention: Wqkv [h, 3h] (= [W_Q | W_K | W_V]), bqkv [3h], Wo [h, h], bo [h];
       layer: both sets plus ln1_g, ln1_b, ln2_g, ln2_b [h];
-      swiglu (gated MLP): Wg, Wu [h, F], B [F, h], b2 [h].
+      swiglu (gated MLP): Wg, Wu [h, F], B [F, h], b2 [h];
+      attn_gqa: Wqkv [h, (n_q + 2 n_kv) d], Wo [h, h], bqkv, bo.
     """
     rng = np.random.Generator(np.random.Philox(seed))
     kind = cfg["kind"]
@@ -101,6 +107,13 @@ def make_inputs(cfg: dict, seed: int = 0) -> dict:
     if kind in ("attn", "layer"):
         out["Wqkv"] = _draw(rng, (h, 3 * h), w)
         out["Wo"] = _draw(rng, (h, h), w)
+    if kind == "attn_gqa":
+        d = h // cfg["n_heads"]
+        qkv_cols = (cfg["n_heads"] + 2 * cfg["n_kv_heads"]) * d
+        out["Wqkv"] = _draw(rng, (h, qkv_cols), w)
+        out["Wo"] = _draw(rng, (h, h), w)
+        out["bqkv"] = _draw(rng, (qkv_cols,), b)
+        out["bo"] = _draw(rng, (h,), b)
     if kind in ("mlp", "layer"):
         F = cfg["ffn"]
         out["A"] = _draw(rng, (h, F), w)

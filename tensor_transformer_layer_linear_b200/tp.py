@@ -66,6 +66,10 @@ _SIGS = {
     "tp_all_gather_sequence": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _vp]),
     "tp_layer_forward_sp": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32,
                                    ctypes.POINTER(tp_layer_weights), _f32, _vp, _sz, _vp, _vp]),
+    "tp_shard_qkv_gqa": (_i32, [_vp, _i64, _i64, _i64, _i64, _i32, _vp, _vp]),
+    "tp_attention_gqa": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp]),
+    "tp_attn_forward_gqa": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp,
+                                   _vp, _vp, _vp, _sz, _vp, _vp]),
     "tp_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "tp_get_last_error": (_i32, [_vp]),
     "tp_status_string": (ctypes.c_char_p, [_i32]),
@@ -244,6 +248,26 @@ def tp_layer_forward_sp(X_shards, batch, seq, h, n_heads, ffn, n_shards,
     _check(lib.tp_layer_forward_sp(_p(X_shards), batch, seq, h, n_heads, ffn, n_shards,
                                    ctypes.byref(weights), ln_eps, _p(ws), ws_bytes, _p(Y_shards),
                                    _s(stream)), "tp_layer_forward_sp")
+
+
+def tp_shard_qkv_gqa(W, h_in, n_q, n_kv, head_dim, n_shards, W_shards, stream=None):
+    _check(lib.tp_shard_qkv_gqa(_p(W), h_in, n_q, n_kv, head_dim, n_shards, _p(W_shards),
+                                _s(stream)), "tp_shard_qkv_gqa")
+
+
+def tp_attention_gqa(QKV_shards, batch, seq, n_q, n_kv, head_dim, causal, n_shards, O_shards,
+                     stream=None):
+    _check(lib.tp_attention_gqa(_p(QKV_shards), batch, seq, n_q, n_kv, head_dim,
+                                int(bool(causal)), n_shards, _p(O_shards), _s(stream)),
+           "tp_attention_gqa")
+
+
+def tp_attn_forward_gqa(X, batch, seq, h, n_q, n_kv, causal, n_shards, Wqkv_shards, bqkv_shards,
+                        Wo_shards, bo, residual, ws, ws_bytes, Y, stream=None):
+    _check(lib.tp_attn_forward_gqa(_p(X), batch, seq, h, n_q, n_kv, int(bool(causal)), n_shards,
+                                   _p(Wqkv_shards), _p(bqkv_shards), _p(Wo_shards), _p(bo),
+                                   _p(residual), _p(ws), ws_bytes, _p(Y), _s(stream)),
+           "tp_attn_forward_gqa")
 
 
 def tp_get_last_error(stream=None) -> int:

@@ -1,0 +1,119 @@
+"""Grouped-query attention under tensor parallelism on a B200, against the
+fp64 oracle ("Tensor Parallelism in Large Language Models", "Grouped-Query
+Attention (GQA) Constraints"): the packing of query heads with their (possibly
+duplicated) key/value heads, the attention kernel on shared K/V, and the
+block, for N both dividing n_kv and exceeding it.
+"""
+import numpy as np
+import pytest
+
+from oracle import tp_oracle as O
+from tensor_transformer_layer_linear_b200 import synth
+
+from helpers import assert_parity, f64, from_dev_bf16, to_dev
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def tp():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from tensor_transformer_layer_linear_b200 import tp as _tp
+    return _tp
+
+
+def _bits(rng, shape, std=1.0):
+    return synth.f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32) * np.float32(std))
+
+
+def _kvl(n_kv, n):
+    return n_kv // n if n <= n_kv else 1
+
+
+def _pack(tp, W, h_in, n_q, n_kv, d, n):
+    cols = (n_q // n + 2 * _kvl(n_kv, n)) * d
+    out = torch.empty(n * cols * h_in, dtype=torch.int16, device="cuda")
+    tp.tp_shard_qkv_gqa(to_dev(W), h_in, n_q, n_kv, d, n, out)
+    return out, cols
+
+
+@pytest.mark.parametrize("n_q,n_kv,n", [(8, 2, 1), (8, 2, 2), (8, 2, 4), (8, 2, 8), (16, 4, 8),
+                                        (8, 1, 4)])
+def test_gqa_packing_bit_exact(tp, n_q, n_kv, n):
+    rng = np.random.default_rng(1200 + n_q + n_kv + n)
+    d, h_in = 16, 72
+    W = _bits(rng, (h_in, (n_q + 2 * n_kv) * d))
+    out, cols = _pack(tp, W, h_in, n_q, n_kv, d, n)
+    got = out.cpu().numpy().view(np.uint16).reshape(n, cols, h_in)
+    assert np.array_equal(got, O.packed_gqa_shards(W, n_q, n_kv, d, n))
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("n_q,n_kv,n", [(4, 2, 1), (4, 2, 2), (4, 2, 4), (4, 1, 2)])
+def test_gqa_attention_kernel(tp, n_q, n_kv, n, causal):
+    rng = np.random.default_rng(1300 + n_q + n_kv + n)
+    batch, seq, d = 2, 300, 128
+    qs, kvl = n_q // n, _kvl(n_kv, n)
+    QKV = _bits(rng, (n, batch * seq, (qs + 2 * kvl) * d))
+    O_ = torch.empty((n, batch * seq, qs * d), dtype=torch.int16, device="cuda")
+    tp.tp_attention_gqa(to_dev(QKV), batch, seq, n_q, n_kv, d, causal, n, O_)
+    got = from_dev_bf16(O_)
+    q = f64(QKV)
+    for i in range(n):
+        ref = O.gqa_attention_heads(q[i][:, :qs * d], q[i][:, qs * d:(qs + kvl) * d],
+                                    q[i][:, (qs + kvl) * d:], batch, seq, qs, kvl, causal)
+        assert_parity(got[i], ref, f"shard {i}")
+
+
+def _run_block(tp, inp, cfg, n):
+    b, s, h, nq, nkv = cfg["batch"], cfg["seq"], cfg["h"], cfg["n_heads"], cfg["n_kv_heads"]
+    d = h // nq
+    M = b * s
+    dev = {k: to_dev(v) for k, v in inp.items()}
+    Wqkv, cols = _pack(tp, inp["Wqkv"], h, nq, nkv, d, n)
+    bqkv, _ = _pack(tp, inp["bqkv"].reshape(1, -1), 1, nq, nkv, d, n)
+    Wo = torch.empty(h * h, dtype=torch.int16, device="cuda")
+    tp.tp_shard_weights(dev["Wo"], h, h, n, tp.TP_SPLIT_ROW, 0, Wo)
+    nb = tp.tp_workspace_bytes(tp.TP_WS_ATTN, M, h, 0, n)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    Y = torch.empty((M, h), dtype=torch.int16, device="cuda")
+    tp.tp_attn_forward_gqa(dev["X"], b, s, h, nq, nkv, True, n, Wqkv, bqkv, Wo, dev["bo"],
+                           dev["X"], ws, nb, Y)
+    assert tp.tp_get_last_error() == tp.TP_OK
+    return from_dev_bf16(Y)
+
+
+@pytest.mark.parametrize("n", [2, 4, 8])
+def test_gqa_block_small_all_elements(tp, n):
+    cfg = dict(kind="attn_gqa", batch=2, seq=192, h=1024, n_heads=8, n_kv_heads=2, causal=True,
+               x_std=1.0, w_std=0.05, b_std=0.05, residual=True)
+    inp = synth.make_inputs(cfg, seed=6)
+    x = f64(inp["X"])
+    ref = O.gqa_self_attention(x, f64(inp["Wqkv"]), f64(inp["bqkv"]), f64(inp["Wo"]),
+                               f64(inp["bo"]), x, 2, 192, 8, 2)
+    assert_parity(_run_block(tp, inp, cfg, n), ref)
+
+
+def test_gqa_workload_sampled_rows(tp):
+    cfg = synth.config("attn_gqa_4x2048_h2048_16q4kv_n8")
+    inp = synth.make_inputs(cfg)
+    Y = _run_block(tp, inp, cfg, cfg["n_shards"])
+    rows = synth.sample_rows(cfg["batch"], cfg["seq"])
+    x = f64(inp["X"])
+    # the oracle restricted to the sampled rows: full K, V of every sequence
+    ref_full = O.gqa_self_attention(x, f64(inp["Wqkv"]), f64(inp["bqkv"]), f64(inp["Wo"]),
+                                    f64(inp["bo"]), x, cfg["batch"], cfg["seq"],
+                                    cfg["n_heads"], cfg["n_kv_heads"])
+    assert_parity(Y[rows], ref_full[rows])
+
+
+def test_gqa_rejects_bad_group_split(tp):
+    X = torch.zeros(1024, dtype=torch.int16, device="cuda")
+    with pytest.raises(tp.TPError) as e:
+        tp.tp_attention_gqa(X, 1, 64, 8, 4, 128, True, 3, X)   # 8 % 3
+    assert e.value.status == tp.TP_ERR_SHAPE
+    with pytest.raises(tp.TPError) as e:
+        tp.tp_shard_qkv_gqa(X, 8, 8, 4, 16, 6, X)              # N = 6 vs n_kv = 4
+    assert e.value.status == tp.TP_ERR_SHAPE
