@@ -417,6 +417,15 @@ int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, i
   p.M = M;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(FA_D));
   p.err = err;
+  // The setmaxnreg split assumes FA_REGS_LAUNCH registers per thread at
+  // launch; with fewer, the softmax warpgroups' increase could never be
+  // granted, so refuse to launch.
+  static int launch_regs = -1;
+  if (launch_regs < 0) {
+    cudaFuncAttributes fa;
+    launch_regs = cudaFuncGetAttributes(&fa, attention_tc_kernel) == cudaSuccess ? fa.numRegs : 0;
+  }
+  if (launch_regs * FA_THREADS < 256 * FA_REGS_SOFTMAX + 128 * FA_REGS_OTHER) return 3;
   cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM);
   const dim3 grid(p.nq, static_cast<unsigned>(n_shards * batch * hps));
   attention_tc_kernel<<<grid, FA_THREADS, FA_SMEM, s>>>(tm, static_cast<uint16_t*>(O), p);

@@ -400,11 +400,10 @@ tp_status tp_attention(const uint16_t* QKV_shards, int64_t batch, int64_t seq, i
   tp_status st = device_info(&d);
   if (st != TP_OK) return st;
   TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
-  return tpk::launch_attention(QKV_shards, batch, seq, n_heads, n_heads / n_shards, n_shards,
-                               causal ? 1 : 0,
-                               O_shards, as_stream(stream), d.err) == 0
-             ? TP_OK
-             : TP_ERR_CUDA;
+  const int rc = tpk::launch_attention(QKV_shards, batch, seq, n_heads, n_heads / n_shards,
+                                       n_shards, causal ? 1 : 0, O_shards, as_stream(stream),
+                                       d.err);
+  return rc == 0 ? TP_OK : (rc == 3 ? TP_ERR_UNSUPPORTED : TP_ERR_CUDA);
 }
 
 size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int n_shards) {
@@ -698,10 +697,10 @@ tp_status tp_attention_gqa(const uint16_t* QKV_shards, int64_t batch, int64_t se
   tp_status st = device_info(&d);
   if (st != TP_OK) return st;
   TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
-  return tpk::launch_attention(QKV_shards, batch, seq, n_q, gqa_kv_local(n_kv, n_shards),
-                               n_shards, causal ? 1 : 0, O_shards, as_stream(stream), d.err) == 0
-             ? TP_OK
-             : TP_ERR_CUDA;
+  const int rc = tpk::launch_attention(QKV_shards, batch, seq, n_q, gqa_kv_local(n_kv, n_shards),
+                                       n_shards, causal ? 1 : 0, O_shards, as_stream(stream),
+                                       d.err);
+  return rc == 0 ? TP_OK : (rc == 3 ? TP_ERR_UNSUPPORTED : TP_ERR_CUDA);
 }
 
 tp_status tp_attn_forward_gqa(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,

@@ -64,7 +64,9 @@ int launch_rows_sum_ln(const float* P, int n_shards, int64_t rows, int64_t h, co
 
 // Causal / full attention of every shard's heads, head_dim 128. Shard rows
 // of QKV are [Q (n_q/N heads) | K (kv_local heads) | V (kv_local heads)];
-// local query head k uses local kv head k / (n_q/N / kv_local).
+// local query head k uses local kv head k / (n_q/N / kv_local). Returns 3 if
+// the kernel was built with fewer launch registers than its warpgroup
+// register split needs (it is then not launched).
 int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, int64_t kv_local,
                      int n_shards, int causal, void* O, cudaStream_t s, unsigned* err);
 
