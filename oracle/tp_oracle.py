@@ -391,6 +391,52 @@ def packed_gate_up(W_gate: np.ndarray, W_up: np.ndarray, n_shards: int) -> np.nd
 
 
 # --------------------------------------------------------------------------
+# MLP backward ([TP-LLM] MLP block: "exactly one All-Reduce in the backward
+# pass (to synchronize input gradients across the column-parallel layer)")
+# --------------------------------------------------------------------------
+
+def gelu_grad(z: np.ndarray) -> np.ndarray:
+    """d GeLU / dz = Phi(z) + z phi(z), phi the standard normal density."""
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * (1.0 + _erf(z / math.sqrt(2.0))) + z * np.exp(-0.5 * z * z) / math.sqrt(2.0 * math.pi)
+
+
+def mlp_backward(X, A, b1, B, dY, residual: bool = True) -> dict:
+    """Gradients of Y = GeLU(X A + b1) B + b2 (+ X) given dY = dL/dY:
+    dX, dA, db1, dB, db2 (unsharded)."""
+    Z = linear(X, A, b1)
+    H = gelu(Z)
+    dH = dY @ B.T
+    dZ = dH * gelu_grad(Z)
+    dX = dZ @ A.T
+    if residual:
+        dX = dX + dY
+    return dict(dX=dX, dA=X.T @ dZ, db1=dZ.sum(axis=0), dB=H.T @ dY, db2=dY.sum(axis=0))
+
+
+def mlp_backward_sharded(X, A, b1, B, dY, n_shards: int, residual: bool = True) -> dict:
+    """The tensor-parallel backward: dY reaches every shard whole (the
+    row-parallel layer's backward needs no exchange); each shard forms
+    dH_i = dY B_i^T, dZ_i = dH_i GeLU'(Z_i), its weight gradients dB_i, dA_i,
+    db1_i locally, and a full-size partial dX_i = dZ_i A_i^T; the one
+    reduction is dX = sum_i dX_i (+ dY for the residual)."""
+    A_i = shard_matrices(A, SPLIT_COLUMN, n_shards)
+    b_i = shard_matrices(np.asarray(b1).reshape(1, -1), SPLIT_COLUMN, n_shards)
+    B_i = shard_matrices(B, SPLIT_ROW, n_shards)
+    parts, dA, db1, dB = [], [], [], []
+    for Ai, bi, Bi in zip(A_i, b_i, B_i):
+        Z = linear(X, Ai, bi[0])
+        dZ = (dY @ Bi.T) * gelu_grad(Z)
+        parts.append(dZ @ Ai.T)
+        dA.append(X.T @ dZ)
+        db1.append(dZ.sum(axis=0))
+        dB.append(gelu(Z).T @ dY)
+    dX = reduce_partials(parts, None, dY if residual else None)
+    return dict(dX=dX, dA=np.concatenate(dA, axis=1), db1=np.concatenate(db1),
+                dB=np.concatenate(dB, axis=0), db2=dY.sum(axis=0), dX_partials=parts)
+
+
+# --------------------------------------------------------------------------
 # grouped-query attention ([TP-LLM] "Grouped-Query Attention (GQA)
 # Constraints")
 # --------------------------------------------------------------------------

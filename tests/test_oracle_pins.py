@@ -590,3 +590,59 @@ def test_gqa_shard_columns_and_constraints():
         O.gqa_shard_columns(8, 4, 1, 3)          # 8 % 3
     with pytest.raises(ValueError):
         O.gqa_kv_local(4, 6)                     # N = 6 neither divides nor is divided by 4
+
+
+
+# ---------------------------------------------------------------- MLP backward
+
+def test_gelu_grad_values_and_finite_difference():
+    assert O.gelu_grad(np.array([0.0]))[0] == pytest.approx(0.5, abs=1e-15)
+    # Phi(1) + phi(1) = 0.8413447460685429 + 0.24197072451914337 (normal table values)
+    assert O.gelu_grad(np.array([1.0]))[0] == pytest.approx(0.8413447460685429 + 0.24197072451914337,
+                                                            abs=1e-14)
+    assert O.gelu_grad(np.array([12.0]))[0] == pytest.approx(1.0, abs=1e-12)
+    assert abs(O.gelu_grad(np.array([-12.0]))[0]) < 1e-20
+    z = np.linspace(-4, 4, 41)
+    eps = 1e-6
+    fd = (O.gelu(z + eps) - O.gelu(z - eps)) / (2 * eps)
+    np.testing.assert_allclose(O.gelu_grad(z), fd, atol=1e-8)
+
+
+def _mlp_loss(X, A, b1, B, b2, dY):
+    return float(np.sum(O.mlp(X, A, b1, B, b2, X) * dY))
+
+
+def test_mlp_backward_matches_finite_differences():
+    """Every gradient against central differences of <Y, dY> (an independent
+    check of the chain rule, the transposes and the residual term)."""
+    rng = np.random.default_rng(20)
+    M, h, F = 3, 4, 6
+    X, A, B = rng.standard_normal((M, h)), rng.standard_normal((h, F)) * .5, rng.standard_normal((F, h)) * .5
+    b1, b2 = rng.standard_normal(F) * .1, rng.standard_normal(h) * .1
+    dY = rng.standard_normal((M, h))
+    g = O.mlp_backward(X, A, b1, B, dY)
+    eps = 1e-6
+    for name, arr in (("dX", X), ("dA", A), ("db1", b1), ("dB", B), ("db2", b2)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            up = _mlp_loss(X, A, b1, B, b2, dY)
+            arr[idx] = orig - eps
+            dn = _mlp_loss(X, A, b1, B, b2, dY)
+            arr[idx] = orig
+            num[idx] = (up - dn) / (2 * eps)
+        np.testing.assert_allclose(g[name], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 6])
+def test_mlp_backward_sharded_equals_unsharded(n):
+    rng = np.random.default_rng(21)
+    M, h, F = 5, 4, 12
+    X, A, B = rng.standard_normal((M, h)), rng.standard_normal((h, F)), rng.standard_normal((F, h))
+    b1, dY = rng.standard_normal(F), rng.standard_normal((M, h))
+    ref = O.mlp_backward(X, A, b1, B, dY)
+    got = O.mlp_backward_sharded(X, A, b1, B, dY, n)
+    for k in ("dX", "dA", "db1", "dB", "db2"):
+        np.testing.assert_allclose(got[k], ref[k], rtol=1e-12, atol=1e-12, err_msg=k)
+    assert len(got["dX_partials"]) == n and all(p.shape == (M, h) for p in got["dX_partials"])
