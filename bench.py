@@ -94,6 +94,12 @@ def work(cfg: dict) -> dict:
         fl["attention"] += 4.0 * cfg["seq"] ** 2 * d * cfg["n_heads"] * cfg["batch"] / (
             2 if cfg.get("causal", True) else 1)
         fl["gemm_row_parallel"] += 2.0 * M * h * h
+    if kind == "mlp" and cfg.get("backward"):
+        # algorithmic backward: dH, dX, dA, dB (the recomputed forward GEMM is extra)
+        F = cfg["ffn"]
+        fl = {"gemm_backward": 8.0 * M * h * F, "gemm_column_parallel": 0.0,
+              "gemm_row_parallel": 0.0, "attention": 0.0}
+        by["reduce_partials"] = n * M * h * 4 + 2 * M * h * 2
     if kind == "swiglu":
         F = cfg["ffn"]
         fl["gemm_column_parallel"] += 2.0 * M * h * 2 * F   # gate and up
@@ -303,10 +309,32 @@ class Model:
         self.ws_bytes = tp.tp_workspace_bytes(wsk, self.M, h, cfg.get("ffn", 0), n)
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
         self.Y = torch.empty((self.M, h), dtype=torch.int16, device="cuda")
+        if cfg.get("backward"):
+            self.setup_backward()
         torch.cuda.synchronize()
+
+    def setup_backward(self):
+        """Gradient buffers for the MLP backward step (dY drawn once)."""
+        torch, cfg = self.torch, self.cfg
+        M, h, F, n = self.M, cfg["h"], cfg["ffn"], cfg["n_shards"]
+        g = torch.Generator(device="cuda").manual_seed(1)
+        self.dY = (torch.randn((M, h), device="cuda", generator=g)).to(torch.bfloat16).view(torch.int16)
+        self.dX = torch.empty((M, h), dtype=torch.int16, device="cuda")
+        self.dA = torch.empty(h * F, dtype=torch.float32, device="cuda")
+        self.dB = torch.empty(h * F, dtype=torch.float32, device="cuda")
+        self.db1 = torch.empty(F, dtype=torch.float32, device="cuda")
+        self.db2 = torch.empty(h, dtype=torch.float32, device="cuda")
+        self.ws_bwd_bytes = self.tp.tp_workspace_bytes(self.tp.TP_WS_MLP_BWD, M, h, F, n)
+        self.ws_bwd = torch.empty(self.ws_bwd_bytes, dtype=torch.uint8, device="cuda")
 
     def step(self, X=None, Y=None):
         tp, cfg = self.tp, self.cfg
+        if cfg.get("backward"):
+            X = self.X if X is None else X
+            tp.tp_mlp_backward(X, self.M, cfg["h"], cfg["ffn"], cfg["n_shards"], self.A, self.b1,
+                               self.B, self.dY, cfg.get("residual", False), self.ws_bwd,
+                               self.ws_bwd_bytes, self.dX, self.dA, self.db1, self.dB, self.db2)
+            return
         X = self.X if X is None else X
         Y = self.Y if Y is None else Y
         n, h = cfg["n_shards"], cfg["h"]
@@ -431,18 +459,19 @@ def run_ours(args, cfg) -> None:
 
     def kernel_fig(name):
         n_l, t_ms = per[name]
-        if name in w["flops"] and w["flops"][name] > 0:
+        base = dict(launches=n_l, avg_launch_ms=t_ms / n_l, share=t_ms / total_k,
+                    traffic=NCU_TRAFFIC.get((cfg["name"], name)))
+        if w["flops"].get(name, 0) > 0:
             units = w["flops"][name] * steps_traced
             achieved = units / (t_ms * 1e-3) / 1e12
             return dict(bound="tensor", achieved=achieved, peak=pk["bf16"], unit="TFLOP/s",
-                        frac=achieved / pk["bf16"], launches=n_l,
-                        avg_launch_ms=t_ms / n_l, share=t_ms / total_k,
-                        traffic=NCU_TRAFFIC.get((cfg["name"], name)))
-        units = w["bytes"][name] * steps_traced
-        achieved = units / (t_ms * 1e-3) / 1e9
-        return dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
-                    frac=achieved / pk["hbm"], launches=n_l, avg_launch_ms=t_ms / n_l,
-                    share=t_ms / total_k, traffic=NCU_TRAFFIC.get((cfg["name"], name)))
+                        frac=achieved / pk["bf16"], **base)
+        if name in w["bytes"]:
+            units = w["bytes"][name] * steps_traced
+            achieved = units / (t_ms * 1e-3) / 1e9
+            return dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
+                        frac=achieved / pk["hbm"], **base)
+        return dict(bound="other", achieved=None, peak=None, unit=None, frac=None, **base)
 
     roof = kernel_fig(dom)
     roof["kernel"] = dom
@@ -474,7 +503,7 @@ def run_ours(args, cfg) -> None:
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": cfg["name"] + ("+sequence_parallel" if cfg.get("sequence_parallel")
-                                              else ""),
+                                              else "") + ("+backward" if cfg.get("backward") else ""),
                    "tokens": M, "h": h, "n_shards": cfg["n_shards"],
                    "heads": cfg.get("n_heads"), "ffn": cfg.get("ffn"),
                    "l2": "inputs larger than L2 (per-step working set "
@@ -560,6 +589,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sequence-parallel", action="store_true",
                     help="layer workload: run tp_layer_forward_sp on sequence-sharded input")
+    ap.add_argument("--backward", action="store_true",
+                    help="MLP workloads: time tp_mlp_backward (dX, weight and bias gradients)")
     ap.add_argument("--sweep", action="store_true",
                     help="run the workload at every shard count of its sweep (one JSON line)")
     args = ap.parse_args()
@@ -568,6 +599,10 @@ def main():
     cfg = synth.config(args.workload)
     if args.shards:
         cfg["n_shards"] = args.shards
+    if args.backward:
+        if cfg["kind"] != "mlp":
+            ap.error("--backward applies to the MLP workloads")
+        cfg["backward"] = True
     if args.sequence_parallel:
         if cfg["kind"] != "layer":
             ap.error("--sequence-parallel applies to the layer workload")

@@ -95,7 +95,9 @@ typedef enum {
     TP_ACT_SWIGLU = 2
 } tp_act;
 
-typedef enum { TP_WS_MLP = 0, TP_WS_ATTN = 1, TP_WS_LAYER = 2, TP_WS_LAYER_SP = 3 } tp_ws_kind;
+typedef enum {
+    TP_WS_MLP = 0, TP_WS_ATTN = 1, TP_WS_LAYER = 2, TP_WS_LAYER_SP = 3, TP_WS_MLP_BWD = 4
+} tp_ws_kind;
 
 /* Weights of one pre-LN layer, all device pointers in the packed shard
    layouts below. h = hidden, F = FFN width, N = shards. */
@@ -231,6 +233,28 @@ tp_status tp_mlp_forward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn,
                          const uint16_t* b2, const uint16_t* residual,
                          void* ws, size_t ws_bytes, uint16_t* Y, void* stream);
 
+/* tp_mlp_backward - gradients of Y = GeLU(X A + b1) B + b2 (+ X) by the
+ * tensor-parallel route ([TP-LLM] MLP block: exactly one all-reduce in the
+ * backward pass, of the input gradient across the column-parallel layer).
+ * dY reaches every shard whole (the row-parallel layer's backward needs no
+ * exchange); each shard recomputes Z_i = X A_i + b1_i, forms
+ * dZ_i = (dY B_i^T) * GeLU'(Z_i), its weight gradients locally, and a
+ * full-size partial dX_i = dZ_i A_i^T; dX = sum_i dX_i (+ dY when residual)
+ * is the one reduction.
+ * Inputs: X [B][h], the forward's packed A_shards [N][F/N][h], b1_shards
+ * [N][F/N] or NULL, B_shards [N][h][F/N], dY [B][h] (all bf16).
+ * Outputs: dX [B][h] bf16; dA_shards [N][F/N][h] and dB_shards [N][h][F/N]
+ * fp32 in the packed layouts of A_shards and B_shards (dA_shards[i] =
+ * dA_i^T, dB_shards[i] = dB_i^T); db1 [F] and db2 [h] fp32.
+ * ws >= tp_workspace_bytes(TP_WS_MLP_BWD, B, h, F, N). */
+tp_status tp_mlp_backward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn,
+                          int n_shards, const uint16_t* A_shards,
+                          const uint16_t* b1_shards, const uint16_t* B_shards,
+                          const uint16_t* dY, int residual, void* ws,
+                          size_t ws_bytes, uint16_t* dX, float* dA_shards,
+                          float* db1, float* dB_shards, float* db2,
+                          void* stream);
+
 /* tp_attn_forward - Y = concat_heads(attention) W_O + b_O + residual by the
  * tensor-parallel route: QKV column-parallel by whole heads (+ bias), local
  * attention per shard, W_O row-parallel into N partials, one sum
@@ -364,7 +388,7 @@ tp_status tp_mlp_forward_noalloc(const uint16_t* X, int64_t B, int64_t h,
 
 /* Workspace bytes for tp_mlp_forward (kind TP_WS_MLP), tp_attn_forward
  * (TP_WS_ATTN, ffn ignored), tp_layer_forward (TP_WS_LAYER) or
- * tp_layer_forward_sp (TP_WS_LAYER_SP). tokens =
+ * tp_layer_forward_sp (TP_WS_LAYER_SP) or tp_mlp_backward (TP_WS_MLP_BWD). tokens =
  * batch * seq. Returns 0 for invalid arguments. */
 size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn,
                           int n_shards);

@@ -64,19 +64,30 @@ struct GemmCfg {
 struct GemmParams {
   int M, Nc, K, G;
   int num_m, num_n, num_k, num_tiles;
-  int a_batched;
+  int a_batched, b_batched;
   int act;
   const uint16_t* bias;
+  const uint16_t* aux;  // EPI_DGELU: the pre-activation Z [G][M][Nc]
   unsigned* err;
 };
 
 // Epilogue kinds: bf16 + bias + activation (column-parallel), fp32 partials
-// (row-parallel), gated SiLU(gate) * up over interleaved 128-column blocks.
-enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU = 2 };
+// (row-parallel), gated SiLU(gate) * up over interleaved 128-column blocks,
+// and the GeLU backward: bf16 of acc * GeLU'(Z).
+enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU = 2, EPI_DGELU = 3 };
 
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + __expf(-x)); }
 
-template <int BN, int EPI, int CTAS>
+// d GeLU / dz = Phi(z) + z phi(z)
+__device__ __forceinline__ float gelu_grad(float z) {
+  return 0.5f * (1.0f + erff(z * 0.70710678118654752f)) +
+         z * 0.39894228040143268f * __expf(-0.5f * z * z);
+}
+
+// A_MN / B_MN: the operand is stored MN-major (its M, resp. N, index
+// contiguous; K strided), as the backward products need; it is loaded as
+// 64 x 64 boxes and described to the MMA as MN-major.
+template <int BN, int EPI, int CTAS, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -154,16 +165,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           const uint32_t sa = smem_u32(tiles + stage * C::kStageBytes);
-          if constexpr (CTAS == 2) {
-            // both CTAs' bytes are counted on the leader's full barrier
-            const uint32_t fb = mapa_shared(full_bar(stage), 0);
-            if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * C::kStageBytes);
-            tma_load_3d_pair(sa, &tmA, fb, kb * BK, arow, p.a_batched ? g : 0);
-            tma_load_3d_pair(sa + C::kABytes, &tmB, fb, kb * BK, brow, g);
+          const int ga = p.a_batched ? g : 0, gb = p.b_batched ? g : 0;
+          // both CTAs of a pair count their bytes on the leader's full barrier
+          const uint32_t fb = (CTAS == 2) ? mapa_shared(full_bar(stage), 0) : full_bar(stage);
+          if (leader)
+            mbar_arrive_expect_tx(full_bar(stage), CTAS * C::kStageBytes);
+          auto load = [&](uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2) {
+            if constexpr (CTAS == 2)
+              tma_load_3d_pair(dst, tm, fb, c0, c1, c2);
+            else
+              tma_load_3d(dst, tm, fb, c0, c1, c2);
+          };
+          if constexpr (A_MN) {
+            for (int j = 0; j < BM / 64; ++j) load(sa + j * 8192, &tmA, arow + 64 * j, kb * BK, ga);
           } else {
-            mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
-            tma_load_3d(sa, &tmA, full_bar(stage), kb * BK, arow, p.a_batched ? g : 0);
-            tma_load_3d(sa + C::kABytes, &tmB, full_bar(stage), kb * BK, brow, g);
+            load(sa, &tmA, kb * BK, arow, ga);
+          }
+          if constexpr (B_MN) {
+            for (int j = 0; j < C::kBRows / 64; ++j)
+              load(sa + C::kABytes + j * 8192, &tmB, brow + 64 * j, kb * BK, gb);
+          } else {
+            load(sa + C::kABytes, &tmB, kb * BK, brow, gb);
           }
           ++issued;
           if (++stage == C::kStages) {
@@ -189,7 +211,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(C::kTileM, BN);
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(C::kTileM, BN) | (A_MN ? (1u << 15) : 0u) |
+                                 (B_MN ? (1u << 16) : 0u);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -212,8 +235,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t sb = sa + C::kABytes;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = umma_desc_sw128(sa + kk * 32);
-            const uint64_t bd = umma_desc_sw128(sb + kk * 32);
+            const uint64_t ad =
+                A_MN ? umma_desc_sw128_mn(sa + kk * 2048, 8192) : umma_desc_sw128(sa + kk * 32);
+            const uint64_t bd =
+                B_MN ? umma_desc_sw128_mn(sb + kk * 2048, 8192) : umma_desc_sw128(sb + kk * 32);
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
             if constexpr (CTAS == 2)
               umma_bf16_pair(d_tmem, ad, bd, idesc, accum);
@@ -261,6 +286,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // output are clipped by the TMA unit). The next chunk's TMEM load is in
     // flight while the current chunk is converted and stored.
     constexpr bool OUT_F32 = EPI == EPI_F32;
+    constexpr bool DGELU = EPI == EPI_DGELU;
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const uint32_t sbase =
@@ -360,6 +386,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int e = 0; e < 8; ++e) v[e] = gelu_erf(v[e]);
             }
+            if constexpr (DGELU) {
+              if (col < p.Nc && row0 + lane < p.M) {
+                const uint4 zv = *reinterpret_cast<const uint4*>(
+                    p.aux + (static_cast<int64_t>(g) * p.M + row0 + lane) * p.Nc + col);
+                v[0] *= gelu_grad(bf16_lo(zv.x)); v[1] *= gelu_grad(bf16_hi(zv.x));
+                v[2] *= gelu_grad(bf16_lo(zv.y)); v[3] *= gelu_grad(bf16_hi(zv.y));
+                v[4] *= gelu_grad(bf16_lo(zv.z)); v[5] *= gelu_grad(bf16_hi(zv.z));
+                v[6] *= gelu_grad(bf16_lo(zv.w)); v[7] *= gelu_grad(bf16_hi(zv.w));
+              }
+            }
             w[4 * j + 0] = pack_bf16x2(v[0], v[1]);
             w[4 * j + 1] = pack_bf16x2(v[2], v[3]);
             w[4 * j + 2] = pack_bf16x2(v[4], v[5]);
@@ -451,13 +487,19 @@ static bool encode_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int EPI, int CTAS>
+template <int BN, int EPI, int CTAS, bool A_MN = false, bool B_MN = false>
 static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, int num_sms) {
   using C = GemmCfg<BN, CTAS>;
   constexpr bool OUT_F32 = EPI == EPI_F32;
   CUtensorMap tmA, tmB, tmD;
-  if (!encode_3d(&tmA, pr.A, pr.K, pr.M, pr.a_batched ? pr.G : 1, BK, BM)) return 1;
-  if (!encode_3d(&tmB, pr.B, pr.K, pr.Nc, pr.G, BK, C::kBRows)) return 1;
+  const uint64_t ga = pr.a_batched ? pr.G : 1, gb = pr.b_batched ? pr.G : 1;
+  // K-major: [g][rows][K] in boxes of 64 (K) x rows; MN-major: [g][K][rows] in 64 x 64 boxes
+  if (A_MN ? !encode_3d(&tmA, pr.A, pr.M, pr.K, ga, 64, 64)
+           : !encode_3d(&tmA, pr.A, pr.K, pr.M, ga, BK, BM))
+    return 1;
+  if (B_MN ? !encode_3d(&tmB, pr.B, pr.Nc, pr.K, gb, 64, 64)
+           : !encode_3d(&tmB, pr.B, pr.K, pr.Nc, gb, BK, C::kBRows))
+    return 1;
   const uint64_t out_cols = (EPI == EPI_SWIGLU) ? pr.Nc / 2 : pr.Nc;
   if (!encode_3d(&tmD, pr.D, out_cols, pr.M, pr.G, OUT_F32 ? 32 : 64, 32, OUT_F32)) return 1;
   GemmParams p;
@@ -470,10 +512,12 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
   p.num_k = (pr.K + BK - 1) / BK;
   p.num_tiles = p.num_m * p.num_n * pr.G;
   p.a_batched = pr.a_batched ? 1 : 0;
+  p.b_batched = pr.b_batched ? 1 : 0;
   p.act = pr.act;
   p.bias = static_cast<const uint16_t*>(pr.bias);
+  p.aux = static_cast<const uint16_t*>(pr.aux);
   p.err = err;
-  auto kern = gemm_tcgen05_kernel<BN, EPI, CTAS>;
+  auto kern = gemm_tcgen05_kernel<BN, EPI, CTAS, A_MN, B_MN>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kGemmThreads);
@@ -510,6 +554,19 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
 int launch_gemm(const GemmProblem& p, cudaStream_t s, unsigned* err, int num_sms) {
   const bool wide = p.Nc > 128;
   const bool pair = wide && p.M > BM;  // 256-row tiles only when there are rows to fill them
+  // backward products: 256-wide tiles, pairs when M > 128
+  if (p.act == 3) {  // dZ = (dY B_i^T) GeLU'(Z): A K-major, B MN-major
+    return p.M > BM ? launch_gemm_t<256, EPI_DGELU, 2, false, true>(p, s, err, num_sms)
+                    : launch_gemm_t<256, EPI_DGELU, 1, false, true>(p, s, err, num_sms);
+  }
+  if (p.a_mn && p.b_mn) {
+    return p.M > BM ? launch_gemm_t<256, EPI_F32, 2, true, true>(p, s, err, num_sms)
+                    : launch_gemm_t<256, EPI_F32, 1, true, true>(p, s, err, num_sms);
+  }
+  if (p.b_mn) {
+    return p.M > BM ? launch_gemm_t<256, EPI_F32, 2, false, true>(p, s, err, num_sms)
+                    : launch_gemm_t<256, EPI_F32, 1, false, true>(p, s, err, num_sms);
+  }
   if (p.act == 2) {  // gated: 256-wide tiles always (128 gate + 128 up columns)
     return p.M > BM ? launch_gemm_t<256, EPI_SWIGLU, 2>(p, s, err, num_sms)
                     : launch_gemm_t<256, EPI_SWIGLU, 1>(p, s, err, num_sms);

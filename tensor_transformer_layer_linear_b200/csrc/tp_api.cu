@@ -98,6 +98,7 @@ inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 inline size_t round256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 constexpr int64_t kIntMax = 2147483647;
+constexpr int kColsumSlabs = 64;
 
 tp_status gemm_status(int rc) {
   return rc == 0 ? TP_OK : TP_ERR_CUDA;
@@ -131,6 +132,9 @@ const char* tp_kernel_name(int kid) {
     case tpk::KID_LAYERNORM: return "layernorm";
     case tpk::KID_ATTENTION: return "attention";
     case tpk::KID_ALL_GATHER: return "all_gather_sequence";
+    case tpk::KID_GEMM_BACKWARD: return "gemm_backward";
+    case tpk::KID_ELEMENTWISE: return "gelu_elementwise";
+    case tpk::KID_COLSUM: return "column_sum";
     default: return "unknown";
   }
 }
@@ -417,6 +421,12 @@ size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int 
   }
   if (kind == TP_WS_ATTN) {
     return round256(M * 3 * H * 2) + round256(M * H * 2) + partials;
+  }
+  if (kind == TP_WS_MLP_BWD) {
+    if (ffn <= 0) return 0;
+    // Z, H, dZ [N][M][F/N] bf16; dX partials [N][M][h] fp32; column-sum slabs
+    return 3 * round256(M * static_cast<size_t>(ffn) * 2) + partials +
+           round256(static_cast<size_t>(kColsumSlabs) * (static_cast<size_t>(ffn) + H) * 4);
   }
   if (kind == TP_WS_LAYER || kind == TP_WS_LAYER_SP) {
     if (ffn <= 0) return 0;
@@ -735,5 +745,77 @@ tp_status tp_attn_forward_gqa(const uint16_t* X, int64_t batch, int64_t seq, int
   st = tp_row_linear(o, M, h, Wo_shards, h, n_shards, part, stream);
   if (st != TP_OK) return st;
   return tp_reduce_partials(part, n_shards, M, h, bo, residual, Y, stream);
+}
+
+tp_status tp_mlp_backward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, int n_shards,
+                          const uint16_t* A_shards, const uint16_t* b1_shards,
+                          const uint16_t* B_shards, const uint16_t* dY, int residual, void* ws,
+                          size_t ws_bytes, uint16_t* dX, float* dA_shards, float* db1,
+                          float* dB_shards, float* db2, void* stream) {
+  if (X == nullptr || A_shards == nullptr || B_shards == nullptr || dY == nullptr ||
+      dX == nullptr || dA_shards == nullptr || db1 == nullptr || dB_shards == nullptr ||
+      db2 == nullptr || ws == nullptr)
+    return TP_ERR_NULL;
+  if (B <= 0 || h <= 0 || ffn <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (ffn % n_shards || (ffn / n_shards) % 8 || h % 8) return TP_ERR_SHAPE;
+  if (B > kIntMax || h > kIntMax || ffn > kIntMax) return TP_ERR_SHAPE;
+  const size_t need = tp_workspace_bytes(TP_WS_MLP_BWD, B, h, ffn, n_shards);
+  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  if (!al16(ws) || !al16(X) || !al16(A_shards) || !al16(B_shards) || !al16(dY) || !al16(dX) ||
+      !al16(dA_shards) || !al16(db1) || !al16(dB_shards) || !al16(db2) ||
+      (b1_shards && !al16(b1_shards)))
+    return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  const int M = static_cast<int>(B), H = static_cast<int>(h), F = static_cast<int>(ffn);
+  const int fs = F / n_shards;
+  const size_t act_b = round256(static_cast<size_t>(M) * F * 2);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  uint16_t* Z = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* Hs = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* dZ = reinterpret_cast<uint16_t*>(p); p += act_b;
+  float* part = reinterpret_cast<float*>(p);
+  p += round256(static_cast<size_t>(n_shards) * M * H * 4);
+  float* slabs = reinterpret_cast<float*>(p);
+  cudaStream_t s = as_stream(stream);
+
+  // recompute the pre-activation Z_i = X A_i + b1_i and H_i = GeLU(Z_i)
+  st = tp_column_linear(X, B, h, A_shards, b1_shards, ffn, n_shards, TP_ACT_NONE, Z, stream);
+  if (st != TP_OK) return st;
+  {
+    TraceScope ts(tpk::KID_ELEMENTWISE, s);
+    if (tpk::launch_gelu_bf16(Z, Hs, static_cast<int64_t>(M) * F, s, d.num_sms) != 0)
+      return TP_ERR_CUDA;
+  }
+  auto gemm = [&](const void* A, bool a_b, bool a_mn, const void* Bop, bool b_b, bool b_mn,
+                  void* D, int m, int nc, int k, bool f32, int act, const void* aux) {
+    tpk::GemmProblem g;
+    g.A = A; g.B = Bop; g.D = D; g.bias = nullptr;
+    g.M = m; g.Nc = nc; g.K = k; g.G = n_shards;
+    g.a_batched = a_b; g.b_batched = b_b; g.a_mn = a_mn; g.b_mn = b_mn;
+    g.out_f32 = f32; g.act = act; g.aux = aux;
+    TraceScope ts(tpk::KID_GEMM_BACKWARD, s);
+    return tpk::launch_gemm(g, s, d.err, d.num_sms) == 0 ? TP_OK : TP_ERR_CUDA;
+  };
+  // dZ_i = (dY B_i^T) * GeLU'(Z_i): dY shared; B_shards[i] = B_i^T is the MN-major operand
+  st = gemm(dY, false, false, B_shards, true, true, dZ, M, fs, H, false, 3, Z);
+  if (st != TP_OK) return st;
+  // dX partials: dZ_i A_i^T; A_shards[i] = A_i^T is the MN-major operand
+  st = gemm(dZ, true, false, A_shards, true, true, part, M, H, fs, true, 0, nullptr);
+  if (st != TP_OK) return st;
+  // the one reduction of the backward: dX = sum_i dX_i (+ dY through the residual)
+  st = tp_reduce_partials(part, n_shards, B, h, nullptr, residual ? dY : nullptr, dX, stream);
+  if (st != TP_OK) return st;
+  // dA_i^T = dZ_i^T X (packed like A_shards), dB_i^T = dY^T H_i (packed like B_shards)
+  st = gemm(dZ, true, true, X, false, true, dA_shards, fs, H, M, true, 0, nullptr);
+  if (st != TP_OK) return st;
+  st = gemm(dY, false, true, Hs, true, true, dB_shards, H, fs, M, true, 0, nullptr);
+  if (st != TP_OK) return st;
+  // bias gradients: column sums over the token rows
+  TraceScope ts(tpk::KID_COLSUM, s);
+  if (tpk::launch_colsum(dZ, n_shards, M, fs, slabs, kColsumSlabs, db1, s) != 0) return TP_ERR_CUDA;
+  if (tpk::launch_colsum(dY, 1, M, H, slabs, kColsumSlabs, db2, s) != 0) return TP_ERR_CUDA;
+  return TP_OK;
 }
 }  // extern "C"

@@ -16,13 +16,21 @@ enum KernelId {
   KID_LAYERNORM = 5,
   KID_ATTENTION = 6,
   KID_ALL_GATHER = 7,
-  KID_COUNT = 8
+  KID_GEMM_BACKWARD = 8,
+  KID_ELEMENTWISE = 9,
+  KID_COLSUM = 10,
+  KID_COUNT = 11
 };
 
 // One batched GEMM over G shards: D[g] (M x Nc) = A[g] (M x K) . B[g]^T with
 // A [G_A][M][K] (G_A = G when a_batched, else 1: the replicated input) and
 // B [G][Nc][K], both K-major bf16. D [G][M][Nc] is either bf16 with an
 // optional bias [G][Nc] and activation, or fp32 (no bias, no activation).
+//
+// Backward variants: with a_mn (b_mn) the operand is MN-major, A [G_A][K][M]
+// (B [G_B][K][Nc]); b_batched = false shares B across the batch; act 3 is the
+// GeLU backward epilogue D = bf16(acc * GeLU'(aux)), aux [G][M][Nc] bf16.
+// MN-major products write fp32 (act 0, out_f32).
 struct GemmProblem {
   const void* A;
   const void* B;
@@ -31,7 +39,11 @@ struct GemmProblem {
   int M, Nc, K, G;
   bool a_batched;
   bool out_f32;
-  int act;  // 0 none, 1 GeLU (erf form), 2 gated SiLU(gate) * up (D has Nc / 2 columns)
+  int act;  // 0 none, 1 GeLU (erf form), 2 gated SiLU(gate) * up (D has Nc / 2 columns), 3 GeLU'
+  bool b_batched = true;
+  bool a_mn = false;
+  bool b_mn = false;
+  const void* aux = nullptr;
 };
 
 // Returns 0 on success, 1 if a tensor map could not be encoded, 2 if the
@@ -74,5 +86,13 @@ int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, i
 // QKV with n_q query and n_kv key/value heads of head_dim).
 int launch_shard(const void* W, int64_t h_in, int64_t h_out, int n_shards, int kind,
                  int64_t head_dim, void* out, cudaStream_t s, int64_t n_q = 0, int64_t n_kv = 0);
+
+// H = GeLU(Z) element-wise, bf16 in and out; n % 8 == 0.
+int launch_gelu_bf16(const void* Z, void* H, int64_t n, cudaStream_t s, int num_sms);
+
+// out[g][c] = sum_r X[g][r][c] (bf16 in, fp32 out) in two deterministic
+// passes through partial[groups][slabs][cols]. cols % 8 == 0.
+int launch_colsum(const void* X, int groups, int rows, int cols, float* partial, int slabs,
+                  float* out, cudaStream_t s);
 
 }  // namespace tpk

@@ -31,7 +31,7 @@ TP_OK, TP_ERR_NULL, TP_ERR_SHAPE, TP_ERR_ALIGN = 0, 1, 2, 3
 TP_ERR_WORKSPACE, TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_TIMEOUT = 4, 5, 6, 7
 TP_SPLIT_COLUMN, TP_SPLIT_ROW, TP_SPLIT_QKV_HEADS, TP_SPLIT_GATE_UP = 0, 1, 2, 3
 TP_ACT_NONE, TP_ACT_GELU_ERF, TP_ACT_SWIGLU = 0, 1, 2
-TP_WS_MLP, TP_WS_ATTN, TP_WS_LAYER, TP_WS_LAYER_SP = 0, 1, 2, 3
+TP_WS_MLP, TP_WS_ATTN, TP_WS_LAYER, TP_WS_LAYER_SP, TP_WS_MLP_BWD = 0, 1, 2, 3, 4
 
 _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
@@ -70,6 +70,8 @@ _SIGS = {
     "tp_attention_gqa": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp]),
     "tp_attn_forward_gqa": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp,
                                    _vp, _vp, _vp, _sz, _vp, _vp]),
+    "tp_mlp_backward": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _sz,
+                               _vp, _vp, _vp, _vp, _vp, _vp]),
     "tp_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "tp_get_last_error": (_i32, [_vp]),
     "tp_status_string": (ctypes.c_char_p, [_i32]),
@@ -268,6 +270,14 @@ def tp_attn_forward_gqa(X, batch, seq, h, n_q, n_kv, causal, n_shards, Wqkv_shar
                                    _p(Wqkv_shards), _p(bqkv_shards), _p(Wo_shards), _p(bo),
                                    _p(residual), _p(ws), ws_bytes, _p(Y), _s(stream)),
            "tp_attn_forward_gqa")
+
+
+def tp_mlp_backward(X, B, h, ffn, n_shards, A_shards, b1_shards, B_shards, dY, residual, ws,
+                    ws_bytes, dX, dA_shards, db1, dB_shards, db2, stream=None):
+    _check(lib.tp_mlp_backward(_p(X), B, h, ffn, n_shards, _p(A_shards), _p(b1_shards),
+                               _p(B_shards), _p(dY), int(bool(residual)), _p(ws), ws_bytes, _p(dX),
+                               _p(dA_shards), _p(db1), _p(dB_shards), _p(db2), _s(stream)),
+           "tp_mlp_backward")
 
 
 def tp_get_last_error(stream=None) -> int:
