@@ -237,7 +237,8 @@ tp_status tp_mlp_forward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn,
  * tensor-parallel route ([TP-LLM] MLP block: exactly one all-reduce in the
  * backward pass, of the input gradient across the column-parallel layer).
  * dY reaches every shard whole (the row-parallel layer's backward needs no
- * exchange); each shard recomputes Z_i = X A_i + b1_i, forms
+ * exchange); each shard recomputes Z_i = X A_i + b1_i (one GEMM whose
+ * epilogue emits GeLU(Z_i) and GeLU'(Z_i), both stored as bf16), forms
  * dZ_i = (dY B_i^T) * GeLU'(Z_i), its weight gradients locally, and a
  * full-size partial dX_i = dZ_i A_i^T; dX = sum_i dX_i (+ dY when residual)
  * is the one reduction.

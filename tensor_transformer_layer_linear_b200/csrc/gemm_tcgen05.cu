@@ -67,22 +67,20 @@ struct GemmParams {
   int a_batched, b_batched;
   int act;
   const uint16_t* bias;
-  const uint16_t* aux;  // EPI_DGELU: the pre-activation Z [G][M][Nc]
+  const uint16_t* aux;  // EPI_MUL_AUX: the factor GeLU'(Z) [G][M][Nc] bf16
+  uint16_t* aux_out;    // EPI_GELU_AUX: receives GeLU'(Z) [G][M][Nc] bf16
   unsigned* err;
 };
 
 // Epilogue kinds: bf16 + bias + activation (column-parallel), fp32 partials
 // (row-parallel), gated SiLU(gate) * up over interleaved 128-column blocks,
-// and the GeLU backward: bf16 of acc * GeLU'(Z).
-enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU = 2, EPI_DGELU = 3 };
+// the GeLU backward bf16(acc * GeLU'(Z)) with GeLU'(Z) read from aux, and the
+// backward's recompute of the column layer: bf16 GeLU(Z) out, GeLU'(Z) to
+// aux_out (Z = acc + bias).
+enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU = 2, EPI_MUL_AUX = 3, EPI_GELU_AUX = 4 };
 
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + __expf(-x)); }
 
-// d GeLU / dz = Phi(z) + z phi(z)
-__device__ __forceinline__ float gelu_grad(float z) {
-  return 0.5f * (1.0f + erff(z * 0.70710678118654752f)) +
-         z * 0.39894228040143268f * __expf(-0.5f * z * z);
-}
 
 // A_MN / B_MN: the operand is stored MN-major (its M, resp. N, index
 // contiguous; K strided), as the backward products need; it is loaded as
@@ -91,7 +89,8 @@ template <int BN, int EPI, int CTAS, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmD,
+                        const __grid_constant__ CUtensorMap tmE, const GemmParams p) {
   using C = GemmCfg<BN, CTAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -132,6 +131,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmD);
+    if constexpr (EPI == EPI_GELU_AUX) tma_prefetch_desc(&tmE);
   }
   if (warp == 1) {
     if constexpr (CTAS == 2)
@@ -286,7 +286,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // output are clipped by the TMA unit). The next chunk's TMEM load is in
     // flight while the current chunk is converted and stored.
     constexpr bool OUT_F32 = EPI == EPI_F32;
-    constexpr bool DGELU = EPI == EPI_DGELU;
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const uint32_t sbase =
@@ -353,6 +352,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t r[2][CW];
       tmem_ld_32x32b_x32(tbase, &r[0][0]);
       if constexpr (!OUT_F32) tmem_ld_32x32b_x32(tbase + 32, &r[0][32]);
+      const bool row_ok = row0 + lane < p.M;
+      const int64_t aux_row = (static_cast<int64_t>(g) * p.M + row0 + lane) * p.Nc;
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
         tmem_ld_wait();  // chunk c has arrived
@@ -364,6 +365,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (col0 >= p.Nc) continue;  // warp-uniform: the whole chunk is past the edge
         const uint32_t* rc = r[c & 1];
         uint32_t w[32];  // this thread's 128-byte row of the chunk
+        uint32_t wg[(EPI == EPI_GELU_AUX) ? 32 : 1];  // and of GeLU'(Z)
         if constexpr (OUT_F32) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) w[e] = rc[e];
@@ -386,15 +388,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int e = 0; e < 8; ++e) v[e] = gelu_erf(v[e]);
             }
-            if constexpr (DGELU) {
-              if (col < p.Nc && row0 + lane < p.M) {
-                const uint4 zv = *reinterpret_cast<const uint4*>(
-                    p.aux + (static_cast<int64_t>(g) * p.M + row0 + lane) * p.Nc + col);
-                v[0] *= gelu_grad(bf16_lo(zv.x)); v[1] *= gelu_grad(bf16_hi(zv.x));
-                v[2] *= gelu_grad(bf16_lo(zv.y)); v[3] *= gelu_grad(bf16_hi(zv.y));
-                v[4] *= gelu_grad(bf16_lo(zv.z)); v[5] *= gelu_grad(bf16_hi(zv.z));
-                v[6] *= gelu_grad(bf16_lo(zv.w)); v[7] *= gelu_grad(bf16_hi(zv.w));
-              }
+            if constexpr (EPI == EPI_MUL_AUX) {
+              uint4 gz = make_uint4(0u, 0u, 0u, 0u);
+              if (row_ok && col < p.Nc)
+                gz = __ldcs(reinterpret_cast<const uint4*>(p.aux + aux_row + col));
+              v[0] *= bf16_lo(gz.x); v[1] *= bf16_hi(gz.x);
+              v[2] *= bf16_lo(gz.y); v[3] *= bf16_hi(gz.y);
+              v[4] *= bf16_lo(gz.z); v[5] *= bf16_hi(gz.z);
+              v[6] *= bf16_lo(gz.w); v[7] *= bf16_hi(gz.w);
+            }
+            if constexpr (EPI == EPI_GELU_AUX) {
+              float gr[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = gelu_erf_with_grad(v[e], &gr[e]);
+              wg[4 * j + 0] = pack_bf16x2(gr[0], gr[1]);
+              wg[4 * j + 1] = pack_bf16x2(gr[2], gr[3]);
+              wg[4 * j + 2] = pack_bf16x2(gr[4], gr[5]);
+              wg[4 * j + 3] = pack_bf16x2(gr[6], gr[7]);
             }
             w[4 * j + 0] = pack_bf16x2(v[0], v[1]);
             w[4 * j + 1] = pack_bf16x2(v[2], v[3]);
@@ -416,6 +426,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) {
           tma_store_3d(&tmD, sbuf, col0, row0, g);
           bulk_commit();
+        }
+        if constexpr (EPI == EPI_GELU_AUX) {
+          // the same staging rows, once the store above has read them
+          if (lane == 0) bulk_wait_read<0>();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4), wg[4 * j],
+                         wg[4 * j + 1], wg[4 * j + 2], wg[4 * j + 3]);
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmE, sbuf, col0, row0, g);
+            bulk_commit();
+          }
         }
       }
       }  // EPI
@@ -491,7 +516,7 @@ template <int BN, int EPI, int CTAS, bool A_MN = false, bool B_MN = false>
 static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, int num_sms) {
   using C = GemmCfg<BN, CTAS>;
   constexpr bool OUT_F32 = EPI == EPI_F32;
-  CUtensorMap tmA, tmB, tmD;
+  CUtensorMap tmA, tmB, tmD, tmE;
   const uint64_t ga = pr.a_batched ? pr.G : 1, gb = pr.b_batched ? pr.G : 1;
   // K-major: [g][rows][K] in boxes of 64 (K) x rows; MN-major: [g][K][rows] in 64 x 64 boxes
   if (A_MN ? !encode_3d(&tmA, pr.A, pr.M, pr.K, ga, 64, 64)
@@ -502,6 +527,9 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
     return 1;
   const uint64_t out_cols = (EPI == EPI_SWIGLU) ? pr.Nc / 2 : pr.Nc;
   if (!encode_3d(&tmD, pr.D, out_cols, pr.M, pr.G, OUT_F32 ? 32 : 64, 32, OUT_F32)) return 1;
+  tmE = tmD;  // GeLU' output (same shape as D) for EPI_GELU_AUX only
+  if (EPI == EPI_GELU_AUX && !encode_3d(&tmE, pr.aux_out, out_cols, pr.M, pr.G, 64, 32, false))
+    return 1;
   GemmParams p;
   p.M = pr.M;
   p.Nc = pr.Nc;
@@ -516,6 +544,7 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
   p.act = pr.act;
   p.bias = static_cast<const uint16_t*>(pr.bias);
   p.aux = static_cast<const uint16_t*>(pr.aux);
+  p.aux_out = static_cast<uint16_t*>(pr.aux_out);
   p.err = err;
   auto kern = gemm_tcgen05_kernel<BN, EPI, CTAS, A_MN, B_MN>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -547,7 +576,7 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
   }
   const int units = p.num_tiles < resident_units ? p.num_tiles : resident_units;
   cfg.gridDim = dim3(static_cast<unsigned>(units * CTAS));
-  if (cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, p) != cudaSuccess) return 2;
+  if (cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmD, tmE, p) != cudaSuccess) return 2;
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
 
@@ -556,8 +585,12 @@ int launch_gemm(const GemmProblem& p, cudaStream_t s, unsigned* err, int num_sms
   const bool pair = wide && p.M > BM;  // 256-row tiles only when there are rows to fill them
   // backward products: 256-wide tiles, pairs when M > 128
   if (p.act == 3) {  // dZ = (dY B_i^T) GeLU'(Z): A K-major, B MN-major
-    return p.M > BM ? launch_gemm_t<256, EPI_DGELU, 2, false, true>(p, s, err, num_sms)
-                    : launch_gemm_t<256, EPI_DGELU, 1, false, true>(p, s, err, num_sms);
+    return p.M > BM ? launch_gemm_t<256, EPI_MUL_AUX, 2, false, true>(p, s, err, num_sms)
+                    : launch_gemm_t<256, EPI_MUL_AUX, 1, false, true>(p, s, err, num_sms);
+  }
+  if (p.act == 4) {  // recompute: GeLU(X A_i + b_i) and GeLU' of it
+    return p.M > BM ? launch_gemm_t<256, EPI_GELU_AUX, 2>(p, s, err, num_sms)
+                    : launch_gemm_t<256, EPI_GELU_AUX, 1>(p, s, err, num_sms);
   }
   if (p.a_mn && p.b_mn) {
     return p.M > BM ? launch_gemm_t<256, EPI_F32, 2, true, true>(p, s, err, num_sms)

@@ -98,7 +98,7 @@ inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 inline size_t round256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 constexpr int64_t kIntMax = 2147483647;
-constexpr int kColsumSlabs = 64;
+constexpr int kColsumSlabs = 256;  // upper bound on the column-sum slabs
 
 tp_status gemm_status(int rc) {
   return rc == 0 ? TP_OK : TP_ERR_CUDA;
@@ -424,7 +424,7 @@ size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int 
   }
   if (kind == TP_WS_MLP_BWD) {
     if (ffn <= 0) return 0;
-    // Z, H, dZ [N][M][F/N] bf16; dX partials [N][M][h] fp32; column-sum slabs
+    // GeLU'(Z), H, dZ [N][M][F/N] bf16; dX partials [N][M][h] fp32; column-sum slabs
     return 3 * round256(M * static_cast<size_t>(ffn) * 2) + partials +
            round256(static_cast<size_t>(kColsumSlabs) * (static_cast<size_t>(ffn) + H) * 4);
   }
@@ -772,7 +772,7 @@ tp_status tp_mlp_backward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, 
   const int fs = F / n_shards;
   const size_t act_b = round256(static_cast<size_t>(M) * F * 2);
   uint8_t* p = static_cast<uint8_t*>(ws);
-  uint16_t* Z = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* Gp = reinterpret_cast<uint16_t*>(p); p += act_b;
   uint16_t* Hs = reinterpret_cast<uint16_t*>(p); p += act_b;
   uint16_t* dZ = reinterpret_cast<uint16_t*>(p); p += act_b;
   float* part = reinterpret_cast<float*>(p);
@@ -780,26 +780,25 @@ tp_status tp_mlp_backward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, 
   float* slabs = reinterpret_cast<float*>(p);
   cudaStream_t s = as_stream(stream);
 
-  // recompute the pre-activation Z_i = X A_i + b1_i and H_i = GeLU(Z_i)
-  st = tp_column_linear(X, B, h, A_shards, b1_shards, ffn, n_shards, TP_ACT_NONE, Z, stream);
-  if (st != TP_OK) return st;
-  {
-    TraceScope ts(tpk::KID_ELEMENTWISE, s);
-    if (tpk::launch_gelu_bf16(Z, Hs, static_cast<int64_t>(M) * F, s, d.num_sms) != 0)
-      return TP_ERR_CUDA;
-  }
   auto gemm = [&](const void* A, bool a_b, bool a_mn, const void* Bop, bool b_b, bool b_mn,
-                  void* D, int m, int nc, int k, bool f32, int act, const void* aux) {
+                  void* D, int m, int nc, int k, bool f32, int act, const void* aux,
+                  const void* bias = nullptr, void* aux_out = nullptr,
+                  int kid = tpk::KID_GEMM_BACKWARD) {
     tpk::GemmProblem g;
-    g.A = A; g.B = Bop; g.D = D; g.bias = nullptr;
+    g.A = A; g.B = Bop; g.D = D; g.bias = bias;
     g.M = m; g.Nc = nc; g.K = k; g.G = n_shards;
     g.a_batched = a_b; g.b_batched = b_b; g.a_mn = a_mn; g.b_mn = b_mn;
-    g.out_f32 = f32; g.act = act; g.aux = aux;
-    TraceScope ts(tpk::KID_GEMM_BACKWARD, s);
+    g.out_f32 = f32; g.act = act; g.aux = aux; g.aux_out = aux_out;
+    TraceScope ts(kid, s);
     return tpk::launch_gemm(g, s, d.err, d.num_sms) == 0 ? TP_OK : TP_ERR_CUDA;
   };
+  // recompute the column layer: H_i = GeLU(Z_i), Z_i = X A_i + b1_i, with
+  // GeLU'(Z_i) kept for the backward of the activation
+  st = gemm(X, false, false, A_shards, true, false, Hs, M, fs, H, false, 4, nullptr, b1_shards,
+            Gp, tpk::KID_GEMM_COLUMN);
+  if (st != TP_OK) return st;
   // dZ_i = (dY B_i^T) * GeLU'(Z_i): dY shared; B_shards[i] = B_i^T is the MN-major operand
-  st = gemm(dY, false, false, B_shards, true, true, dZ, M, fs, H, false, 3, Z);
+  st = gemm(dY, false, false, B_shards, true, true, dZ, M, fs, H, false, 3, Gp);
   if (st != TP_OK) return st;
   // dX partials: dZ_i A_i^T; A_shards[i] = A_i^T is the MN-major operand
   st = gemm(dZ, true, false, A_shards, true, true, part, M, H, fs, true, 0, nullptr);
@@ -814,8 +813,10 @@ tp_status tp_mlp_backward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, 
   if (st != TP_OK) return st;
   // bias gradients: column sums over the token rows
   TraceScope ts(tpk::KID_COLSUM, s);
-  if (tpk::launch_colsum(dZ, n_shards, M, fs, slabs, kColsumSlabs, db1, s) != 0) return TP_ERR_CUDA;
-  if (tpk::launch_colsum(dY, 1, M, H, slabs, kColsumSlabs, db2, s) != 0) return TP_ERR_CUDA;
+  if (tpk::launch_colsum(dZ, n_shards, M, fs, slabs, kColsumSlabs, db1, s, d.num_sms) != 0)
+    return TP_ERR_CUDA;
+  if (tpk::launch_colsum(dY, 1, M, H, slabs, kColsumSlabs, db2, s, d.num_sms) != 0)
+    return TP_ERR_CUDA;
   return TP_OK;
 }
 }  // extern "C"

@@ -368,8 +368,43 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
+// GeLU in its erf form, GeLU(z) = z Phi(z), Phi the standard normal CDF.
 __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
+
+// GeLU(z) together with GeLU'(z) = Phi(z) + z phi(z), phi the normal density,
+// for the backward's recompute. Phi is formed from the complementary error
+// function in the rational-times-exponential form of Abramowitz & Stegun,
+// "Handbook of Mathematical Functions", eq. 7.1.26:
+// erfc(x) ~= t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-x^2),
+// t = 1 / (1 + p x), x >= 0, |error| <= 1.5e-7. At x = |z| / sqrt 2 the factor
+// exp(-x^2) = exp(-z^2 / 2) is also phi(z) sqrt(2 pi), so value and
+// derivative share one exponential (where erff and a separate exponential
+// measured slower); for z < 0, Phi(z) = erfc(|z| / sqrt 2) / 2 is taken
+// without cancellation.
+struct GeluAS {
+  static constexpr float p = 0.3275911f;
+  static constexpr float a1 = 0.254829592f, a2 = -0.284496736f, a3 = 1.421413741f,
+                         a4 = -1.453152027f, a5 = 1.061405429f;
+};
+
+__device__ __forceinline__ float normal_cdf_parts(float z, float* gauss) {
+  const float x = fabsf(z) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(GeluAS::p, x, 1.0f));
+  const float poly =
+      t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, GeluAS::a5, GeluAS::a4), GeluAS::a3), GeluAS::a2),
+               GeluAS::a1);
+  *gauss = __expf(-0.5f * z * z);  // exp(-z^2 / 2)
+  const float half_erfc = 0.5f * poly * *gauss;
+  return z >= 0.0f ? 1.0f - half_erfc : half_erfc;
+}
+
+__device__ __forceinline__ float gelu_erf_with_grad(float z, float* grad) {
+  float g;
+  const float cdf = normal_cdf_parts(z, &g);
+  *grad = fmaf(z * 0.39894228040143268f, g, cdf);  // Phi + z exp(-z^2/2) / sqrt(2 pi)
+  return z * cdf;
 }
 
 }  // namespace tpk

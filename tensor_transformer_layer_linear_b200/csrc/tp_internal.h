@@ -29,8 +29,10 @@ enum KernelId {
 //
 // Backward variants: with a_mn (b_mn) the operand is MN-major, A [G_A][K][M]
 // (B [G_B][K][Nc]); b_batched = false shares B across the batch; act 3 is the
-// GeLU backward epilogue D = bf16(acc * GeLU'(aux)), aux [G][M][Nc] bf16.
-// MN-major products write fp32 (act 0, out_f32).
+// GeLU backward epilogue D = bf16(acc * aux), aux = GeLU'(Z) [G][M][Nc] bf16;
+// act 4 is the forward recompute D = bf16(GeLU(acc + bias)) that also writes
+// aux_out = bf16(GeLU'(acc + bias)) [G][M][Nc]. MN-major products write fp32
+// (act 0, out_f32).
 struct GemmProblem {
   const void* A;
   const void* B;
@@ -39,11 +41,13 @@ struct GemmProblem {
   int M, Nc, K, G;
   bool a_batched;
   bool out_f32;
-  int act;  // 0 none, 1 GeLU (erf form), 2 gated SiLU(gate) * up (D has Nc / 2 columns), 3 GeLU'
+  int act;  // 0 none, 1 GeLU (erf form), 2 gated SiLU(gate) * up (D has Nc / 2 columns),
+            // 3 times aux, 4 GeLU with GeLU' to aux_out
   bool b_batched = true;
   bool a_mn = false;
   bool b_mn = false;
   const void* aux = nullptr;
+  void* aux_out = nullptr;
 };
 
 // Returns 0 on success, 1 if a tensor map could not be encoded, 2 if the
@@ -87,12 +91,10 @@ int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, i
 int launch_shard(const void* W, int64_t h_in, int64_t h_out, int n_shards, int kind,
                  int64_t head_dim, void* out, cudaStream_t s, int64_t n_q = 0, int64_t n_kv = 0);
 
-// H = GeLU(Z) element-wise, bf16 in and out; n % 8 == 0.
-int launch_gelu_bf16(const void* Z, void* H, int64_t n, cudaStream_t s, int num_sms);
-
 // out[g][c] = sum_r X[g][r][c] (bf16 in, fp32 out) in two deterministic
-// passes through partial[groups][slabs][cols]. cols % 8 == 0.
-int launch_colsum(const void* X, int groups, int rows, int cols, float* partial, int slabs,
-                  float* out, cudaStream_t s);
+// passes through partial[groups][slabs][cols], slabs <= max_slabs chosen to
+// fill the GPU. cols % 8 == 0.
+int launch_colsum(const void* X, int groups, int rows, int cols, float* partial, int max_slabs,
+                  float* out, cudaStream_t s, int num_sms);
 
 }  // namespace tpk

@@ -114,6 +114,26 @@ def test_column_linear_random(tp, n, act):
     assert_parity(np.concatenate(list(got), axis=1), O.gelu(full) if act else full, "gather")
 
 
+def test_column_linear_gelu_pointwise(tp):
+    """With an identity weight the column GEMM's epilogue applies GeLU to each
+    input value exactly (the products and sums are exact), so the output can
+    be held to one bf16 rounding of the true erf GeLU at 16384 points."""
+    z = np.linspace(-8.0, 8.0, 256 * 64).astype(np.float32)
+    z[:4] = [0.0, 1e-30, -1e-30, -0.0]
+    X = synth.f32_to_bf16_bits(z).reshape(256, 64)
+    W = synth.f32_to_bf16_bits(np.eye(64, dtype=np.float32))
+    Y = torch.empty((1, 256, 64), dtype=torch.int16, device="cuda")
+    tp.tp_column_linear(to_dev(X), 256, 64, _shard(tp, W, 0, 1), None, 64, 1, 1, Y)
+    zx = f64(X)
+    ref = O.gelu(zx)
+    got = from_dev_bf16(Y)[0]
+    # bf16 keeps 8 significant bits: one rounding is within 2^-8 relative; the
+    # absolute floor covers the far negative tail where GeLU is ~1e-9
+    tol = np.maximum(2.0 ** -8 * np.abs(ref), 1e-7 * np.abs(zx))
+    bad = np.abs(got - ref) > tol
+    assert not bad.any(), (zx[bad][:5], got[bad][:5], ref[bad][:5])
+
+
 def test_column_linear_qkv_heads(tp):
     rng = np.random.default_rng(450)
     M, h, d, n = 192, 512, 128, 2
