@@ -437,6 +437,149 @@ def mlp_backward_sharded(X, A, b1, B, dY, n_shards: int, residual: bool = True) 
 
 
 # --------------------------------------------------------------------------
+# attention-block and layer backward ([TP-LLM] "Communication Budget and
+# Scaling Limits": two all-reduces in the forward pass and two in the
+# backward pass of every layer, one per block)
+# --------------------------------------------------------------------------
+
+def attention_head_backward(Q, K, V, dO, causal: bool) -> tuple:
+    """Gradients of O = softmax(Q K^T / sqrt d) V for one head of one
+    sequence, given dO = dL/dO: (dQ, dK, dV). The chain rule through the
+    three steps S = Q K^T / sqrt d, P = softmax_rows(S), O = P V:
+    dV = P^T dO, dP = dO V^T, dS = P * (dP - rowsum(dP * P)) (the softmax
+    Jacobian applied row by row), dQ = dS K / sqrt d, dK = dS^T Q / sqrt d.
+    Masked (causal) entries have P = 0 and receive no gradient."""
+    d = Q.shape[1]
+    S = (Q @ K.T) / math.sqrt(d)
+    if causal:
+        t = np.arange(Q.shape[0])[:, None]
+        s = np.arange(K.shape[0])[None, :]
+        S = np.where(s <= t, S, -np.inf)
+    P = softmax_rows(S)
+    dV = P.T @ dO
+    dP = dO @ V.T
+    dS = P * (dP - np.sum(dP * P, axis=1, keepdims=True))
+    return dS @ K / math.sqrt(d), dS.T @ Q / math.sqrt(d), dV
+
+
+def attention_heads_backward(Q, K, V, dO, batch: int, seq: int, n_heads: int,
+                             causal: bool) -> tuple:
+    """attention_head_backward for every (sequence, head) pair; head k is
+    columns [k d, (k+1) d) of Q, K, V, dO. Returns (dQ, dK, dV) [M][h]."""
+    M, h = Q.shape
+    d = h // n_heads
+    dQ, dK, dV = np.zeros((M, h)), np.zeros((M, h)), np.zeros((M, h))
+    for s in range(batch):
+        r = slice(s * seq, (s + 1) * seq)
+        for k in range(n_heads):
+            c = slice(k * d, (k + 1) * d)
+            dQ[r, c], dK[r, c], dV[r, c] = attention_head_backward(
+                Q[r, c], K[r, c], V[r, c], dO[r, c], causal)
+    return dQ, dK, dV
+
+
+def self_attention_backward(X, Wqkv, bqkv, Wo, bo, dY, batch: int, seq: int,
+                            n_heads: int, causal: bool = True,
+                            residual: bool = True) -> dict:
+    """Gradients of Y = concat_heads(attention) W_O + b_O (+ X) given dY
+    (unsharded): dX, dWqkv, dbqkv, dWo, dbo."""
+    h = X.shape[1]
+    QKV = linear(X, Wqkv, bqkv)
+    Q, K, V = QKV[:, :h], QKV[:, h:2 * h], QKV[:, 2 * h:]
+    O = attention_heads(Q, K, V, batch, seq, n_heads, causal)
+    dO = dY @ Wo.T
+    dQ, dK, dV = attention_heads_backward(Q, K, V, dO, batch, seq, n_heads, causal)
+    dQKV = np.concatenate([dQ, dK, dV], axis=1)
+    dX = dQKV @ Wqkv.T
+    if residual:
+        dX = dX + dY
+    return dict(dX=dX, dWqkv=X.T @ dQKV, dbqkv=dQKV.sum(axis=0), dWo=O.T @ dY,
+                dbo=dY.sum(axis=0))
+
+
+def self_attention_backward_sharded(X, Wqkv, bqkv, Wo, bo, dY, batch: int,
+                                    seq: int, n_heads: int, n_shards: int,
+                                    causal: bool = True,
+                                    residual: bool = True) -> dict:
+    """The tensor-parallel backward of the attention block: dY reaches every
+    shard whole (the backward of the row-parallel W_O needs no exchange);
+    shard i forms dO_i = dY W_O,i^T, the attention backward of its own heads,
+    dQKV_i = [dQ_i | dK_i | dV_i], its weight gradients dW_QKV,i = X^T dQKV_i,
+    db_QKV,i, dW_O,i = O_i^T dY locally, and a full-size partial
+    dX_i = dQKV_i W_QKV,i^T; the one reduction is dX = sum_i dX_i (+ dY).
+    The gradients of the sharded weights are returned in the unsharded
+    orientation (the shards' pieces put back in place)."""
+    h = X.shape[1]
+    d = h // n_heads
+    hs = h // n_shards
+    hps = n_heads // n_shards
+    owner, local = shard_index_map(SPLIT_QKV_HEADS, h, 3 * h, n_shards, d)
+    Wqkv_i = shard_matrices(Wqkv, SPLIT_QKV_HEADS, n_shards, d)
+    bqkv_i = shard_matrices(np.asarray(bqkv).reshape(1, -1), SPLIT_QKV_HEADS, n_shards, d)
+    Wo_i = shard_matrices(Wo, SPLIT_ROW, n_shards)
+    parts, dqkv_shards = [], []
+    dWqkv, dbqkv = np.zeros((h, 3 * h)), np.zeros(3 * h)
+    dWo = np.zeros((h, h))
+    for i in range(n_shards):
+        QKV = linear(X, Wqkv_i[i], bqkv_i[i][0])
+        Q, K, V = QKV[:, :hs], QKV[:, hs:2 * hs], QKV[:, 2 * hs:]
+        O = attention_heads(Q, K, V, batch, seq, hps, causal)
+        dO = dY @ Wo_i[i].T
+        dQ, dK, dV = attention_heads_backward(Q, K, V, dO, batch, seq, hps, causal)
+        dQKV = np.concatenate([dQ, dK, dV], axis=1)
+        dqkv_shards.append(dQKV)
+        parts.append(dQKV @ Wqkv_i[i].T)
+        mine = owner == i                      # W_QKV columns of shard i
+        dWqkv[:, mine] = (X.T @ dQKV)[:, local[mine]]
+        dbqkv[mine] = dQKV.sum(axis=0)[local[mine]]
+        dWo[i * hs:(i + 1) * hs, :] = O.T @ dY
+    dX = reduce_partials(parts, None, dY if residual else None)
+    return dict(dX=dX, dWqkv=dWqkv, dbqkv=dbqkv, dWo=dWo, dbo=dY.sum(axis=0),
+                dX_partials=parts, dQKV_shards=dqkv_shards)
+
+
+def layernorm_backward(x, gamma, dy, eps: float = 1e-5) -> tuple:
+    """Gradients of y = gamma * (x - mu) / sqrt(var + eps) + beta per row
+    (population variance) given dy: (dx, dgamma, dbeta). With x_hat the
+    normalised row and g = dy * gamma, the row's dx is
+    (g - mean(g) - x_hat * mean(g * x_hat)) / sqrt(var + eps)."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=1, keepdims=True)
+    rstd = 1.0 / np.sqrt(var + eps)
+    xh = (x - mu) * rstd
+    g = dy * gamma
+    dx = rstd * (g - g.mean(axis=1, keepdims=True) - xh * (g * xh).mean(axis=1, keepdims=True))
+    return dx, (dy * xh).sum(axis=0), dy.sum(axis=0)
+
+
+def transformer_layer_backward(X, p: dict, dY, batch: int, seq: int,
+                               n_heads: int, n_shards: int, eps: float = 1e-5,
+                               causal: bool = True) -> dict:
+    """Gradients of the pre-LN layer Y = h1 + MLP(LN2(h1)),
+    h1 = X + Attn(LN1(X)), by the tensor-parallel route: the MLP block's
+    backward (one reduction, of its input gradient) and the attention
+    block's backward (one reduction) with the LayerNorm backward and the
+    residual paths between them. Returns dX and every parameter gradient
+    (LN gammas and betas included)."""
+    x1 = layernorm(X, p["ln1_g"], p["ln1_b"], eps)
+    h1 = self_attention_sharded(x1, p["Wqkv"], p["bqkv"], p["Wo"], p["bo"], X,
+                                batch, seq, n_heads, n_shards, causal)
+    x2 = layernorm(h1, p["ln2_g"], p["ln2_b"], eps)
+    gm = mlp_backward_sharded(x2, p["A"], p["b1"], p["B"], dY, n_shards, residual=False)
+    dx2 = gm["dX"]
+    dln2, dg2, db2n = layernorm_backward(h1, p["ln2_g"], dx2, eps)
+    dh1 = dY + dln2
+    ga = self_attention_backward_sharded(x1, p["Wqkv"], p["bqkv"], p["Wo"], p["bo"], dh1,
+                                         batch, seq, n_heads, n_shards, causal, residual=False)
+    dln1, dg1, db1n = layernorm_backward(X, p["ln1_g"], ga["dX"], eps)
+    return dict(dX=dh1 + dln1, dh1=dh1,
+                dWqkv=ga["dWqkv"], dbqkv=ga["dbqkv"], dWo=ga["dWo"], dbo=ga["dbo"],
+                dA=gm["dA"], db1=gm["db1"], dB=gm["dB"], db2=gm["db2"],
+                dln1_g=dg1, dln1_b=db1n, dln2_g=dg2, dln2_b=db2n)
+
+
+# --------------------------------------------------------------------------
 # grouped-query attention ([TP-LLM] "Grouped-Query Attention (GQA)
 # Constraints")
 # --------------------------------------------------------------------------

@@ -646,3 +646,123 @@ def test_mlp_backward_sharded_equals_unsharded(n):
     for k in ("dX", "dA", "db1", "dB", "db2"):
         np.testing.assert_allclose(got[k], ref[k], rtol=1e-12, atol=1e-12, err_msg=k)
     assert len(got["dX_partials"]) == n and all(p.shape == (M, h) for p in got["dX_partials"])
+
+
+# ---------------------------------------------------------------- attention and layer backward
+
+def _num_grad(loss, arr, eps=1e-6):
+    """Central differences of loss() with respect to every element of arr."""
+    num = np.zeros_like(arr)
+    for idx in np.ndindex(arr.shape):
+        orig = arr[idx]
+        arr[idx] = orig + eps
+        up = loss()
+        arr[idx] = orig - eps
+        dn = loss()
+        arr[idx] = orig
+        num[idx] = (up - dn) / (2 * eps)
+    return num
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_attention_head_backward_matches_finite_differences(causal):
+    rng = np.random.default_rng(30)
+    T, d = 5, 4
+    Q, K, V = (rng.standard_normal((T, d)) for _ in range(3))
+    dO = rng.standard_normal((T, d))
+    dQ, dK, dV = O.attention_head_backward(Q, K, V, dO, causal)
+    loss = lambda: float(np.sum(O.attention_head(Q, K, V, causal) * dO))  # noqa: E731
+    for name, g, arr in (("dQ", dQ, Q), ("dK", dK, K), ("dV", dV, V)):
+        np.testing.assert_allclose(g, _num_grad(loss, arr), rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_attention_head_backward_closed_forms(causal):
+    """Exact identities of the softmax attention gradient: every softmax row
+    sums to 1, so sum_j dV_j = sum_i dO_i; adding one vector to every key
+    leaves each softmax row unchanged, so sum_j dK_j = 0; the first causal
+    query attends to one key with weight 1, so its dQ row is 0."""
+    rng = np.random.default_rng(31)
+    T, d = 7, 4
+    Q, K, V, dO = (rng.standard_normal((T, d)) for _ in range(4))
+    dQ, dK, dV = O.attention_head_backward(Q, K, V, dO, causal)
+    np.testing.assert_allclose(dV.sum(axis=0), dO.sum(axis=0), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dK.sum(axis=0), np.zeros(d), rtol=0, atol=1e-12)
+    if causal:
+        assert np.all(dQ[0] == 0.0)
+        # the last key is seen by the last query only: dV_last = P[last, last] dO_last
+        S = Q[-1] @ K.T / math.sqrt(d)
+        p_last = math.exp(S[-1] - S.max()) / np.exp(S - S.max()).sum()
+        np.testing.assert_allclose(dV[-1], p_last * dO[-1], rtol=1e-12, atol=1e-14)
+
+
+def test_self_attention_backward_matches_finite_differences():
+    rng = np.random.default_rng(32)
+    b, s, h, nh = 2, 3, 4, 2
+    X = rng.standard_normal((b * s, h))
+    Wqkv, Wo = rng.standard_normal((h, 3 * h)) * .4, rng.standard_normal((h, h)) * .4
+    bqkv, bo = rng.standard_normal(3 * h) * .1, rng.standard_normal(h) * .1
+    dY = rng.standard_normal((b * s, h))
+    g = O.self_attention_backward(X, Wqkv, bqkv, Wo, bo, dY, b, s, nh)
+    loss = lambda: float(np.sum(O.self_attention(X, Wqkv, bqkv, Wo, bo, X, b, s, nh) * dY))  # noqa: E731
+    for name, arr in (("dX", X), ("dWqkv", Wqkv), ("dbqkv", bqkv), ("dWo", Wo), ("dbo", bo)):
+        np.testing.assert_allclose(g[name], _num_grad(loss, arr), rtol=1e-6, atol=1e-8,
+                                   err_msg=name)
+
+
+@pytest.mark.parametrize("n", [1, 2, 4])
+def test_self_attention_backward_sharded_equals_unsharded(n):
+    rng = np.random.default_rng(33)
+    b, s, h, nh = 2, 5, 16, 4
+    X = rng.standard_normal((b * s, h))
+    Wqkv, Wo = rng.standard_normal((h, 3 * h)) * .3, rng.standard_normal((h, h)) * .3
+    bqkv, bo = rng.standard_normal(3 * h) * .1, rng.standard_normal(h) * .1
+    dY = rng.standard_normal((b * s, h))
+    ref = O.self_attention_backward(X, Wqkv, bqkv, Wo, bo, dY, b, s, nh)
+    got = O.self_attention_backward_sharded(X, Wqkv, bqkv, Wo, bo, dY, b, s, nh, n)
+    for k in ("dX", "dWqkv", "dbqkv", "dWo", "dbo"):
+        np.testing.assert_allclose(got[k], ref[k], rtol=1e-12, atol=1e-12, err_msg=k)
+    assert len(got["dX_partials"]) == n
+    # the one reduction: the partials sum to dX - dY
+    np.testing.assert_allclose(sum(got["dX_partials"]), ref["dX"] - dY, rtol=1e-12, atol=1e-12)
+
+
+def test_layernorm_backward_matches_finite_differences_and_identities():
+    rng = np.random.default_rng(34)
+    x = rng.standard_normal((3, 6)) * 2 + 1
+    gamma, beta = rng.standard_normal(6), rng.standard_normal(6)
+    dy = rng.standard_normal((3, 6))
+    dx, dg, db = O.layernorm_backward(x, gamma, dy, 1e-5)
+    loss = lambda: float(np.sum(O.layernorm(x, gamma, beta, 1e-5) * dy))  # noqa: E731
+    np.testing.assert_allclose(dx, _num_grad(loss, x), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dg, _num_grad(loss, gamma), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(db, _num_grad(loss, beta), rtol=1e-6, atol=1e-8)
+    # LN is invariant to shifting a row and (with eps = 0) to scaling it, so
+    # each row of dx is orthogonal to the ones vector and to the row itself
+    dx0, _, _ = O.layernorm_backward(x, gamma, dy, 0.0)
+    np.testing.assert_allclose(dx0.sum(axis=1), 0.0, atol=1e-12)
+    np.testing.assert_allclose((dx0 * x).sum(axis=1), 0.0, atol=1e-11)
+
+
+def test_transformer_layer_backward_matches_finite_differences():
+    """The tensor-parallel layer backward (N = 2) against central differences
+    of <Y, dY> through the unsharded layer definition."""
+    rng = np.random.default_rng(35)
+    b, s, h, nh, F, n = 1, 3, 4, 2, 8, 2
+    X = rng.standard_normal((b * s, h))
+    p = dict(Wqkv=rng.standard_normal((h, 3 * h)) * .4, bqkv=rng.standard_normal(3 * h) * .1,
+             Wo=rng.standard_normal((h, h)) * .4, bo=rng.standard_normal(h) * .1,
+             A=rng.standard_normal((h, F)) * .4, b1=rng.standard_normal(F) * .1,
+             B=rng.standard_normal((F, h)) * .4, b2=rng.standard_normal(h) * .1,
+             ln1_g=1 + rng.standard_normal(h) * .1, ln1_b=rng.standard_normal(h) * .1,
+             ln2_g=1 + rng.standard_normal(h) * .1, ln2_b=rng.standard_normal(h) * .1)
+    dY = rng.standard_normal((b * s, h))
+    g = O.transformer_layer_backward(X, p, dY, b, s, nh, n)
+    loss = lambda: float(np.sum(O.transformer_layer(X, p, b, s, nh) * dY))  # noqa: E731
+    np.testing.assert_allclose(g["dX"], _num_grad(loss, X), rtol=1e-5, atol=1e-7, err_msg="dX")
+    for key, name in (("Wqkv", "dWqkv"), ("bqkv", "dbqkv"), ("Wo", "dWo"), ("bo", "dbo"),
+                      ("A", "dA"), ("b1", "db1"), ("B", "dB"), ("b2", "db2"),
+                      ("ln1_g", "dln1_g"), ("ln1_b", "dln1_b"), ("ln2_g", "dln2_g"),
+                      ("ln2_b", "dln2_b")):
+        np.testing.assert_allclose(g[name], _num_grad(loss, p[key]), rtol=1e-5, atol=1e-7,
+                                   err_msg=name)
