@@ -96,7 +96,8 @@ typedef enum {
 } tp_act;
 
 typedef enum {
-    TP_WS_MLP = 0, TP_WS_ATTN = 1, TP_WS_LAYER = 2, TP_WS_LAYER_SP = 3, TP_WS_MLP_BWD = 4
+    TP_WS_MLP = 0, TP_WS_ATTN = 1, TP_WS_LAYER = 2, TP_WS_LAYER_SP = 3, TP_WS_MLP_BWD = 4,
+    TP_WS_ATTN_CORE_BWD = 5, TP_WS_ATTN_BWD = 6, TP_WS_LAYER_BWD = 7
 } tp_ws_kind;
 
 /* Weights of one pre-LN layer, all device pointers in the packed shard
@@ -256,6 +257,58 @@ tp_status tp_mlp_backward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn,
                           float* db1, float* dB_shards, float* db2,
                           void* stream);
 
+/* tp_attention_lse - tp_attention that also writes what its backward needs:
+ * for every shard i, local head k and token row r (of batch*seq = M),
+ * lse[(i*n_heads/N + k)*(M + 128) + r] = log2 sum_s exp(q_r . k_s / sqrt(d))
+ * over the keys s the query sees (the base-2 log-sum-exp of its scaled
+ * scores). lse holds n_heads*(M + 128) floats; the last 128 of each head's
+ * row are not written. Other arguments as tp_attention. */
+tp_status tp_attention_lse(const uint16_t* QKV_shards, int64_t batch,
+                           int64_t seq, int64_t h, int64_t n_heads, int causal,
+                           int n_shards, uint16_t* O_shards, float* lse,
+                           void* stream);
+
+/* tp_attention_backward - gradients of the local attention of every shard's
+ * heads (the backward of tp_attention, local to each shard like the forward:
+ * [TP-LLM] "Local Self-Attention Computation"). With P = softmax(Q K^T /
+ * sqrt d) rebuilt from lse: dV = P^T dO, dP = dO V^T,
+ * dS = P * (dP - rowsum(dO * O)), dQ = dS K / sqrt d, dK = dS^T Q / sqrt d.
+ * Inputs: QKV_shards [N][M][3h/N], O_shards and dO_shards [N][M][h/N] (bf16)
+ * and lse from tp_attention_lse on the same QKV. Output: dQKV_shards
+ * [N][M][3h/N] bf16, packed like QKV ([dQ_i | dK_i | dV_i]). Multi-head
+ * attention only (no GQA); head_dim must be 128. dQ is accumulated in fp32
+ * with atomic additions, so its last bits can differ between runs.
+ * ws >= tp_workspace_bytes(TP_WS_ATTN_CORE_BWD, M, h, 0, N). */
+tp_status tp_attention_backward(const uint16_t* QKV_shards,
+                                const uint16_t* O_shards,
+                                const uint16_t* dO_shards, const float* lse,
+                                int64_t batch, int64_t seq, int64_t h,
+                                int64_t n_heads, int causal, int n_shards,
+                                void* ws, size_t ws_bytes,
+                                uint16_t* dQKV_shards, void* stream);
+
+/* tp_attn_backward - gradients of the attention block
+ * Y = concat_heads(attention) W_O + b_O (+ X) by the tensor-parallel route:
+ * dY reaches every shard whole (the row-parallel W_O's backward needs no
+ * exchange); shard i recomputes QKV_i, O_i and lse, forms dO_i = dY W_O,i^T,
+ * its heads' attention backward, its weight gradients locally and a
+ * full-size partial dX_i = dQKV_i W_QKV,i^T; dX = sum_i dX_i (+ dY when
+ * residual) is the block's one reduction ([TP-LLM] "Communication Budget and
+ * Scaling Limits": two all-reduces per layer in the backward pass, one per
+ * block). Inputs as tp_attn_forward plus dY [M][h] (bf16). Outputs: dX [M][h]
+ * bf16; dWqkv_shards [N][3h/N][h], dbqkv_shards [N][3h/N], dWo_shards
+ * [N][h][h/N] fp32 in the packed layouts of the weights; dbo [h] fp32.
+ * ws >= tp_workspace_bytes(TP_WS_ATTN_BWD, M, h, 0, N). */
+tp_status tp_attn_backward(const uint16_t* X, int64_t batch, int64_t seq,
+                           int64_t h, int64_t n_heads, int causal, int n_shards,
+                           const uint16_t* Wqkv_shards,
+                           const uint16_t* bqkv_shards,
+                           const uint16_t* Wo_shards, const uint16_t* dY,
+                           int residual, void* ws, size_t ws_bytes,
+                           uint16_t* dX, float* dWqkv_shards,
+                           float* dbqkv_shards, float* dWo_shards, float* dbo,
+                           void* stream);
+
 /* tp_attn_forward - Y = concat_heads(attention) W_O + b_O + residual by the
  * tensor-parallel route: QKV column-parallel by whole heads (+ bias), local
  * attention per shard, W_O row-parallel into N partials, one sum
@@ -388,9 +441,11 @@ tp_status tp_mlp_forward_noalloc(const uint16_t* X, int64_t B, int64_t h,
                                  void* stream);
 
 /* Workspace bytes for tp_mlp_forward (kind TP_WS_MLP), tp_attn_forward
- * (TP_WS_ATTN, ffn ignored), tp_layer_forward (TP_WS_LAYER) or
- * tp_layer_forward_sp (TP_WS_LAYER_SP) or tp_mlp_backward (TP_WS_MLP_BWD). tokens =
- * batch * seq. Returns 0 for invalid arguments. */
+ * (TP_WS_ATTN, ffn ignored), tp_layer_forward (TP_WS_LAYER),
+ * tp_layer_forward_sp (TP_WS_LAYER_SP), tp_mlp_backward (TP_WS_MLP_BWD),
+ * tp_attention_backward (TP_WS_ATTN_CORE_BWD, ffn ignored), tp_attn_backward
+ * (TP_WS_ATTN_BWD, ffn ignored) or tp_layer_backward (TP_WS_LAYER_BWD).
+ * tokens = batch * seq. Returns 0 for invalid arguments. */
 size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn,
                           int n_shards);
 

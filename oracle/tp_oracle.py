@@ -462,6 +462,20 @@ def attention_head_backward(Q, K, V, dO, causal: bool) -> tuple:
     return dS @ K / math.sqrt(d), dS.T @ Q / math.sqrt(d), dV
 
 
+def attention_logsumexp(Q, K, causal: bool) -> np.ndarray:
+    """Per query row: ln sum_s exp(q . k_s / sqrt d) over the keys the query
+    sees (the normaliser of its softmax row), for one head of one
+    sequence."""
+    d = Q.shape[1]
+    S = (Q @ K.T) / math.sqrt(d)
+    if causal:
+        t = np.arange(Q.shape[0])[:, None]
+        s = np.arange(K.shape[0])[None, :]
+        S = np.where(s <= t, S, -np.inf)
+    m = S.max(axis=1, keepdims=True)
+    return (m + np.log(np.exp(S - m).sum(axis=1, keepdims=True)))[:, 0]
+
+
 def attention_heads_backward(Q, K, V, dO, batch: int, seq: int, n_heads: int,
                              causal: bool) -> tuple:
     """attention_head_backward for every (sequence, head) pair; head k is

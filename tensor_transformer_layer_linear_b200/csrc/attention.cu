@@ -81,6 +81,8 @@ struct AttnParams {
   int group;  // local query heads per local kv head
   long long M;  // tokens per shard
   float scale_log2;
+  float* lse;  // optional: base-2 log-sum-exp of each query's scaled scores
+  long long lse_stride;  // per (shard, head): tokens per shard + 128
   unsigned* err;
 };
 
@@ -339,6 +341,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     } else if (mbar_wait(bar(B_ODONE), 0, abort_flag)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float base_final = (m_used == -INFINITY) ? 0.f : m_used * sl2;
       uint16_t* orow = O + (static_cast<int64_t>(g) * p.M + row_base + t) * p.q_w + head * FA_D;
 #pragma unroll 1
       for (int c = 0; c < FA_D / 32; ++c) {
@@ -357,6 +360,10 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
           }
         }
       }
+      // P = exp2(s sl2 - base) / l = exp2(s sl2 - (base + log2 l))
+      if (p.lse != nullptr && t < p.seq)
+        p.lse[(static_cast<int64_t>(g) * p.hps + head) * p.lse_stride + row_base + t] =
+            base_final + log2f(l);
     } else {
       if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
       *abort_flag = 1;
@@ -388,7 +395,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 attn_map_encoder() {
 }
 
 int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, int64_t kv_local,
-                     int n_shards, int causal, void* O, cudaStream_t s, unsigned* err) {
+                     int n_shards, int causal, void* O, cudaStream_t s, unsigned* err,
+                     float* lse) {
   const int hps = static_cast<int>(n_q / n_shards);
   const int64_t q_w = hps * FA_D, kv_w = kv_local * FA_D;
   const int64_t ld = q_w + 2 * kv_w;  // QKV row width per shard
@@ -416,6 +424,8 @@ int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, i
   p.nq = static_cast<int>((seq + FA_BM * FA_TILES - 1) / (FA_BM * FA_TILES));
   p.M = M;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(FA_D));
+  p.lse = lse;
+  p.lse_stride = M + 128;
   p.err = err;
   // The setmaxnreg split assumes FA_REGS_LAUNCH registers per thread at
   // launch; with fewer, the softmax warpgroups' increase could never be

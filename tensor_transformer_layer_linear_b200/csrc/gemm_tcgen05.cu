@@ -596,6 +596,10 @@ int launch_gemm(const GemmProblem& p, cudaStream_t s, unsigned* err, int num_sms
     return p.M > BM ? launch_gemm_t<256, EPI_F32, 2, true, true>(p, s, err, num_sms)
                     : launch_gemm_t<256, EPI_F32, 1, true, true>(p, s, err, num_sms);
   }
+  if (p.b_mn && !p.out_f32) {  // dO = dY W_O,i^T in bf16: A K-major, B MN-major
+    return p.M > BM ? launch_gemm_t<256, EPI_BF16, 2, false, true>(p, s, err, num_sms)
+                    : launch_gemm_t<256, EPI_BF16, 1, false, true>(p, s, err, num_sms);
+  }
   if (p.b_mn) {
     return p.M > BM ? launch_gemm_t<256, EPI_F32, 2, false, true>(p, s, err, num_sms)
                     : launch_gemm_t<256, EPI_F32, 1, false, true>(p, s, err, num_sms);

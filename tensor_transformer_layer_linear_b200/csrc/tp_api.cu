@@ -135,6 +135,8 @@ const char* tp_kernel_name(int kid) {
     case tpk::KID_GEMM_BACKWARD: return "gemm_backward";
     case tpk::KID_ELEMENTWISE: return "gelu_elementwise";
     case tpk::KID_COLSUM: return "column_sum";
+    case tpk::KID_ATTENTION_BWD: return "attention_backward";
+    case tpk::KID_LAYERNORM_BWD: return "reduce_partials_layernorm_backward";
     default: return "unknown";
   }
 }
@@ -427,6 +429,17 @@ size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int 
     // GeLU'(Z), H, dZ [N][M][F/N] bf16; dX partials [N][M][h] fp32; column-sum slabs
     return 3 * round256(M * static_cast<size_t>(ffn) * 2) + partials +
            round256(static_cast<size_t>(kColsumSlabs) * (static_cast<size_t>(ffn) + H) * 4);
+  }
+  if (kind == TP_WS_ATTN_CORE_BWD || kind == TP_WS_ATTN_BWD) {
+    // D [n_heads][M + 128] and the dQ accumulator [n_heads][128][M + 128]
+    // fp32 (head_dim 128: n_heads = h / 128)
+    const size_t rows = M + 128;
+    const size_t core = round256(H / 128 * rows * 4) + round256(H * rows * 4);
+    if (kind == TP_WS_ATTN_CORE_BWD) return core;
+    // + QKV, O, dO, dQKV (bf16), lse, the dX partials and column-sum slabs
+    return core + 2 * round256(M * 3 * H * 2) + 2 * round256(M * H * 2) +
+           round256(H / 128 * rows * 4) + partials +
+           round256(static_cast<size_t>(kColsumSlabs) * 4 * H * 4);
   }
   if (kind == TP_WS_LAYER || kind == TP_WS_LAYER_SP) {
     if (ffn <= 0) return 0;
@@ -816,6 +829,140 @@ tp_status tp_mlp_backward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, 
   if (tpk::launch_colsum(dZ, n_shards, M, fs, slabs, kColsumSlabs, db1, s, d.num_sms) != 0)
     return TP_ERR_CUDA;
   if (tpk::launch_colsum(dY, 1, M, H, slabs, kColsumSlabs, db2, s, d.num_sms) != 0)
+    return TP_ERR_CUDA;
+  return TP_OK;
+}
+
+tp_status tp_attention_lse(const uint16_t* QKV_shards, int64_t batch, int64_t seq, int64_t h,
+                           int64_t n_heads, int causal, int n_shards, uint16_t* O_shards,
+                           float* lse, void* stream) {
+  if (QKV_shards == nullptr || O_shards == nullptr || lse == nullptr) return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || n_heads <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (h % n_heads || n_heads % n_shards) return TP_ERR_SHAPE;
+  if (h / n_heads != 128) return TP_ERR_UNSUPPORTED;
+  if (batch * seq > kIntMax || seq > kIntMax) return TP_ERR_SHAPE;
+  if (static_cast<int64_t>(n_shards) * batch * (n_heads / n_shards) > 65535) return TP_ERR_SHAPE;
+  if (!al16(QKV_shards) || !al16(O_shards) || !al16(lse)) return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
+  const int rc = tpk::launch_attention(QKV_shards, batch, seq, n_heads, n_heads / n_shards,
+                                       n_shards, causal ? 1 : 0, O_shards, as_stream(stream),
+                                       d.err, lse);
+  return rc == 0 ? TP_OK : (rc == 3 ? TP_ERR_UNSUPPORTED : TP_ERR_CUDA);
+}
+
+tp_status tp_attention_backward(const uint16_t* QKV_shards, const uint16_t* O_shards,
+                                const uint16_t* dO_shards, const float* lse, int64_t batch,
+                                int64_t seq, int64_t h, int64_t n_heads, int causal,
+                                int n_shards, void* ws, size_t ws_bytes, uint16_t* dQKV_shards,
+                                void* stream) {
+  if (QKV_shards == nullptr || O_shards == nullptr || dO_shards == nullptr || lse == nullptr ||
+      dQKV_shards == nullptr || ws == nullptr)
+    return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || n_heads <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (h % n_heads || n_heads % n_shards) return TP_ERR_SHAPE;
+  if (h / n_heads != 128) return TP_ERR_UNSUPPORTED;
+  if (batch * seq > kIntMax || seq > kIntMax) return TP_ERR_SHAPE;
+  if (static_cast<int64_t>(n_shards) * batch * (n_heads / n_shards) > 0x7FFFFFFF) return TP_ERR_SHAPE;
+  const int64_t M = batch * seq;
+  const size_t need = tp_workspace_bytes(TP_WS_ATTN_CORE_BWD, M, h, 0, n_shards);
+  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  if (!al16(QKV_shards) || !al16(O_shards) || !al16(dO_shards) || !al16(lse) ||
+      !al16(dQKV_shards) || !al16(ws))
+    return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  const size_t rows = static_cast<size_t>(M) + 128;
+  float* dsum = static_cast<float*>(ws);
+  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                           round256(static_cast<size_t>(h) / 128 * rows * 4));
+  TraceScope ts(tpk::KID_ATTENTION_BWD, as_stream(stream));
+  const int rc = tpk::launch_attention_bwd(QKV_shards, O_shards, dO_shards, lse, batch, seq,
+                                           n_heads, n_shards, causal ? 1 : 0, dQKV_shards, dsum,
+                                           dq_acc, as_stream(stream), d.err, d.num_sms);
+  return rc == 0 ? TP_OK : TP_ERR_CUDA;
+}
+
+tp_status tp_attn_backward(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
+                           int64_t n_heads, int causal, int n_shards, const uint16_t* Wqkv_shards,
+                           const uint16_t* bqkv_shards, const uint16_t* Wo_shards,
+                           const uint16_t* dY, int residual, void* ws, size_t ws_bytes,
+                           uint16_t* dX, float* dWqkv_shards, float* dbqkv_shards,
+                           float* dWo_shards, float* dbo, void* stream) {
+  if (X == nullptr || Wqkv_shards == nullptr || Wo_shards == nullptr || dY == nullptr ||
+      dX == nullptr || dWqkv_shards == nullptr || dbqkv_shards == nullptr ||
+      dWo_shards == nullptr || dbo == nullptr || ws == nullptr)
+    return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || n_heads <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
+  if (h % n_heads || n_heads % n_shards) return TP_ERR_SHAPE;
+  if (h / n_heads != 128) return TP_ERR_UNSUPPORTED;
+  if (batch * seq > kIntMax || seq > kIntMax) return TP_ERR_SHAPE;
+  const int64_t M64 = batch * seq;
+  const size_t need = tp_workspace_bytes(TP_WS_ATTN_BWD, M64, h, 0, n_shards);
+  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  if (!al16(ws) || !al16(X) || !al16(Wqkv_shards) || !al16(Wo_shards) || !al16(dY) ||
+      !al16(dX) || !al16(dWqkv_shards) || !al16(dbqkv_shards) || !al16(dWo_shards) ||
+      !al16(dbo) || (bqkv_shards && !al16(bqkv_shards)))
+    return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  const int M = static_cast<int>(M64), H = static_cast<int>(h);
+  const int hs = H / n_shards;
+  const size_t rows = static_cast<size_t>(M) + 128;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  void* core = p; p += tp_workspace_bytes(TP_WS_ATTN_CORE_BWD, M64, h, 0, n_shards);
+  uint16_t* qkv = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * 3 * H * 2);
+  uint16_t* dqkv = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * 3 * H * 2);
+  uint16_t* o = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * H * 2);
+  uint16_t* dO = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * H * 2);
+  float* lse = reinterpret_cast<float*>(p); p += round256(static_cast<size_t>(H) / 128 * rows * 4);
+  float* part = reinterpret_cast<float*>(p);
+  p += round256(static_cast<size_t>(n_shards) * M * H * 4);
+  float* slabs = reinterpret_cast<float*>(p);
+  cudaStream_t s = as_stream(stream);
+  auto gemm = [&](const void* A, bool a_b, bool a_mn, const void* Bop, bool b_b, bool b_mn,
+                  void* D, int m, int nc, int k, bool f32) {
+    tpk::GemmProblem g;
+    g.A = A; g.B = Bop; g.D = D; g.bias = nullptr;
+    g.M = m; g.Nc = nc; g.K = k; g.G = n_shards;
+    g.a_batched = a_b; g.b_batched = b_b; g.a_mn = a_mn; g.b_mn = b_mn;
+    g.out_f32 = f32; g.act = 0;
+    TraceScope ts(tpk::KID_GEMM_BACKWARD, s);
+    return tpk::launch_gemm(g, s, d.err, d.num_sms) == 0 ? TP_OK : TP_ERR_CUDA;
+  };
+  // recompute the forward: QKV_i = X W_QKV,i + b_i, O_i and the lse
+  st = tp_column_linear(X, M64, h, Wqkv_shards, bqkv_shards, 3 * h, n_shards, TP_ACT_NONE, qkv,
+                        stream);
+  if (st != TP_OK) return st;
+  st = tp_attention_lse(qkv, batch, seq, h, n_heads, causal, n_shards, o, lse, stream);
+  if (st != TP_OK) return st;
+  // dO_i = dY W_O,i^T; Wo_shards[i] = W_O,i^T is the MN-major operand
+  st = gemm(dY, false, false, Wo_shards, true, true, dO, M, hs, H, false);
+  if (st != TP_OK) return st;
+  st = tp_attention_backward(qkv, o, dO, lse, batch, seq, h, n_heads, causal, n_shards, core,
+                             tp_workspace_bytes(TP_WS_ATTN_CORE_BWD, M64, h, 0, n_shards), dqkv,
+                             stream);
+  if (st != TP_OK) return st;
+  // dX partials: dQKV_i W_QKV,i^T; Wqkv_shards[i] = W_QKV,i^T is the MN-major operand
+  st = gemm(dqkv, true, false, Wqkv_shards, true, true, part, M, H, 3 * hs, true);
+  if (st != TP_OK) return st;
+  // the one reduction of the block's backward: dX = sum_i dX_i (+ dY)
+  st = tp_reduce_partials(part, n_shards, M64, h, nullptr, residual ? dY : nullptr, dX, stream);
+  if (st != TP_OK) return st;
+  // dW_QKV,i^T = dQKV_i^T X (packed like Wqkv_shards), dW_O,i^T = dY^T O_i (like Wo_shards)
+  st = gemm(dqkv, true, true, X, false, true, dWqkv_shards, 3 * hs, H, M, true);
+  if (st != TP_OK) return st;
+  st = gemm(dY, false, true, o, true, true, dWo_shards, H, hs, M, true);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_COLSUM, s);
+  if (tpk::launch_colsum(dqkv, n_shards, M, 3 * hs, slabs, kColsumSlabs, dbqkv_shards, s,
+                         d.num_sms) != 0)
+    return TP_ERR_CUDA;
+  if (tpk::launch_colsum(dY, 1, M, H, slabs, kColsumSlabs, dbo, s, d.num_sms) != 0)
     return TP_ERR_CUDA;
   return TP_OK;
 }

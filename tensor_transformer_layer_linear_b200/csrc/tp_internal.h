@@ -19,7 +19,9 @@ enum KernelId {
   KID_GEMM_BACKWARD = 8,
   KID_ELEMENTWISE = 9,
   KID_COLSUM = 10,
-  KID_COUNT = 11
+  KID_ATTENTION_BWD = 11,
+  KID_LAYERNORM_BWD = 12,
+  KID_COUNT = 13
 };
 
 // One batched GEMM over G shards: D[g] (M x Nc) = A[g] (M x K) . B[g]^T with
@@ -31,8 +33,8 @@ enum KernelId {
 // (B [G_B][K][Nc]); b_batched = false shares B across the batch; act 3 is the
 // GeLU backward epilogue D = bf16(acc * aux), aux = GeLU'(Z) [G][M][Nc] bf16;
 // act 4 is the forward recompute D = bf16(GeLU(acc + bias)) that also writes
-// aux_out = bf16(GeLU'(acc + bias)) [G][M][Nc]. MN-major products write fp32
-// (act 0, out_f32).
+// aux_out = bf16(GeLU'(acc + bias)) [G][M][Nc]. Products with an MN-major
+// A write fp32; with only B MN-major, fp32 or bf16 (act 0, no bias).
 struct GemmProblem {
   const void* A;
   const void* B;
@@ -82,9 +84,21 @@ int launch_rows_sum_ln(const float* P, int n_shards, int64_t rows, int64_t h, co
 // of QKV are [Q (n_q/N heads) | K (kv_local heads) | V (kv_local heads)];
 // local query head k uses local kv head k / (n_q/N / kv_local). Returns 3 if
 // the kernel was built with fewer launch registers than its warpgroup
-// register split needs (it is then not launched).
+// register split needs (it is then not launched). With lse != nullptr the
+// base-2 log-sum-exp of every query's scaled scores is written to
+// lse[(shard * (n_q/N) + k) * (M + 128) + token], M = batch * seq.
 int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, int64_t kv_local,
-                     int n_shards, int causal, void* O, cudaStream_t s, unsigned* err);
+                     int n_shards, int causal, void* O, cudaStream_t s, unsigned* err,
+                     float* lse = nullptr);
+
+// Attention backward of every shard's heads (n_kv = n_q, head_dim 128):
+// dQKV [N][M][3 hs] (packed like QKV) from QKV, O, dO [N][M][hs] and the
+// forward's lse. dsum [n_heads][M + 128] fp32 and dq_acc
+// [n_heads][128][M + 128] fp32 are scratch.
+int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const float* lse,
+                         int64_t batch, int64_t seq, int64_t n_heads, int n_shards, int causal,
+                         void* dQKV, float* dsum, float* dq_acc, cudaStream_t s, unsigned* err,
+                         int num_sms);
 
 // out[i][c][r] = W[row(i, r)][col(i, c)] for the split kinds (kind 4: GQA
 // QKV with n_q query and n_kv key/value heads of head_dim).

@@ -32,6 +32,7 @@ TP_ERR_WORKSPACE, TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_TIMEOUT = 4, 5, 6, 7
 TP_SPLIT_COLUMN, TP_SPLIT_ROW, TP_SPLIT_QKV_HEADS, TP_SPLIT_GATE_UP = 0, 1, 2, 3
 TP_ACT_NONE, TP_ACT_GELU_ERF, TP_ACT_SWIGLU = 0, 1, 2
 TP_WS_MLP, TP_WS_ATTN, TP_WS_LAYER, TP_WS_LAYER_SP, TP_WS_MLP_BWD = 0, 1, 2, 3, 4
+TP_WS_ATTN_CORE_BWD, TP_WS_ATTN_BWD, TP_WS_LAYER_BWD = 5, 6, 7
 
 _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
@@ -72,6 +73,11 @@ _SIGS = {
                                    _vp, _vp, _vp, _sz, _vp, _vp]),
     "tp_mlp_backward": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _sz,
                                _vp, _vp, _vp, _vp, _vp, _vp]),
+    "tp_attention_lse": (_i32, [_vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
+    "tp_attention_backward": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32,
+                                     _vp, _sz, _vp, _vp]),
+    "tp_attn_backward": (_i32, [_vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp,
+                                _i32, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _vp]),
     "tp_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "tp_get_last_error": (_i32, [_vp]),
     "tp_status_string": (ctypes.c_char_p, [_i32]),
@@ -278,6 +284,30 @@ def tp_mlp_backward(X, B, h, ffn, n_shards, A_shards, b1_shards, B_shards, dY, r
                                _p(B_shards), _p(dY), int(bool(residual)), _p(ws), ws_bytes, _p(dX),
                                _p(dA_shards), _p(db1), _p(dB_shards), _p(db2), _s(stream)),
            "tp_mlp_backward")
+
+
+def tp_attention_lse(QKV_shards, batch, seq, h, n_heads, causal, n_shards, O_shards, lse,
+                     stream=None):
+    _check(lib.tp_attention_lse(_p(QKV_shards), batch, seq, h, n_heads, int(bool(causal)),
+                                n_shards, _p(O_shards), _p(lse), _s(stream)), "tp_attention_lse")
+
+
+def tp_attention_backward(QKV_shards, O_shards, dO_shards, lse, batch, seq, h, n_heads, causal,
+                          n_shards, ws, ws_bytes, dQKV_shards, stream=None):
+    _check(lib.tp_attention_backward(_p(QKV_shards), _p(O_shards), _p(dO_shards), _p(lse), batch,
+                                     seq, h, n_heads, int(bool(causal)), n_shards, _p(ws),
+                                     ws_bytes, _p(dQKV_shards), _s(stream)),
+           "tp_attention_backward")
+
+
+def tp_attn_backward(X, batch, seq, h, n_heads, causal, n_shards, Wqkv_shards, bqkv_shards,
+                     Wo_shards, dY, residual, ws, ws_bytes, dX, dWqkv_shards, dbqkv_shards,
+                     dWo_shards, dbo, stream=None):
+    _check(lib.tp_attn_backward(_p(X), batch, seq, h, n_heads, int(bool(causal)), n_shards,
+                                _p(Wqkv_shards), _p(bqkv_shards), _p(Wo_shards), _p(dY),
+                                int(bool(residual)), _p(ws), ws_bytes, _p(dX), _p(dWqkv_shards),
+                                _p(dbqkv_shards), _p(dWo_shards), _p(dbo), _s(stream)),
+           "tp_attn_backward")
 
 
 def tp_get_last_error(stream=None) -> int:

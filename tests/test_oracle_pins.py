@@ -766,3 +766,18 @@ def test_transformer_layer_backward_matches_finite_differences():
                       ("ln2_b", "dln2_b")):
         np.testing.assert_allclose(g[name], _num_grad(loss, p[key]), rtol=1e-5, atol=1e-7,
                                    err_msg=name)
+
+
+def test_attention_logsumexp_closed_forms():
+    """Q = 0 makes every score 0, so causal row t sums t + 1 ones (ln(t + 1))
+    and a full row sums T ones; one key scored log 3 above the other gives
+    ln(e^a + 3 e^a)."""
+    T, d = 6, 4
+    K = np.random.default_rng(36).standard_normal((T, d))
+    np.testing.assert_allclose(O.attention_logsumexp(np.zeros((T, d)), K, True),
+                               np.log(np.arange(1, T + 1)), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(O.attention_logsumexp(np.zeros((T, d)), K, False),
+                               np.full(T, math.log(T)), rtol=0, atol=1e-15)
+    q = np.array([[2.0, 0.0]])                     # d = 2: scores k . q / sqrt 2
+    k = np.array([[0.0, 0.0], [math.log(3) * math.sqrt(2) / 2, 0.0]])
+    assert O.attention_logsumexp(q, k, False)[0] == pytest.approx(math.log(4.0), abs=1e-14)
