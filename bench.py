@@ -94,12 +94,25 @@ def work(cfg: dict) -> dict:
         fl["attention"] += 4.0 * cfg["seq"] ** 2 * d * cfg["n_heads"] * cfg["batch"] / (
             2 if cfg.get("causal", True) else 1)
         fl["gemm_row_parallel"] += 2.0 * M * h * h
-    if kind == "mlp" and cfg.get("backward"):
-        # algorithmic backward: dH, dX, dA, dB (the recomputed forward GEMM is extra)
-        F = cfg["ffn"]
-        fl = {"gemm_backward": 8.0 * M * h * F, "gemm_column_parallel": 0.0,
+    if cfg.get("backward"):
+        # algorithmic backward work (recomputed forward products are extra):
+        # MLP dH, dX, dA, dB; attention block dO, dX, dW_QKV, dW_O and the
+        # head gradients dV, dP, dK, dQ (twice the forward attention)
+        F = cfg.get("ffn", 0)
+        gb, ab = 0.0, 0.0
+        if kind in ("mlp", "layer"):
+            gb += 8.0 * M * h * F
+        if kind in ("attn", "layer"):
+            gb += 16.0 * M * h * h
+            ab = 2.0 * fl["attention"]
+        fl = {"gemm_backward": gb, "attention_backward": ab, "gemm_column_parallel": 0.0,
               "gemm_row_parallel": 0.0, "attention": 0.0}
-        by["reduce_partials"] = n * M * h * 4 + 2 * M * h * 2
+        if kind == "layer":
+            by["reduce_partials_layernorm_backward"] = n * M * h * 4 + 3 * M * h * 2 + h * 2
+        else:
+            res = M * h * 2 if cfg.get("residual") else 0
+            by["reduce_partials"] = n * M * h * 4 + res + M * h * 2
+        return dict(flops=fl, bytes=by, total_flops=sum(fl.values()))
     if kind == "swiglu":
         F = cfg["ffn"]
         fl["gemm_column_parallel"] += 2.0 * M * h * 2 * F   # gate and up
@@ -190,7 +203,21 @@ def oracle_sample(cfg: dict, inp: dict, tokens: int):
     f64 = synth.bf16_bits_to_f64
     x = f64(inp["X"][:T])
     t0 = time.perf_counter()
-    if cfg["kind"] == "layer":
+    if cfg.get("backward"):
+        dY = np.random.default_rng(1).standard_normal(x.shape)
+        if cfg["kind"] == "layer":
+            p = {k: f64(v) for k, v in inp.items() if k != "X"}
+            O.transformer_layer_backward(x, p, dY, 1, T, cfg["n_heads"], cfg["n_shards"],
+                                         cfg.get("ln_eps", 1e-5))
+        elif cfg["kind"] == "attn":
+            O.self_attention_backward_sharded(x, f64(inp["Wqkv"]), f64(inp["bqkv"]),
+                                              f64(inp["Wo"]), f64(inp["bo"]), dY, 1, T,
+                                              cfg["n_heads"], cfg["n_shards"],
+                                              cfg.get("causal", True), bool(cfg.get("residual")))
+        else:
+            O.mlp_backward_sharded(x, f64(inp["A"]), f64(inp["b1"]), f64(inp["B"]), dY,
+                                   cfg["n_shards"], bool(cfg.get("residual")))
+    elif cfg["kind"] == "layer":
         p = {k: f64(v) for k, v in inp.items() if k != "X"}
         O.transformer_layer(x, p, 1, T, cfg["n_heads"], cfg.get("ln_eps", 1e-5))
     elif cfg["kind"] == "attn_gqa":
@@ -314,26 +341,52 @@ class Model:
         torch.cuda.synchronize()
 
     def setup_backward(self):
-        """Gradient buffers for the MLP backward step (dY drawn once)."""
-        torch, cfg = self.torch, self.cfg
-        M, h, F, n = self.M, cfg["h"], cfg["ffn"], cfg["n_shards"]
+        """Gradient buffers for the backward step (dY drawn once)."""
+        torch, tp, cfg = self.torch, self.tp, self.cfg
+        M, h, n, kind = self.M, cfg["h"], cfg["n_shards"], cfg["kind"]
+        F = cfg.get("ffn", 0)
         g = torch.Generator(device="cuda").manual_seed(1)
         self.dY = (torch.randn((M, h), device="cuda", generator=g)).to(torch.bfloat16).view(torch.int16)
         self.dX = torch.empty((M, h), dtype=torch.int16, device="cuda")
-        self.dA = torch.empty(h * F, dtype=torch.float32, device="cuda")
-        self.dB = torch.empty(h * F, dtype=torch.float32, device="cuda")
-        self.db1 = torch.empty(F, dtype=torch.float32, device="cuda")
-        self.db2 = torch.empty(h, dtype=torch.float32, device="cuda")
-        self.ws_bwd_bytes = self.tp.tp_workspace_bytes(self.tp.TP_WS_MLP_BWD, M, h, F, n)
+
+        def f32(k):
+            return torch.empty(k, dtype=torch.float32, device="cuda")
+        if kind == "mlp":
+            self.dA, self.dB, self.db1, self.db2 = f32(h * F), f32(h * F), f32(F), f32(h)
+            wsk = tp.TP_WS_MLP_BWD
+        elif kind == "attn":
+            self.dWqkv, self.dbqkv, self.dWo, self.dbo = f32(3 * h * h), f32(3 * h), f32(h * h), f32(h)
+            wsk = tp.TP_WS_ATTN_BWD
+        else:
+            sizes = dict(ln1_gamma=h, ln1_beta=h, Wqkv_shards=3 * h * h, bqkv_shards=3 * h,
+                         Wo_shards=h * h, bo=h, ln2_gamma=h, ln2_beta=h, A_shards=h * F,
+                         b1_shards=F, B_shards=F * h, b2=h)
+            self.grad_keep = {k: f32(v) for k, v in sizes.items()}
+            self.grads = tp.make_layer_grads(**self.grad_keep)
+            wsk = tp.TP_WS_LAYER_BWD
+        self.ws_bwd_bytes = tp.tp_workspace_bytes(wsk, M, h, F, n)
         self.ws_bwd = torch.empty(self.ws_bwd_bytes, dtype=torch.uint8, device="cuda")
 
     def step(self, X=None, Y=None):
         tp, cfg = self.tp, self.cfg
         if cfg.get("backward"):
             X = self.X if X is None else X
-            tp.tp_mlp_backward(X, self.M, cfg["h"], cfg["ffn"], cfg["n_shards"], self.A, self.b1,
-                               self.B, self.dY, cfg.get("residual", False), self.ws_bwd,
-                               self.ws_bwd_bytes, self.dX, self.dA, self.db1, self.dB, self.db2)
+            dX = self.dX if Y is None else Y
+            n, h, kind = cfg["n_shards"], cfg["h"], cfg["kind"]
+            if kind == "mlp":
+                tp.tp_mlp_backward(X, self.M, h, cfg["ffn"], n, self.A, self.b1, self.B, self.dY,
+                                   cfg.get("residual", False), self.ws_bwd, self.ws_bwd_bytes, dX,
+                                   self.dA, self.db1, self.dB, self.db2)
+            elif kind == "attn":
+                tp.tp_attn_backward(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"],
+                                    cfg.get("causal", True), n, self.Wqkv, self.bqkv, self.Wo,
+                                    self.dY, cfg.get("residual", False), self.ws_bwd,
+                                    self.ws_bwd_bytes, dX, self.dWqkv, self.dbqkv, self.dWo,
+                                    self.dbo)
+            else:
+                tp.tp_layer_backward(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"], cfg["ffn"],
+                                     n, self.w, cfg.get("ln_eps", 1e-5), self.dY, self.ws_bwd,
+                                     self.ws_bwd_bytes, dX, self.grads)
             return
         X = self.X if X is None else X
         Y = self.Y if Y is None else Y
@@ -420,25 +473,30 @@ def run_ours(args, cfg) -> None:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
 
-    # end-to-end through the public API with host buffers: pinned X in,
-    # layer, Y out, every step
+    # end-to-end through the public API with host buffers: pinned X (and,
+    # for a backward step, dY) in, the step, Y (dX) out, every step
     M, h = model.M, cfg["h"]
+    bwd = bool(cfg.get("backward"))
     Xh = torch.from_numpy(inp["X"].view(np.int16)).pin_memory()
     Yh = torch.empty((M, h), dtype=torch.int16).pin_memory()
     Xd = torch.empty_like(model.X)
     Yd = torch.empty_like(model.Y)
-    for _ in range(2):
+    dYh = model.dY.cpu().pin_memory() if bwd else None
+
+    def e2e_step():
         Xd.copy_(Xh, non_blocking=True)
+        if bwd:
+            model.dY.copy_(dYh, non_blocking=True)
         model.step(Xd, Yd)
         Yh.copy_(Yd, non_blocking=True)
+    for _ in range(2):
+        e2e_step()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        Xd.copy_(Xh, non_blocking=True)
-        model.step(Xd, Yd)
-        Yh.copy_(Yd, non_blocking=True)
+        e2e_step()
     e1.record(stream)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / args.steps
@@ -484,7 +542,7 @@ def run_ours(args, cfg) -> None:
         for pos in range(per_step):
             times = [recs[s * per_step + pos][1] for s in range(args.steps)]
             step_breakdown.append([recs[pos][0], round(sum(times) / len(times), 5)])
-    reduce_fig = kernels.get("reduce_partials")
+    reduce_fig = kernels.get("reduce_partials") or kernels.get("reduce_partials_layernorm_backward")
 
     value = w["total_flops"] * world / (ms * 1e-3) / 1e12
     e2e_value = w["total_flops"] * world / (e2e_ms * 1e-3) / 1e12
@@ -515,7 +573,8 @@ def run_ours(args, cfg) -> None:
         "partial_reduce": reduce_fig,
         "kernels": kernels,
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": M * h * 2,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": M * h * 2 * (2 if bwd else 1),
                 "d2h_bytes_per_step": M * h * 2, "ms_per_step": e2e_ms},
         "clocks": clocks,
         "gpu_launches": launches,
@@ -590,7 +649,8 @@ def main():
     ap.add_argument("--sequence-parallel", action="store_true",
                     help="layer workload: run tp_layer_forward_sp on sequence-sharded input")
     ap.add_argument("--backward", action="store_true",
-                    help="MLP workloads: time tp_mlp_backward (dX, weight and bias gradients)")
+                    help="MLP, attention and layer workloads: time the backward pass "
+                         "(tp_mlp_backward / tp_attn_backward / tp_layer_backward)")
     ap.add_argument("--sweep", action="store_true",
                     help="run the workload at every shard count of its sweep (one JSON line)")
     args = ap.parse_args()
@@ -600,8 +660,8 @@ def main():
     if args.shards:
         cfg["n_shards"] = args.shards
     if args.backward:
-        if cfg["kind"] != "mlp":
-            ap.error("--backward applies to the MLP workloads")
+        if cfg["kind"] not in ("mlp", "attn", "layer"):
+            ap.error("--backward applies to the MLP, attention and layer workloads")
         cfg["backward"] = True
     if args.sequence_parallel:
         if cfg["kind"] != "layer":

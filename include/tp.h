@@ -97,7 +97,7 @@ typedef enum {
 
 typedef enum {
     TP_WS_MLP = 0, TP_WS_ATTN = 1, TP_WS_LAYER = 2, TP_WS_LAYER_SP = 3, TP_WS_MLP_BWD = 4,
-    TP_WS_ATTN_CORE_BWD = 5, TP_WS_ATTN_BWD = 6, TP_WS_LAYER_BWD = 7
+    TP_WS_ATTN_CORE_BWD = 5, TP_WS_ATTN_BWD = 6, TP_WS_LAYER_BWD = 7, TP_WS_LN_BWD = 8
 } tp_ws_kind;
 
 /* Weights of one pre-LN layer, all device pointers in the packed shard
@@ -116,6 +116,23 @@ typedef struct {
     const uint16_t* B_shards;    /* TP_SPLIT_ROW of [F][h]: [N][h][F/N] */
     const uint16_t* b2;          /* [h], added once after the sum */
 } tp_layer_weights;
+
+/* Gradients of one layer's parameters (fp32 device buffers), in the same
+   packed layouts as the weights of tp_layer_weights. */
+typedef struct {
+    float* ln1_gamma;    /* [h] */
+    float* ln1_beta;     /* [h] */
+    float* Wqkv_shards;  /* [N][3h/N][h] */
+    float* bqkv_shards;  /* [N][3h/N] */
+    float* Wo_shards;    /* [N][h][h/N] */
+    float* bo;           /* [h] */
+    float* ln2_gamma;    /* [h] */
+    float* ln2_beta;     /* [h] */
+    float* A_shards;     /* [N][F/N][h] */
+    float* b1_shards;    /* [N][F/N] */
+    float* B_shards;     /* [N][h][F/N] */
+    float* b2;           /* [h] */
+} tp_layer_grads;
 
 /* tp_shard_weights - pack W (H_in x H_out, bf16) into N shards.
  * [TP-LLM] "The Core Primitives" (column and row splits); attention section
@@ -309,6 +326,41 @@ tp_status tp_attn_backward(const uint16_t* X, int64_t batch, int64_t seq,
                            float* dbqkv_shards, float* dWo_shards, float* dbo,
                            void* stream);
 
+/* tp_reduce_partials_layernorm_backward - the backward reduction of a pre-LN
+ * block: g = sum_i partials_i (the gradient reaching LN(x), the block's one
+ * reduction, fp32 sum in shard order) through the LayerNorm backward, plus the
+ * residual gradient:
+ *   dX = residual_grad + rstd (g gamma - mean(g gamma) - x_hat mean(g gamma x_hat))
+ * per row (x_hat = (x - mean) rstd, population variance, eps as the forward),
+ * dgamma = sum_rows g x_hat, dbeta = sum_rows g (fp32, deterministic).
+ * partials [N][B][h] fp32; x (the LN input), residual_grad (or NULL), dX
+ * [B][h] bf16; gamma [h] bf16. h % 8 == 0, h <= 16384.
+ * ws >= tp_workspace_bytes(TP_WS_LN_BWD, B, h, 0, N). */
+tp_status tp_reduce_partials_layernorm_backward(const float* partials, int n_shards,
+                                                int64_t B, int64_t h, const uint16_t* x,
+                                                const uint16_t* gamma,
+                                                const uint16_t* residual_grad, float eps,
+                                                void* ws, size_t ws_bytes, uint16_t* dX,
+                                                float* dgamma, float* dbeta, void* stream);
+
+/* tp_layer_backward - gradients of the pre-LN layer of tp_layer_forward
+ * (causal attention) by the tensor-parallel route: the forward is recomputed
+ * from X (LN1, QKV, attention with its log-sum-exp, W_O, LN2); the MLP
+ * block's backward ends in its one reduction, fused with LN2's backward and
+ * the residual (dh1 = dY + LN2'^T sum_i dx2_i); the attention block's backward
+ * ends in its one reduction, fused with LN1's backward and the residual
+ * (dX = dh1 + LN1'^T sum_i dx1_i): two reductions in the backward pass, as
+ * [TP-LLM] "Communication Budget and Scaling Limits" counts. X, dY, dX
+ * [batch*seq][h] bf16; w as tp_layer_forward; g receives every parameter
+ * gradient (fp32, packed layouts). head_dim must be 128.
+ * ws >= tp_workspace_bytes(TP_WS_LAYER_BWD, batch*seq, h, F, N). */
+tp_status tp_layer_backward(const uint16_t* X, int64_t batch, int64_t seq,
+                            int64_t h, int64_t n_heads, int64_t ffn,
+                            int n_shards, const tp_layer_weights* w,
+                            float ln_eps, const uint16_t* dY, void* ws,
+                            size_t ws_bytes, uint16_t* dX,
+                            const tp_layer_grads* g, void* stream);
+
 /* tp_attn_forward - Y = concat_heads(attention) W_O + b_O + residual by the
  * tensor-parallel route: QKV column-parallel by whole heads (+ bias), local
  * attention per shard, W_O row-parallel into N partials, one sum
@@ -444,7 +496,8 @@ tp_status tp_mlp_forward_noalloc(const uint16_t* X, int64_t B, int64_t h,
  * (TP_WS_ATTN, ffn ignored), tp_layer_forward (TP_WS_LAYER),
  * tp_layer_forward_sp (TP_WS_LAYER_SP), tp_mlp_backward (TP_WS_MLP_BWD),
  * tp_attention_backward (TP_WS_ATTN_CORE_BWD, ffn ignored), tp_attn_backward
- * (TP_WS_ATTN_BWD, ffn ignored) or tp_layer_backward (TP_WS_LAYER_BWD).
+ * (TP_WS_ATTN_BWD, ffn ignored), tp_layer_backward (TP_WS_LAYER_BWD) or
+ * tp_reduce_partials_layernorm_backward (TP_WS_LN_BWD, tokens and ffn ignored).
  * tokens = batch * seq. Returns 0 for invalid arguments. */
 size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn,
                           int n_shards);

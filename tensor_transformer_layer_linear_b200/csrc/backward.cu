@@ -101,4 +101,10 @@ int launch_colsum(const void* X, int groups, int rows, int cols, float* partial,
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
 
+int launch_slab_sum(const float* partial, int slabs, int cols, float* out, cudaStream_t s) {
+  colsum_final_kernel<<<static_cast<unsigned>((cols + 31) / 32), 256, 0, s>>>(partial, out, cols,
+                                                                              slabs, 1);
+  return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
+
 }  // namespace tpk

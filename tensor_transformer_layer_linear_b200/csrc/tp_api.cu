@@ -412,6 +412,25 @@ tp_status tp_attention(const uint16_t* QKV_shards, int64_t batch, int64_t seq, i
   return rc == 0 ? TP_OK : (rc == 3 ? TP_ERR_UNSUPPORTED : TP_ERR_CUDA);
 }
 
+// Backward-pass workspace pieces (bytes). Attention rows: per head,
+// tokens + 128 (the query-block overhang), head_dim 128 (n_heads = h / 128).
+static size_t mlp_bwd_bytes(size_t M, size_t H, size_t F, size_t N) {
+  return 3 * round256(M * F * 2) + round256(N * M * H * 4) +
+         round256(static_cast<size_t>(kColsumSlabs) * (F + H) * 4);
+}
+static size_t attn_core_bwd_bytes(size_t M, size_t H) {
+  const size_t rows = M + 128;
+  return round256(H / 128 * rows * 4) + round256(H * rows * 4);
+}
+static size_t attn_bwd_bytes(size_t M, size_t H, size_t N) {
+  // core + QKV, dQKV, O, dO (bf16) + lse + dX partials + column-sum slabs
+  return attn_core_bwd_bytes(M, H) + 2 * round256(M * 3 * H * 2) + 2 * round256(M * H * 2) +
+         round256(H / 128 * (M + 128) * 4) + round256(N * M * H * 4) +
+         round256(static_cast<size_t>(kColsumSlabs) * 4 * H * 4);
+}
+constexpr int kLnBwdMaxCtas = 1024;  // per-CTA column sums of the LN backward
+static size_t ln_bwd_bytes(size_t H) { return round256(2 * static_cast<size_t>(kLnBwdMaxCtas) * H * 4); }
+
 size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int n_shards) {
   if (tokens <= 0 || h <= 0 || n_shards <= 0) return 0;
   const size_t M = static_cast<size_t>(tokens), H = static_cast<size_t>(h);
@@ -427,19 +446,19 @@ size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int 
   if (kind == TP_WS_MLP_BWD) {
     if (ffn <= 0) return 0;
     // GeLU'(Z), H, dZ [N][M][F/N] bf16; dX partials [N][M][h] fp32; column-sum slabs
-    return 3 * round256(M * static_cast<size_t>(ffn) * 2) + partials +
-           round256(static_cast<size_t>(kColsumSlabs) * (static_cast<size_t>(ffn) + H) * 4);
+    return mlp_bwd_bytes(M, H, static_cast<size_t>(ffn), N);
   }
-  if (kind == TP_WS_ATTN_CORE_BWD || kind == TP_WS_ATTN_BWD) {
-    // D [n_heads][M + 128] and the dQ accumulator [n_heads][128][M + 128]
-    // fp32 (head_dim 128: n_heads = h / 128)
-    const size_t rows = M + 128;
-    const size_t core = round256(H / 128 * rows * 4) + round256(H * rows * 4);
-    if (kind == TP_WS_ATTN_CORE_BWD) return core;
-    // + QKV, O, dO, dQKV (bf16), lse, the dX partials and column-sum slabs
-    return core + 2 * round256(M * 3 * H * 2) + 2 * round256(M * H * 2) +
-           round256(H / 128 * rows * 4) + partials +
-           round256(static_cast<size_t>(kColsumSlabs) * 4 * H * 4);
+  if (kind == TP_WS_ATTN_CORE_BWD) return attn_core_bwd_bytes(M, H);
+  if (kind == TP_WS_ATTN_BWD) return attn_bwd_bytes(M, H, N);
+  if (kind == TP_WS_LN_BWD) return ln_bwd_bytes(H);
+  if (kind == TP_WS_LAYER_BWD) {
+    if (ffn <= 0) return 0;
+    // x1, h1, x2, dh1 + the attention part (its own partials and slabs
+    // reused by the MLP) + G, H, dZ of the MLP + LN-backward column sums
+    const size_t F = static_cast<size_t>(ffn);
+    const size_t slabs = round256(static_cast<size_t>(kColsumSlabs) * (F + 4 * H) * 4);
+    return 4 * round256(M * H * 2) + attn_bwd_bytes(M, H, N) + 3 * round256(M * F * 2) + slabs +
+           ln_bwd_bytes(H);
   }
   if (kind == TP_WS_LAYER || kind == TP_WS_LAYER_SP) {
     if (ffn <= 0) return 0;
@@ -760,6 +779,80 @@ tp_status tp_attn_forward_gqa(const uint16_t* X, int64_t batch, int64_t seq, int
   return tp_reduce_partials(part, n_shards, M, h, bo, residual, Y, stream);
 }
 
+// One GEMM of a backward pass over all shards (see tpk::GemmProblem).
+static tp_status bwd_gemm(const DevInfo& d, cudaStream_t s, int n_shards, const void* A, bool a_b,
+                          bool a_mn, const void* B, bool b_b, bool b_mn, void* D, int m, int nc,
+                          int k, bool f32, int act = 0, const void* aux = nullptr,
+                          const void* bias = nullptr, void* aux_out = nullptr,
+                          int kid = tpk::KID_GEMM_BACKWARD) {
+  tpk::GemmProblem g;
+  g.A = A; g.B = B; g.D = D; g.bias = bias;
+  g.M = m; g.Nc = nc; g.K = k; g.G = n_shards;
+  g.a_batched = a_b; g.b_batched = b_b; g.a_mn = a_mn; g.b_mn = b_mn;
+  g.out_f32 = f32; g.act = act; g.aux = aux; g.aux_out = aux_out;
+  TraceScope ts(kid, s);
+  return tpk::launch_gemm(g, s, d.err, d.num_sms) == 0 ? TP_OK : TP_ERR_CUDA;
+}
+
+static tp_status bwd_colsum(const DevInfo& d, cudaStream_t s, const uint16_t* X, int groups,
+                            int rows, int cols, float* slabs, float* out) {
+  TraceScope ts(tpk::KID_COLSUM, s);
+  return tpk::launch_colsum(X, groups, rows, cols, slabs, kColsumSlabs, out, s, d.num_sms) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+struct MlpBwdBufs {
+  uint16_t* G;   // GeLU'(Z) [N][M][F/N]
+  uint16_t* H;   // GeLU(Z)  [N][M][F/N]
+  uint16_t* dZ;  // [N][M][F/N]
+  float* part;   // dX partials [N][M][h]
+  float* slabs;  // column-sum scratch
+};
+
+// The MLP backward except its reduction: recompute, dZ, weight and bias
+// gradients, and last the N partials dX_i = dZ_i A_i^T in b.part.
+static tp_status mlp_backward_core(const DevInfo& d, cudaStream_t s, const uint16_t* X, int M,
+                                   int H, int F, int n_shards, const uint16_t* A_shards,
+                                   const uint16_t* b1_shards, const uint16_t* B_shards,
+                                   const uint16_t* dY, const MlpBwdBufs& b, float* dA_shards,
+                                   float* db1, float* dB_shards, float* db2) {
+  const int fs = F / n_shards;
+  // recompute the column layer: H_i = GeLU(Z_i), Z_i = X A_i + b1_i, with
+  // GeLU'(Z_i) kept for the backward of the activation
+  tp_status st = bwd_gemm(d, s, n_shards, X, false, false, A_shards, true, false, b.H, M, fs, H,
+                          false, 4, nullptr, b1_shards, b.G, tpk::KID_GEMM_COLUMN);
+  if (st != TP_OK) return st;
+  // dZ_i = (dY B_i^T) * GeLU'(Z_i): dY shared; B_shards[i] = B_i^T is the MN-major operand
+  st = bwd_gemm(d, s, n_shards, dY, false, false, B_shards, true, true, b.dZ, M, fs, H, false, 3,
+                b.G);
+  if (st != TP_OK) return st;
+  // dA_i^T = dZ_i^T X (packed like A_shards), dB_i^T = dY^T H_i (packed like B_shards)
+  st = bwd_gemm(d, s, n_shards, b.dZ, true, true, X, false, true, dA_shards, fs, H, M, true);
+  if (st != TP_OK) return st;
+  st = bwd_gemm(d, s, n_shards, dY, false, true, b.H, true, true, dB_shards, H, fs, M, true);
+  if (st != TP_OK) return st;
+  // bias gradients: column sums over the token rows
+  st = bwd_colsum(d, s, b.dZ, n_shards, M, fs, b.slabs, db1);
+  if (st != TP_OK) return st;
+  st = bwd_colsum(d, s, dY, 1, M, H, b.slabs, db2);
+  if (st != TP_OK) return st;
+  // dX partials: dZ_i A_i^T; A_shards[i] = A_i^T is the MN-major operand
+  return bwd_gemm(d, s, n_shards, b.dZ, true, false, A_shards, true, true, b.part, M, H, fs, true);
+}
+
+static MlpBwdBufs mlp_bwd_layout(void* ws, size_t M, size_t H, size_t F, size_t N) {
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  MlpBwdBufs b;
+  const size_t act_b = round256(M * F * 2);
+  b.G = reinterpret_cast<uint16_t*>(p); p += act_b;
+  b.H = reinterpret_cast<uint16_t*>(p); p += act_b;
+  b.dZ = reinterpret_cast<uint16_t*>(p); p += act_b;
+  b.part = reinterpret_cast<float*>(p); p += round256(N * M * H * 4);
+  b.slabs = reinterpret_cast<float*>(p);
+  return b;
+}
+
 tp_status tp_mlp_backward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, int n_shards,
                           const uint16_t* A_shards, const uint16_t* b1_shards,
                           const uint16_t* B_shards, const uint16_t* dY, int residual, void* ws,
@@ -781,56 +874,13 @@ tp_status tp_mlp_backward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, 
   DevInfo d;
   tp_status st = device_info(&d);
   if (st != TP_OK) return st;
-  const int M = static_cast<int>(B), H = static_cast<int>(h), F = static_cast<int>(ffn);
-  const int fs = F / n_shards;
-  const size_t act_b = round256(static_cast<size_t>(M) * F * 2);
-  uint8_t* p = static_cast<uint8_t*>(ws);
-  uint16_t* Gp = reinterpret_cast<uint16_t*>(p); p += act_b;
-  uint16_t* Hs = reinterpret_cast<uint16_t*>(p); p += act_b;
-  uint16_t* dZ = reinterpret_cast<uint16_t*>(p); p += act_b;
-  float* part = reinterpret_cast<float*>(p);
-  p += round256(static_cast<size_t>(n_shards) * M * H * 4);
-  float* slabs = reinterpret_cast<float*>(p);
-  cudaStream_t s = as_stream(stream);
-
-  auto gemm = [&](const void* A, bool a_b, bool a_mn, const void* Bop, bool b_b, bool b_mn,
-                  void* D, int m, int nc, int k, bool f32, int act, const void* aux,
-                  const void* bias = nullptr, void* aux_out = nullptr,
-                  int kid = tpk::KID_GEMM_BACKWARD) {
-    tpk::GemmProblem g;
-    g.A = A; g.B = Bop; g.D = D; g.bias = bias;
-    g.M = m; g.Nc = nc; g.K = k; g.G = n_shards;
-    g.a_batched = a_b; g.b_batched = b_b; g.a_mn = a_mn; g.b_mn = b_mn;
-    g.out_f32 = f32; g.act = act; g.aux = aux; g.aux_out = aux_out;
-    TraceScope ts(kid, s);
-    return tpk::launch_gemm(g, s, d.err, d.num_sms) == 0 ? TP_OK : TP_ERR_CUDA;
-  };
-  // recompute the column layer: H_i = GeLU(Z_i), Z_i = X A_i + b1_i, with
-  // GeLU'(Z_i) kept for the backward of the activation
-  st = gemm(X, false, false, A_shards, true, false, Hs, M, fs, H, false, 4, nullptr, b1_shards,
-            Gp, tpk::KID_GEMM_COLUMN);
-  if (st != TP_OK) return st;
-  // dZ_i = (dY B_i^T) * GeLU'(Z_i): dY shared; B_shards[i] = B_i^T is the MN-major operand
-  st = gemm(dY, false, false, B_shards, true, true, dZ, M, fs, H, false, 3, Gp);
-  if (st != TP_OK) return st;
-  // dX partials: dZ_i A_i^T; A_shards[i] = A_i^T is the MN-major operand
-  st = gemm(dZ, true, false, A_shards, true, true, part, M, H, fs, true, 0, nullptr);
+  const MlpBwdBufs b = mlp_bwd_layout(ws, B, h, ffn, n_shards);
+  st = mlp_backward_core(d, as_stream(stream), X, static_cast<int>(B), static_cast<int>(h),
+                         static_cast<int>(ffn), n_shards, A_shards, b1_shards, B_shards, dY, b,
+                         dA_shards, db1, dB_shards, db2);
   if (st != TP_OK) return st;
   // the one reduction of the backward: dX = sum_i dX_i (+ dY through the residual)
-  st = tp_reduce_partials(part, n_shards, B, h, nullptr, residual ? dY : nullptr, dX, stream);
-  if (st != TP_OK) return st;
-  // dA_i^T = dZ_i^T X (packed like A_shards), dB_i^T = dY^T H_i (packed like B_shards)
-  st = gemm(dZ, true, true, X, false, true, dA_shards, fs, H, M, true, 0, nullptr);
-  if (st != TP_OK) return st;
-  st = gemm(dY, false, true, Hs, true, true, dB_shards, H, fs, M, true, 0, nullptr);
-  if (st != TP_OK) return st;
-  // bias gradients: column sums over the token rows
-  TraceScope ts(tpk::KID_COLSUM, s);
-  if (tpk::launch_colsum(dZ, n_shards, M, fs, slabs, kColsumSlabs, db1, s, d.num_sms) != 0)
-    return TP_ERR_CUDA;
-  if (tpk::launch_colsum(dY, 1, M, H, slabs, kColsumSlabs, db2, s, d.num_sms) != 0)
-    return TP_ERR_CUDA;
-  return TP_OK;
+  return tp_reduce_partials(b.part, n_shards, B, h, nullptr, residual ? dY : nullptr, dX, stream);
 }
 
 tp_status tp_attention_lse(const uint16_t* QKV_shards, int64_t batch, int64_t seq, int64_t h,
@@ -886,6 +936,73 @@ tp_status tp_attention_backward(const uint16_t* QKV_shards, const uint16_t* O_sh
   return rc == 0 ? TP_OK : TP_ERR_CUDA;
 }
 
+struct AttnBwdBufs {
+  void* core;      // D and the dQ accumulator
+  uint16_t* qkv;   // [N][M][3h/N]: the forward's QKV
+  uint16_t* dqkv;  // [N][M][3h/N]
+  uint16_t* o;     // [N][M][h/N]: the forward's attention output
+  uint16_t* dO;    // [N][M][h/N]
+  float* lse;      // the forward's log-sum-exp
+  float* part;     // dX partials [N][M][h]
+  float* slabs;    // column-sum scratch
+};
+
+static AttnBwdBufs attn_bwd_layout(void* ws, size_t M, size_t H, size_t N) {
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  AttnBwdBufs b;
+  b.core = p; p += attn_core_bwd_bytes(M, H);
+  b.qkv = reinterpret_cast<uint16_t*>(p); p += round256(M * 3 * H * 2);
+  b.dqkv = reinterpret_cast<uint16_t*>(p); p += round256(M * 3 * H * 2);
+  b.o = reinterpret_cast<uint16_t*>(p); p += round256(M * H * 2);
+  b.dO = reinterpret_cast<uint16_t*>(p); p += round256(M * H * 2);
+  b.lse = reinterpret_cast<float*>(p); p += round256(H / 128 * (M + 128) * 4);
+  b.part = reinterpret_cast<float*>(p); p += round256(N * M * H * 4);
+  b.slabs = reinterpret_cast<float*>(p);
+  return b;
+}
+
+// The attention block's backward except its reduction, with b.qkv, b.o and
+// b.lse already holding the forward's values for X: dO, the head gradients,
+// the weight and bias gradients, and last the N partials
+// dX_i = dQKV_i W_QKV,i^T in b.part.
+static tp_status attn_backward_core(const DevInfo& d, void* stream, const uint16_t* X,
+                                    int64_t batch, int64_t seq, int64_t h, int64_t n_heads,
+                                    int causal, int n_shards, const uint16_t* Wqkv_shards,
+                                    const uint16_t* Wo_shards, const uint16_t* dY,
+                                    const AttnBwdBufs& b, float* dWqkv_shards, float* dbqkv_shards,
+                                    float* dWo_shards, float* dbo) {
+  cudaStream_t s = as_stream(stream);
+  const int M = static_cast<int>(batch * seq), H = static_cast<int>(h);
+  const int hs = H / n_shards;
+  // dO_i = dY W_O,i^T; Wo_shards[i] = W_O,i^T is the MN-major operand
+  tp_status st = bwd_gemm(d, s, n_shards, dY, false, false, Wo_shards, true, true, b.dO, M, hs,
+                          H, false);
+  if (st != TP_OK) return st;
+  st = tp_attention_backward(b.qkv, b.o, b.dO, b.lse, batch, seq, h, n_heads, causal, n_shards,
+                             b.core, attn_core_bwd_bytes(M, H), b.dqkv, stream);
+  if (st != TP_OK) return st;
+  // dW_QKV,i^T = dQKV_i^T X (packed like Wqkv_shards), dW_O,i^T = dY^T O_i (like Wo_shards)
+  st = bwd_gemm(d, s, n_shards, b.dqkv, true, true, X, false, true, dWqkv_shards, 3 * hs, H, M,
+                true);
+  if (st != TP_OK) return st;
+  st = bwd_gemm(d, s, n_shards, dY, false, true, b.o, true, true, dWo_shards, H, hs, M, true);
+  if (st != TP_OK) return st;
+  st = bwd_colsum(d, s, b.dqkv, n_shards, M, 3 * hs, b.slabs, dbqkv_shards);
+  if (st != TP_OK) return st;
+  st = bwd_colsum(d, s, dY, 1, M, H, b.slabs, dbo);
+  if (st != TP_OK) return st;
+  // dX partials: dQKV_i W_QKV,i^T; Wqkv_shards[i] = W_QKV,i^T is the MN-major operand
+  return bwd_gemm(d, s, n_shards, b.dqkv, true, false, Wqkv_shards, true, true, b.part, M, H,
+                  3 * hs, true);
+}
+
+static bool attn_bwd_shape_ok(int64_t batch, int64_t seq, int64_t h, int64_t n_heads,
+                              int n_shards) {
+  return batch > 0 && seq > 0 && h > 0 && n_heads > 0 && n_shards > 0 && h % n_heads == 0 &&
+         n_heads % n_shards == 0 && batch * seq <= kIntMax &&
+         static_cast<int64_t>(n_shards) * batch * (n_heads / n_shards) <= 65535;
+}
+
 tp_status tp_attn_backward(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
                            int64_t n_heads, int causal, int n_shards, const uint16_t* Wqkv_shards,
                            const uint16_t* bqkv_shards, const uint16_t* Wo_shards,
@@ -896,13 +1013,10 @@ tp_status tp_attn_backward(const uint16_t* X, int64_t batch, int64_t seq, int64_
       dX == nullptr || dWqkv_shards == nullptr || dbqkv_shards == nullptr ||
       dWo_shards == nullptr || dbo == nullptr || ws == nullptr)
     return TP_ERR_NULL;
-  if (batch <= 0 || seq <= 0 || h <= 0 || n_heads <= 0 || n_shards <= 0) return TP_ERR_SHAPE;
-  if (h % n_heads || n_heads % n_shards) return TP_ERR_SHAPE;
+  if (!attn_bwd_shape_ok(batch, seq, h, n_heads, n_shards)) return TP_ERR_SHAPE;
   if (h / n_heads != 128) return TP_ERR_UNSUPPORTED;
-  if (batch * seq > kIntMax || seq > kIntMax) return TP_ERR_SHAPE;
-  const int64_t M64 = batch * seq;
-  const size_t need = tp_workspace_bytes(TP_WS_ATTN_BWD, M64, h, 0, n_shards);
-  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  const int64_t M = batch * seq;
+  if (ws_bytes < tp_workspace_bytes(TP_WS_ATTN_BWD, M, h, 0, n_shards)) return TP_ERR_WORKSPACE;
   if (!al16(ws) || !al16(X) || !al16(Wqkv_shards) || !al16(Wo_shards) || !al16(dY) ||
       !al16(dX) || !al16(dWqkv_shards) || !al16(dbqkv_shards) || !al16(dWo_shards) ||
       !al16(dbo) || (bqkv_shards && !al16(bqkv_shards)))
@@ -910,60 +1024,132 @@ tp_status tp_attn_backward(const uint16_t* X, int64_t batch, int64_t seq, int64_
   DevInfo d;
   tp_status st = device_info(&d);
   if (st != TP_OK) return st;
-  const int M = static_cast<int>(M64), H = static_cast<int>(h);
-  const int hs = H / n_shards;
-  const size_t rows = static_cast<size_t>(M) + 128;
-  uint8_t* p = static_cast<uint8_t*>(ws);
-  void* core = p; p += tp_workspace_bytes(TP_WS_ATTN_CORE_BWD, M64, h, 0, n_shards);
-  uint16_t* qkv = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * 3 * H * 2);
-  uint16_t* dqkv = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * 3 * H * 2);
-  uint16_t* o = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * H * 2);
-  uint16_t* dO = reinterpret_cast<uint16_t*>(p); p += round256(static_cast<size_t>(M) * H * 2);
-  float* lse = reinterpret_cast<float*>(p); p += round256(static_cast<size_t>(H) / 128 * rows * 4);
-  float* part = reinterpret_cast<float*>(p);
-  p += round256(static_cast<size_t>(n_shards) * M * H * 4);
-  float* slabs = reinterpret_cast<float*>(p);
-  cudaStream_t s = as_stream(stream);
-  auto gemm = [&](const void* A, bool a_b, bool a_mn, const void* Bop, bool b_b, bool b_mn,
-                  void* D, int m, int nc, int k, bool f32) {
-    tpk::GemmProblem g;
-    g.A = A; g.B = Bop; g.D = D; g.bias = nullptr;
-    g.M = m; g.Nc = nc; g.K = k; g.G = n_shards;
-    g.a_batched = a_b; g.b_batched = b_b; g.a_mn = a_mn; g.b_mn = b_mn;
-    g.out_f32 = f32; g.act = 0;
-    TraceScope ts(tpk::KID_GEMM_BACKWARD, s);
-    return tpk::launch_gemm(g, s, d.err, d.num_sms) == 0 ? TP_OK : TP_ERR_CUDA;
-  };
+  const AttnBwdBufs b = attn_bwd_layout(ws, M, h, n_shards);
   // recompute the forward: QKV_i = X W_QKV,i + b_i, O_i and the lse
-  st = tp_column_linear(X, M64, h, Wqkv_shards, bqkv_shards, 3 * h, n_shards, TP_ACT_NONE, qkv,
+  st = tp_column_linear(X, M, h, Wqkv_shards, bqkv_shards, 3 * h, n_shards, TP_ACT_NONE, b.qkv,
                         stream);
   if (st != TP_OK) return st;
-  st = tp_attention_lse(qkv, batch, seq, h, n_heads, causal, n_shards, o, lse, stream);
+  st = tp_attention_lse(b.qkv, batch, seq, h, n_heads, causal, n_shards, b.o, b.lse, stream);
   if (st != TP_OK) return st;
-  // dO_i = dY W_O,i^T; Wo_shards[i] = W_O,i^T is the MN-major operand
-  st = gemm(dY, false, false, Wo_shards, true, true, dO, M, hs, H, false);
-  if (st != TP_OK) return st;
-  st = tp_attention_backward(qkv, o, dO, lse, batch, seq, h, n_heads, causal, n_shards, core,
-                             tp_workspace_bytes(TP_WS_ATTN_CORE_BWD, M64, h, 0, n_shards), dqkv,
-                             stream);
-  if (st != TP_OK) return st;
-  // dX partials: dQKV_i W_QKV,i^T; Wqkv_shards[i] = W_QKV,i^T is the MN-major operand
-  st = gemm(dqkv, true, false, Wqkv_shards, true, true, part, M, H, 3 * hs, true);
+  st = attn_backward_core(d, stream, X, batch, seq, h, n_heads, causal, n_shards, Wqkv_shards,
+                          Wo_shards, dY, b, dWqkv_shards, dbqkv_shards, dWo_shards, dbo);
   if (st != TP_OK) return st;
   // the one reduction of the block's backward: dX = sum_i dX_i (+ dY)
-  st = tp_reduce_partials(part, n_shards, M64, h, nullptr, residual ? dY : nullptr, dX, stream);
-  if (st != TP_OK) return st;
-  // dW_QKV,i^T = dQKV_i^T X (packed like Wqkv_shards), dW_O,i^T = dY^T O_i (like Wo_shards)
-  st = gemm(dqkv, true, true, X, false, true, dWqkv_shards, 3 * hs, H, M, true);
-  if (st != TP_OK) return st;
-  st = gemm(dY, false, true, o, true, true, dWo_shards, H, hs, M, true);
-  if (st != TP_OK) return st;
-  TraceScope ts(tpk::KID_COLSUM, s);
-  if (tpk::launch_colsum(dqkv, n_shards, M, 3 * hs, slabs, kColsumSlabs, dbqkv_shards, s,
-                         d.num_sms) != 0)
-    return TP_ERR_CUDA;
-  if (tpk::launch_colsum(dY, 1, M, H, slabs, kColsumSlabs, dbo, s, d.num_sms) != 0)
-    return TP_ERR_CUDA;
-  return TP_OK;
+  return tp_reduce_partials(b.part, n_shards, M, h, nullptr, residual ? dY : nullptr, dX, stream);
 }
+
+tp_status tp_reduce_partials_layernorm_backward(const float* partials, int n_shards, int64_t B,
+                                                int64_t h, const uint16_t* x,
+                                                const uint16_t* gamma,
+                                                const uint16_t* residual_grad, float eps,
+                                                void* ws, size_t ws_bytes, uint16_t* dX,
+                                                float* dgamma, float* dbeta, void* stream) {
+  if (partials == nullptr || x == nullptr || gamma == nullptr || dX == nullptr ||
+      dgamma == nullptr || dbeta == nullptr || ws == nullptr)
+    return TP_ERR_NULL;
+  if (B <= 0 || h <= 0 || n_shards <= 0 || h % 8 || h > 16384) return TP_ERR_SHAPE;
+  if (ws_bytes < tp_workspace_bytes(TP_WS_LN_BWD, B, h, 0, n_shards)) return TP_ERR_WORKSPACE;
+  if (!al16(partials) || !al16(x) || !al16(gamma) || !al16(dX) || !al16(dgamma) ||
+      !al16(dbeta) || !al16(ws) || (residual_grad && !al16(residual_grad)))
+    return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  TraceScope ts(tpk::KID_LAYERNORM_BWD, s);
+  return tpk::launch_rows_sum_ln_bwd(partials, n_shards, B, h, x, gamma, residual_grad, eps, dX,
+                                     dgamma, dbeta, static_cast<float*>(ws), kLnBwdMaxCtas, s,
+                                     d.num_sms) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_layer_backward(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
+                            int64_t n_heads, int64_t ffn, int n_shards, const tp_layer_weights* w,
+                            float ln_eps, const uint16_t* dY, void* ws, size_t ws_bytes,
+                            uint16_t* dX, const tp_layer_grads* g, void* stream) {
+  if (X == nullptr || w == nullptr || dY == nullptr || dX == nullptr || g == nullptr ||
+      ws == nullptr)
+    return TP_ERR_NULL;
+  if (w->ln1_gamma == nullptr || w->ln1_beta == nullptr || w->Wqkv_shards == nullptr ||
+      w->Wo_shards == nullptr || w->ln2_gamma == nullptr || w->ln2_beta == nullptr ||
+      w->A_shards == nullptr || w->B_shards == nullptr)
+    return TP_ERR_NULL;
+  if (g->ln1_gamma == nullptr || g->ln1_beta == nullptr || g->Wqkv_shards == nullptr ||
+      g->bqkv_shards == nullptr || g->Wo_shards == nullptr || g->bo == nullptr ||
+      g->ln2_gamma == nullptr || g->ln2_beta == nullptr || g->A_shards == nullptr ||
+      g->b1_shards == nullptr || g->B_shards == nullptr || g->b2 == nullptr)
+    return TP_ERR_NULL;
+  if (!attn_bwd_shape_ok(batch, seq, h, n_heads, n_shards) || ffn <= 0 || ffn % n_shards ||
+      (ffn / n_shards) % 8 || h % 8 || h > 16384 || ffn > kIntMax)
+    return TP_ERR_SHAPE;
+  if (h / n_heads != 128) return TP_ERR_UNSUPPORTED;
+  const int64_t M = batch * seq;
+  if (ws_bytes < tp_workspace_bytes(TP_WS_LAYER_BWD, M, h, ffn, n_shards)) return TP_ERR_WORKSPACE;
+  if (!al16(ws) || !al16(X) || !al16(dY) || !al16(dX)) return TP_ERR_ALIGN;
+  const float* grads[] = {g->ln1_gamma, g->ln1_beta, g->Wqkv_shards, g->bqkv_shards,
+                          g->Wo_shards, g->bo, g->ln2_gamma, g->ln2_beta, g->A_shards,
+                          g->b1_shards, g->B_shards, g->b2};
+  for (const float* ptr : grads)
+    if (!al16(ptr)) return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  const size_t Mz = static_cast<size_t>(M), H = static_cast<size_t>(h);
+  const size_t F = static_cast<size_t>(ffn);
+  const size_t act_b = round256(Mz * H * 2);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  uint16_t* x1 = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* h1 = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* x2 = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* dh1 = reinterpret_cast<uint16_t*>(p); p += act_b;
+  AttnBwdBufs ab = attn_bwd_layout(p, Mz, H, n_shards);
+  p += attn_bwd_bytes(Mz, H, n_shards);
+  MlpBwdBufs mb;
+  mb.G = reinterpret_cast<uint16_t*>(p); p += round256(Mz * F * 2);
+  mb.H = reinterpret_cast<uint16_t*>(p); p += round256(Mz * F * 2);
+  mb.dZ = reinterpret_cast<uint16_t*>(p); p += round256(Mz * F * 2);
+  float* slabs = reinterpret_cast<float*>(p);
+  p += round256(static_cast<size_t>(kColsumSlabs) * (F + 4 * H) * 4);
+  float* lnb = reinterpret_cast<float*>(p);
+  mb.part = ab.part;  // the two blocks' partials are used one after the other
+  mb.slabs = slabs;
+  ab.slabs = slabs;
+  const size_t lnb_bytes = ln_bwd_bytes(H);
+
+  // forward recompute: x1 = LN1(X), QKV, O, lse, h1 = X + Attn(x1), x2 = LN2(h1)
+  st = tp_layernorm(X, M, h, w->ln1_gamma, w->ln1_beta, ln_eps, x1, stream);
+  if (st != TP_OK) return st;
+  st = tp_column_linear(x1, M, h, w->Wqkv_shards, w->bqkv_shards, 3 * h, n_shards, TP_ACT_NONE,
+                        ab.qkv, stream);
+  if (st != TP_OK) return st;
+  st = tp_attention_lse(ab.qkv, batch, seq, h, n_heads, 1, n_shards, ab.o, ab.lse, stream);
+  if (st != TP_OK) return st;
+  st = tp_row_linear(ab.o, M, h, w->Wo_shards, h, n_shards, ab.part, stream);
+  if (st != TP_OK) return st;
+  st = tp_reduce_partials_layernorm(ab.part, n_shards, M, h, w->bo, X, w->ln2_gamma, w->ln2_beta,
+                                    ln_eps, h1, x2, stream);
+  if (st != TP_OK) return st;
+  // MLP block: gradients and the partials of dx2; its one reduction is fused
+  // with LN2's backward and the residual: dh1 = dY + LN2'(h1)^T sum_i dx2_i
+  st = mlp_backward_core(d, s, x2, static_cast<int>(M), static_cast<int>(h),
+                         static_cast<int>(ffn), n_shards, w->A_shards, w->b1_shards, w->B_shards,
+                         dY, mb, g->A_shards, g->b1_shards, g->B_shards, g->b2);
+  if (st != TP_OK) return st;
+  st = tp_reduce_partials_layernorm_backward(mb.part, n_shards, M, h, h1, w->ln2_gamma, dY,
+                                             ln_eps, lnb, lnb_bytes, dh1, g->ln2_gamma,
+                                             g->ln2_beta, stream);
+  if (st != TP_OK) return st;
+  // attention block: gradients and the partials of dx1; its one reduction is
+  // fused with LN1's backward and the residual: dX = dh1 + LN1'(X)^T sum_i dx1_i
+  st = attn_backward_core(d, stream, x1, batch, seq, h, n_heads, 1, n_shards, w->Wqkv_shards,
+                          w->Wo_shards, dh1, ab, g->Wqkv_shards, g->bqkv_shards, g->Wo_shards,
+                          g->bo);
+  if (st != TP_OK) return st;
+  return tp_reduce_partials_layernorm_backward(ab.part, n_shards, M, h, X, w->ln1_gamma, dh1,
+                                               ln_eps, lnb, lnb_bytes, dX, g->ln1_gamma,
+                                               g->ln1_beta, stream);
+}
+
 }  // extern "C"

@@ -111,4 +111,16 @@ int launch_shard(const void* W, int64_t h_in, int64_t h_out, int n_shards, int k
 int launch_colsum(const void* X, int groups, int rows, int cols, float* partial, int max_slabs,
                   float* out, cudaStream_t s, int num_sms);
 
+// out[c] = sum over s of partial[s][c] (fp32), in slab order.
+int launch_slab_sum(const float* partial, int slabs, int cols, float* out, cudaStream_t s);
+
+// LayerNorm backward fused with the sum of N fp32 partials (the gradient at
+// the LN output) and a residual gradient: dx = residual + LN'(x)^T sum_i P_i
+// (bf16), dgamma, dbeta (fp32). part holds 2 * max_ctas * h floats of
+// per-CTA column sums. h % 8 == 0, h <= 16384.
+int launch_rows_sum_ln_bwd(const float* P, int n_shards, int64_t rows, int64_t h, const void* x,
+                           const void* gamma, const void* residual, float eps, void* dx,
+                           float* dgamma, float* dbeta, float* part, int max_ctas,
+                           cudaStream_t s, int num_sms);
+
 }  // namespace tpk

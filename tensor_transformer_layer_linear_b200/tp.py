@@ -32,12 +32,18 @@ TP_ERR_WORKSPACE, TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_TIMEOUT = 4, 5, 6, 7
 TP_SPLIT_COLUMN, TP_SPLIT_ROW, TP_SPLIT_QKV_HEADS, TP_SPLIT_GATE_UP = 0, 1, 2, 3
 TP_ACT_NONE, TP_ACT_GELU_ERF, TP_ACT_SWIGLU = 0, 1, 2
 TP_WS_MLP, TP_WS_ATTN, TP_WS_LAYER, TP_WS_LAYER_SP, TP_WS_MLP_BWD = 0, 1, 2, 3, 4
-TP_WS_ATTN_CORE_BWD, TP_WS_ATTN_BWD, TP_WS_LAYER_BWD = 5, 6, 7
+TP_WS_ATTN_CORE_BWD, TP_WS_ATTN_BWD, TP_WS_LAYER_BWD, TP_WS_LN_BWD = 5, 6, 7, 8
 
 _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
 
 class tp_layer_weights(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in (
+        "ln1_gamma", "ln1_beta", "Wqkv_shards", "bqkv_shards", "Wo_shards", "bo",
+        "ln2_gamma", "ln2_beta", "A_shards", "b1_shards", "B_shards", "b2")]
+
+
+class tp_layer_grads(ctypes.Structure):
     _fields_ = [(n, _vp) for n in (
         "ln1_gamma", "ln1_beta", "Wqkv_shards", "bqkv_shards", "Wo_shards", "bo",
         "ln2_gamma", "ln2_beta", "A_shards", "b1_shards", "B_shards", "b2")]
@@ -78,6 +84,11 @@ _SIGS = {
                                      _vp, _sz, _vp, _vp]),
     "tp_attn_backward": (_i32, [_vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp,
                                 _i32, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "tp_reduce_partials_layernorm_backward": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _vp, _f32,
+                                                     _vp, _sz, _vp, _vp, _vp, _vp]),
+    "tp_layer_backward": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32,
+                                 ctypes.POINTER(tp_layer_weights), _f32, _vp, _vp, _sz, _vp,
+                                 ctypes.POINTER(tp_layer_grads), _vp]),
     "tp_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "tp_get_last_error": (_i32, [_vp]),
     "tp_status_string": (ctypes.c_char_p, [_i32]),
@@ -308,6 +319,28 @@ def tp_attn_backward(X, batch, seq, h, n_heads, causal, n_shards, Wqkv_shards, b
                                 int(bool(residual)), _p(ws), ws_bytes, _p(dX), _p(dWqkv_shards),
                                 _p(dbqkv_shards), _p(dWo_shards), _p(dbo), _s(stream)),
            "tp_attn_backward")
+
+
+def tp_reduce_partials_layernorm_backward(partials, n_shards, B, h, x, gamma, residual_grad, eps,
+                                          ws, ws_bytes, dX, dgamma, dbeta, stream=None):
+    _check(lib.tp_reduce_partials_layernorm_backward(
+        _p(partials), n_shards, B, h, _p(x), _p(gamma), _p(residual_grad), eps, _p(ws), ws_bytes,
+        _p(dX), _p(dgamma), _p(dbeta), _s(stream)), "tp_reduce_partials_layernorm_backward")
+
+
+def make_layer_grads(**tensors) -> tp_layer_grads:
+    """Build the tp_layer_grads struct from fp32 tensors named like its fields."""
+    g = tp_layer_grads()
+    for name, _ in tp_layer_grads._fields_:
+        setattr(g, name, _p(tensors.get(name)))
+    return g
+
+
+def tp_layer_backward(X, batch, seq, h, n_heads, ffn, n_shards, weights: tp_layer_weights, ln_eps,
+                      dY, ws, ws_bytes, dX, grads: tp_layer_grads, stream=None):
+    _check(lib.tp_layer_backward(_p(X), batch, seq, h, n_heads, ffn, n_shards,
+                                 ctypes.byref(weights), ln_eps, _p(dY), _p(ws), ws_bytes, _p(dX),
+                                 ctypes.byref(grads), _s(stream)), "tp_layer_backward")
 
 
 def tp_get_last_error(stream=None) -> int:

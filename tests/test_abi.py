@@ -57,7 +57,18 @@ def test_workspace_bytes():
     layer = tp.tp_workspace_bytes(tp.TP_WS_LAYER, M, h, F, N)
     assert layer >= mlp + attn - N * M * h * 4
     assert tp.tp_workspace_bytes(tp.TP_WS_MLP, 0, h, F, N) == 0
-    assert tp.tp_workspace_bytes(7, M, h, F, N) == 0
+    assert tp.tp_workspace_bytes(99, M, h, F, N) == 0
+    # backward passes: the recomputed activations, gradients and partials fit
+    mlp_b = tp.tp_workspace_bytes(tp.TP_WS_MLP_BWD, M, h, F, N)
+    assert mlp_b >= 3 * M * F * 2 + N * M * h * 4
+    core = tp.tp_workspace_bytes(tp.TP_WS_ATTN_CORE_BWD, M, h, 0, N)
+    assert core >= h * (M + 128) * 4          # the fp32 dQ accumulator
+    attn_b = tp.tp_workspace_bytes(tp.TP_WS_ATTN_BWD, M, h, 0, N)
+    assert attn_b >= core + 2 * M * 3 * h * 2 + 2 * M * h * 2 + N * M * h * 4
+    layer_b = tp.tp_workspace_bytes(tp.TP_WS_LAYER_BWD, M, h, F, N)
+    assert layer_b >= attn_b + 3 * M * F * 2 + 4 * M * h * 2
+    assert tp.tp_workspace_bytes(tp.TP_WS_LAYER_BWD, M, h, 0, N) == 0
+    assert tp.tp_workspace_bytes(tp.TP_WS_LN_BWD, M, h, 0, N) > 0
 
 
 def test_argument_errors_return_before_launch():
