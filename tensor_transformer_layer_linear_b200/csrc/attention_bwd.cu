@@ -13,25 +13,28 @@
 // One CTA per (shard, sequence, head, 128-key block), 12 warps:
 //   warp 0     TMA: the key block's K and V once, then the 128-query blocks'
 //              Q and dO into a 2-deep ring (128-byte swizzle), straight out
-//              of the QKV projection's [shard][token][3h/N] output and dO;
+//              of the QKV projection's [shard][token][3h/N] output and dO,
+//              and the block's lse and D into shared memory;
 //   warp 1     TMEM owner and the single MMA-issuing thread;
-//   warps 4-7  one thread per key (TMEM lane): P^T = exp2(S^T scale - lse),
-//              masked, stored as bf16 pairs over S^T in TMEM (the A operand
-//              of dV += P^T dO), and dS^T = P^T * (dP^T - D) in bf16 into a
-//              swizzled shared tile that is the K-major A operand of
-//              dK += dS^T Q and, read MN-major, the A operand of dQ = dS K;
-//   warps 8-11 one thread per query: the block's dQ from TMEM, added into an
-//              fp32 accumulator in global memory with vector reductions
-//              (every key block of the sequence contributes to it);
-//   at the end warps 4-7 write dK (scaled) and dV in bf16.
+//   warps 4-11 two threads per key (TMEM lane), each for half of the block's
+//              queries: P^T = exp2(S^T scale - lse), masked, stored as bf16
+//              pairs over S^T in TMEM (the A operand of dV += P^T dO), and
+//              dS^T = P^T * (dP^T - D) in bf16 into a swizzled shared tile
+//              that is the K-major A operand of dK += dS^T Q and, read
+//              MN-major, the A operand of dQ = dS K; warps 8-11 then drain
+//              the block's dQ from TMEM (one thread per query) into an fp32
+//              accumulator in global memory with vector reductions (every key
+//              block of the sequence contributes to it);
+//   at the end warps 4-11 write dK (scaled) and dV in bf16.
 // Per query block the MMAs are S^T = K Q^T, dP^T = V dO^T, then dV, dK and
-// dQ; dQ lands in dP^T's TMEM columns once the dQ warps have drained the
-// previous one. TMEM: S^T / P^T [0, 128), dP^T / dQ [128, 256),
-// dV [256, 384), dK [384, 512). Causal key blocks start at the diagonal
-// query block; the heaviest (first) key blocks launch first. Every barrier
-// wait is bounded; a role that gives up records an error bit and the CTA
-// leaves through the common exit after waiting (bounded) for its copies and
-// MMAs in flight.
+// dQ; dQ lands in dP^T's TMEM columns once the previous one is drained.
+// TMEM: S^T [0, 128) with P^T packed into [0, 32) and [64, 96) (each half of
+// the queries inside the columns its own threads have read), dP^T / dQ
+// [128, 256), dV [256, 384), dK [384, 512). Causal key blocks start at the
+// diagonal query block; the heaviest (first) key blocks launch first. Every
+// barrier wait is bounded; a role that gives up records an error bit and the
+// CTA leaves through the common exit after waiting (bounded) for its copies
+// and MMAs in flight.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -53,13 +56,14 @@ constexpr int AOFF_V = AOFF_K + AB_TILE;
 constexpr int AOFF_Q = AOFF_V + AB_TILE;          // 2 stages
 constexpr int AOFF_DO = AOFF_Q + 2 * AB_TILE;     // 2 stages
 constexpr int AOFF_DS = AOFF_DO + 2 * AB_TILE;
-constexpr int AOFF_BAR = AOFF_DS + AB_TILE;
+constexpr int AOFF_LD = AOFF_DS + AB_TILE;      // lse[128], D[128] of the query block
+constexpr int AOFF_BAR = AOFF_LD + 2 * AB_BQ * 4;
 constexpr int AB_NUM_BARS = 12;
 constexpr int AB_SMEM = 1024 + AOFF_BAR + AB_NUM_BARS * 8 + 16;
 static_assert(AB_SMEM <= 232448, "shared memory budget");
 
 constexpr int AB_KV = 0, AB_QFULL = 1, AB_QEMPTY = 3, AB_SDP = 5, AB_DS = 6, AB_DQFULL = 7,
-              AB_DQEMPTY = 8, AB_DONE = 9;
+              AB_DQEMPTY = 8, AB_DONE = 9, AB_LDFULL = 10;
 constexpr uint32_t TC_S = 0, TC_DP = 128, TC_DV = 256, TC_DK = 384;
 
 struct AttnBwdParams {
@@ -68,6 +72,7 @@ struct AttnBwdParams {
   long long M;   // tokens per shard
   long long stride;  // M + 128: per-head row length of lse, D and dq_acc
   float scale_log2, scale;
+  int ld_bulk;        // lse / D rows 16-byte aligned: copied by the TMA warp
   const float* lse;   // [N * hps][stride], base 2, by token
   const float* dsum;  // D, same layout
   float* dq_acc;      // [N * hps][d / 4][stride][4]
@@ -114,7 +119,8 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       mbar_init(bar(AB_QEMPTY + b), 1);
     }
     mbar_init(bar(AB_SDP), 1);
-    mbar_init(bar(AB_DS), 4);       // one arrival per key warp
+    mbar_init(bar(AB_DS), 8);       // one arrival per compute warp
+    mbar_init(bar(AB_LDFULL), 1);
     mbar_init(bar(AB_DQFULL), 1);
     mbar_init(bar(AB_DQEMPTY), 4);  // one arrival per dQ warp
     mbar_init(bar(AB_DONE), 1);
@@ -140,7 +146,9 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     tma_load_3d(s0 + AOFF_K + AB_SUB, &tm_qkv, bar(AB_KV), kcol + 64, row_base + kv0, g);
     tma_load_3d(s0 + AOFF_V, &tm_qkv, bar(AB_KV), vcol, row_base + kv0, g);
     tma_load_3d(s0 + AOFF_V + AB_SUB, &tm_qkv, bar(AB_KV), vcol + 64, row_base + kv0, g);
-    int issued = 0;
+    int issued = 0, ld_issued = 0;
+    const float* lse_h = p.lse + hb * p.stride + row_base;
+    const float* d_h = p.dsum + hb * p.stride + row_base;
     for (int it = 0; it < n_it; ++it) {
       const int st = it & 1;
       const uint32_t ph = (it >> 1) & 1;
@@ -148,7 +156,8 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         ok = false;
         break;
       }
-      const int qrow = row_base + (i_first + it) * AB_BQ;
+      const int q0 = (i_first + it) * AB_BQ;
+      const int qrow = row_base + q0;
       const uint32_t qd = s0 + AOFF_Q + st * AB_TILE, dd = s0 + AOFF_DO + st * AB_TILE;
       mbar_arrive_expect_tx(bar(AB_QFULL + st), 2 * AB_TILE);
       tma_load_3d(qd, &tm_qkv, bar(AB_QFULL + st), head * AB_D, qrow, g);
@@ -156,6 +165,18 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       tma_load_3d(dd, &tm_do, bar(AB_QFULL + st), head * AB_D, qrow, g);
       tma_load_3d(dd + AB_SUB, &tm_do, bar(AB_QFULL + st), head * AB_D + 64, qrow, g);
       ++issued;
+      if (p.ld_bulk) {
+        // the single lse / D buffer is free once the compute warps are done
+        // with the previous query block
+        if (it > 0 && !mbar_wait(bar(AB_DS), (it - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(AB_LDFULL), 2 * AB_BQ * 4);
+        bulk_load(s0 + AOFF_LD, lse_h + q0, AB_BQ * 4, bar(AB_LDFULL));
+        bulk_load(s0 + AOFF_LD + AB_BQ * 4, d_h + q0, AB_BQ * 4, bar(AB_LDFULL));
+        ++ld_issued;
+      }
     }
     if (!ok) {
       atomicOr(p.err, ERR_WAIT_ATTN);
@@ -167,6 +188,8 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     for (int ii = (issued >= 2 ? issued - 2 : 0); ii < issued; ++ii)
       if (!mbar_wait(bar(AB_QFULL + (ii & 1)), (ii >> 1) & 1, &never))
         atomicOr(p.err, ERR_WAIT_DRAIN);
+    if (ld_issued > 0 && !mbar_wait(bar(AB_LDFULL), (ld_issued - 1) & 1, &never))
+      atomicOr(p.err, ERR_WAIT_DRAIN);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA
     constexpr uint32_t idesc_kk = umma_idesc_bf16_f32(AB_BK, AB_BQ);        // A, B K-major
@@ -213,7 +236,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       // dV += P^T dO (P^T from TMEM, contraction over queries)
 #pragma unroll
       for (int kk = 0; kk < AB_BQ / 16; ++kk)
-        umma_bf16_tmem_a(tmem + TC_DV, tmem + TC_S + kk * 8,
+        umma_bf16_tmem_a(tmem + TC_DV, tmem + TC_S + kk * 8 + (kk >= 4 ? 32 : 0),
                          umma_desc_sw128_mn(sdO + kk * 2048, AB_SUB), idesc_kmn,
                          (it > 0 || kk > 0) ? 1u : 0u);
       // dK += dS^T Q
@@ -238,19 +261,24 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     umma_commit(bar(AB_DONE));
     int never = 0;
     if (!mbar_wait(bar(AB_DONE), 0, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ P^T, dS^T
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ P^T, dS^T, dQ
     const int rq = warp & 3;
-    const int row = rq * 32 + lane;  // key within the block (= TMEM lane)
+    const int grp = (warp - 4) >> 2;  // which half of the block's queries
+    const int row = rq * 32 + lane;   // key within the block (= TMEM lane)
     const int key = kv0 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(rq * 32) << 16;
     const float sl2 = p.scale_log2;
     const float* lse_h = p.lse + hb * p.stride + row_base;
     const float* d_h = p.dsum + hb * p.stride + row_base;
+    const float* s_lse = reinterpret_cast<const float*>(sm + AOFF_LD);
+    const float* s_d = s_lse + AB_BQ;
     const uint32_t ds_row = s0 + AOFF_DS + static_cast<uint32_t>(row) * 128u;
+    float* acc_h = p.dq_acc + hb * (static_cast<int64_t>(AB_D) * p.stride) + row_base * 4LL;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      if (!mbar_wait(bar(AB_SDP), it & 1, abort_flag)) {
+      if (!mbar_wait(bar(AB_SDP), it & 1, abort_flag) ||
+          (p.ld_bulk && !mbar_wait(bar(AB_LDFULL), it & 1, abort_flag))) {
         ok = false;
         break;
       }
@@ -259,12 +287,8 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       const int q0 = i * AB_BQ;
       const bool need_mask =
           (p.causal && i == j) || q0 + AB_BQ > p.seq || kv0 + AB_BK > p.seq;
-      // lse and D of the block's queries are read by every key thread
-      // (broadcast loads; rows past the sequence read whatever follows, and
-      // those queries are masked); 16-byte loads when the row is aligned
-      const bool al4 = ((hb * p.stride + row_base + q0) & 3) == 0;
 #pragma unroll 1
-      for (int c = 0; c < AB_BQ / 32; ++c) {
+      for (int c = 2 * grp; c < 2 * grp + 2; ++c) {
         uint32_t sv[32], dv[32];
         tmem_ld_32x32b_x32(tmem + lane_addr + TC_S + c * 32, sv);
         tmem_ld_32x32b_x32(tmem + lane_addr + TC_DP + c * 32, dv);
@@ -272,25 +296,23 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          float lq[4], dq[4];
-          const float* lp = lse_h + q0 + c * 32 + e;
-          const float* dp = d_h + q0 + c * 32 + e;
-          if (al4) {
-            const float4 l4 = __ldg(reinterpret_cast<const float4*>(lp));
-            const float4 d4 = __ldg(reinterpret_cast<const float4*>(dp));
-            lq[0] = l4.x; lq[1] = l4.y; lq[2] = l4.z; lq[3] = l4.w;
-            dq[0] = d4.x; dq[1] = d4.y; dq[2] = d4.z; dq[3] = d4.w;
+          // lse and D of these 4 queries: the same for every key thread
+          float4 l4, d4;
+          if (p.ld_bulk) {
+            l4 = *reinterpret_cast<const float4*>(s_lse + c * 32 + e);
+            d4 = *reinterpret_cast<const float4*>(s_d + c * 32 + e);
           } else {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              lq[u] = __ldg(lp + u);
-              dq[u] = __ldg(dp + u);
-            }
+            const float* lp = lse_h + q0 + c * 32 + e;
+            const float* dp = d_h + q0 + c * 32 + e;
+            l4 = make_float4(__ldg(lp), __ldg(lp + 1), __ldg(lp + 2), __ldg(lp + 3));
+            d4 = make_float4(__ldg(dp), __ldg(dp + 1), __ldg(dp + 2), __ldg(dp + 3));
           }
+          const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
+          const float dq[4] = {d4.x, d4.y, d4.z, d4.w};
           float pp[4], ds[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const float pv = exp2f(fmaf(__uint_as_float(sv[e + u]), sl2, -lq[u]));
+            const float pv = ex2_approx(fmaf(__uint_as_float(sv[e + u]), sl2, -lq[u]));
             const float dsv = pv * (__uint_as_float(dv[e + u]) - dq[u]);
             if (need_mask) {
               const int q = q0 + c * 32 + e + u;
@@ -307,8 +329,9 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
           dk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
           dk[(e >> 1) + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        // P^T chunk c over columns [16 c, 16 c + 16) of S^T (already read)
-        tmem_st_32x32b_x16(tmem + lane_addr + TC_S + c * 16, pk);
+        // P^T of queries [32 c, 32 c + 32) into 16 columns this thread has
+        // already read: [16 c, 16 c + 16) + 32 for the second half
+        tmem_st_32x32b_x16(tmem + lane_addr + TC_S + c * 16 + grp * 32, pk);
         // dS^T row `row`, queries [32 c, 32 c + 32): 128-byte swizzled rows,
         // queries 0-63 in the first 16 KB half, 64-127 in the second
         const uint32_t half = ds_row + static_cast<uint32_t>(c >> 1) * AB_SUB;
@@ -324,6 +347,31 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(AB_DS));
+      if (grp == 1) {
+        // drain this block's dQ (one thread per query = TMEM lane)
+        if (!mbar_wait(bar(AB_DQFULL), it & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t v[AB_D];
+#pragma unroll
+        for (int c = 0; c < AB_D / 32; ++c)
+          tmem_ld_32x32b_x32(tmem + lane_addr + TC_DP + c * 32, &v[c * 32]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(AB_DQEMPTY));  // the columns may be overwritten now
+        const int q = q0 + row;
+        if (q < p.seq) {
+          // layout [d / 4][stride][4]: a warp's 32 queries are 512 contiguous bytes
+          float* a = acc_h + static_cast<int64_t>(q) * 4;
+#pragma unroll
+          for (int u = 0; u < AB_D / 4; ++u)
+            red_add_v4(a + static_cast<int64_t>(u) * p.stride * 4, v[4 * u], v[4 * u + 1],
+                       v[4 * u + 2], v[4 * u + 3]);
+        }
+      }
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
@@ -331,11 +379,11 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     } else if (mbar_wait(bar(AB_DONE), 0, abort_flag)) {
       tc_fence_after();
       // tcgen05.ld is warp-collective: every lane loads, only rows inside
-      // the sequence are stored
+      // the sequence are stored; each group writes half of the 128 columns
       uint16_t* base = p.dqkv + (static_cast<int64_t>(g) * p.M + row_base + key) * (3 * p.hs) +
                        head * AB_D;
 #pragma unroll 1
-      for (int c = 0; c < AB_D / 32; ++c) {
+      for (int c = 2 * grp; c < 2 * grp + 2; ++c) {
         uint32_t kv[32], vv[32];
         tmem_ld_32x32b_x32(tmem + lane_addr + TC_DK + c * 32, kv);
         tmem_ld_32x32b_x32(tmem + lane_addr + TC_DV + c * 32, vv);
@@ -362,40 +410,6 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         }
       }
     } else {
-      if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
-      *abort_flag = 1;
-    }
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ dQ
-    const int rq = warp & 3;
-    const int row = rq * 32 + lane;  // query within the block (= TMEM lane)
-    const uint32_t lane_addr = static_cast<uint32_t>(rq * 32) << 16;
-    float* acc_h = p.dq_acc + hb * (static_cast<int64_t>(AB_D) * p.stride) + row_base * 4LL;
-    bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      if (!mbar_wait(bar(AB_DQFULL), it & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t v[AB_D];
-#pragma unroll
-      for (int c = 0; c < AB_D / 32; ++c) tmem_ld_32x32b_x32(tmem + lane_addr + TC_DP + c * 32, &v[c * 32]);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(AB_DQEMPTY));  // the columns may be overwritten now
-      const int q = (i_first + it) * AB_BQ + row;
-      if (q < p.seq) {
-        // layout [d / 4][stride][4]: a warp's 32 queries are 512 contiguous bytes
-        float* a = acc_h + static_cast<int64_t>(q) * 4;
-#pragma unroll
-        for (int u = 0; u < AB_D / 4; ++u)
-          red_add_v4(a + static_cast<int64_t>(u) * p.stride * 4, v[4 * u], v[4 * u + 1],
-                     v[4 * u + 2], v[4 * u + 3]);
-      }
-    }
-    if (!ok) {
       if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
       *abort_flag = 1;
     }
@@ -531,6 +545,7 @@ int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const f
   p.stride = stride;
   p.scale = 1.0f / sqrtf(static_cast<float>(AB_D));
   p.scale_log2 = 1.4426950408889634f * p.scale;
+  p.ld_bulk = (M % 4 == 0 && seq % 4 == 0) ? 1 : 0;  // 16-byte aligned lse / D rows
   p.lse = lse;
   p.dsum = dsum;
   p.dq_acc = dq_acc;

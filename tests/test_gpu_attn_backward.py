@@ -56,7 +56,7 @@ def _core_case(tp, rng, n, batch, seq, h, causal, q_std=1.0):
 
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("n,batch,seq,h", [(1, 2, 128, 256), (2, 2, 200, 512), (2, 1, 384, 256),
-                                           (4, 3, 136, 512)])
+                                           (4, 3, 136, 512), (2, 3, 130, 256)])
 def test_attention_backward_parity(tp, n, batch, seq, h, causal):
     rng = np.random.default_rng(1000 + n * 7 + seq + int(causal))
     hs = h // n
