@@ -10,31 +10,36 @@
 //   dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d),
 // where P is rebuilt from the forward's log-sum-exp.
 //
-// One CTA per (shard, sequence, head, 128-key block), 12 warps:
-//   warp 0     TMA: the key block's K and V once, then the 128-query blocks'
-//              Q and dO into a 2-deep ring (128-byte swizzle), straight out
-//              of the QKV projection's [shard][token][3h/N] output and dO,
-//              and the block's lse and D into shared memory;
+// One CTA per (shard, sequence, head, 128-key block), 16 warps, stepping
+// through the sequence's 64-query blocks:
+//   warp 0     TMA: the key block's K and V once, then each query block's Q
+//              and dO into a 4-deep ring (128-byte swizzle), straight out of
+//              the QKV projection's [shard][token][3h/N] output and dO, and
+//              its lse and D into a 2-deep shared ring (bulk copies when the
+//              rows are 16-byte aligned);
 //   warp 1     TMEM owner and the single MMA-issuing thread;
-//   warps 4-11 two threads per key (TMEM lane), each for half of the block's
+//   warps 4-7, 12-15
+//              two threads per key (TMEM lane), each for 32 of the block's 64
 //              queries: P^T = exp2(S^T scale - lse), masked, stored as bf16
-//              pairs over S^T in TMEM (the A operand of dV += P^T dO), and
-//              dS^T = P^T * (dP^T - D) in bf16 into a swizzled shared tile
-//              that is the K-major A operand of dK += dS^T Q and, read
-//              MN-major, the A operand of dQ = dS K; warps 8-11 then drain
-//              the block's dQ from TMEM (one thread per query) into an fp32
-//              accumulator in global memory with vector reductions (every key
-//              block of the sequence contributes to it);
-//   at the end warps 4-11 write dK (scaled) and dV in bf16.
-// Per query block the MMAs are S^T = K Q^T, dP^T = V dO^T, then dV, dK and
-// dQ; dQ lands in dP^T's TMEM columns once the previous one is drained.
-// TMEM: S^T [0, 128) with P^T packed into [0, 32) and [64, 96) (each half of
-// the queries inside the columns its own threads have read), dP^T / dQ
-// [128, 256), dV [256, 384), dK [384, 512). Causal key blocks start at the
-// diagonal query block; the heaviest (first) key blocks launch first. Every
-// barrier wait is bounded; a role that gives up records an error bit and the
-// CTA leaves through the common exit after waiting (bounded) for its copies
-// and MMAs in flight.
+//              pairs over the S^T columns the thread has read (the A operand
+//              of dV += P^T dO), and dS^T = P^T * (dP^T - D) in bf16 into a
+//              swizzled shared tile, the K-major A operand of dK += dS^T Q
+//              and the MN-major B operand of dQ^T = K^T dS^T; at the end they
+//              write dK (scaled) and dV in bf16, half of the columns each;
+//   warps 8-11 one thread per head-dimension column (TMEM lane): drain the
+//              block's dQ^T from TMEM into an fp32 accumulator in global
+//              memory with reductions (every key block of the sequence
+//              contributes to it).
+// S^T and dP^T are double-buffered in TMEM, so the tensor cores compute the
+// next block's S^T = K Q^T and dP^T = V dO^T while the key threads work on
+// the current one; dQ^T of a block lands in that block's dP^T columns once
+// they are read. TMEM: buffer b in [128 b, 128 b + 128) (S^T, then P^T in its
+// columns [0, 16) and [32, 48); dP^T, then dQ^T, in its last 64), dV
+// [256, 384), dK [384, 512). Causal key blocks start at the first query block that sees
+// them; the heaviest (first) key blocks launch first. Every barrier wait is
+// bounded; a role that gives up records an error bit and the CTA leaves
+// through the common exit after waiting (bounded) for its copies and MMAs in
+// flight.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -46,25 +51,36 @@
 namespace tpk {
 
 constexpr int AB_BK = 128;        // keys per CTA
-constexpr int AB_BQ = 128;        // queries per step
+constexpr int AB_BQ = 64;         // queries per step
 constexpr int AB_D = 128;         // head dim
-constexpr int AB_THREADS = 384;
-constexpr int AB_SUB = 128 * 128;          // [128 rows][64 cols] bf16: 16 KB
-constexpr int AB_TILE = 2 * AB_SUB;        // [128][128] bf16: 32 KB
+constexpr int AB_THREADS = 512;
+constexpr int AB_NST = 4;         // Q / dO ring depth
+constexpr int AB_KSUB = 128 * 128;          // [128 rows][64 cols] bf16: 16 KB
+constexpr int AB_KTILE = 2 * AB_KSUB;       // [128][128] bf16: K or V
+constexpr int AB_QSUB = 64 * 128;           // [64 rows][64 cols] bf16: 8 KB
+constexpr int AB_QTILE = 2 * AB_QSUB;       // [64][128] bf16: Q or dO block
+constexpr int AB_DSTILE = 128 * 128;        // dS^T [128 keys][64 queries] bf16: 16 KB
 constexpr int AOFF_K = 0;
-constexpr int AOFF_V = AOFF_K + AB_TILE;
-constexpr int AOFF_Q = AOFF_V + AB_TILE;          // 2 stages
-constexpr int AOFF_DO = AOFF_Q + 2 * AB_TILE;     // 2 stages
-constexpr int AOFF_DS = AOFF_DO + 2 * AB_TILE;
-constexpr int AOFF_LD = AOFF_DS + AB_TILE;      // lse[128], D[128] of the query block
-constexpr int AOFF_BAR = AOFF_LD + 2 * AB_BQ * 4;
-constexpr int AB_NUM_BARS = 12;
+constexpr int AOFF_V = AOFF_K + AB_KTILE;
+constexpr int AOFF_Q = AOFF_V + AB_KTILE;              // AB_NST stages
+constexpr int AOFF_DO = AOFF_Q + AB_NST * AB_QTILE;    // AB_NST stages
+constexpr int AOFF_DS = AOFF_DO + AB_NST * AB_QTILE;   // 2 buffers
+constexpr int AOFF_LD = AOFF_DS + 2 * AB_DSTILE;       // 2 x (lse[64], D[64])
+constexpr int AOFF_BAR = AOFF_LD + 2 * 2 * AB_BQ * 4;
+constexpr int AB_NUM_BARS = 24;
 constexpr int AB_SMEM = 1024 + AOFF_BAR + AB_NUM_BARS * 8 + 16;
 static_assert(AB_SMEM <= 232448, "shared memory budget");
 
-constexpr int AB_KV = 0, AB_QFULL = 1, AB_QEMPTY = 3, AB_SDP = 5, AB_DS = 6, AB_DQFULL = 7,
-              AB_DQEMPTY = 8, AB_DONE = 9, AB_LDFULL = 10;
-constexpr uint32_t TC_S = 0, TC_DP = 128, TC_DV = 256, TC_DK = 384;
+// barriers
+constexpr int AB_KV = 0, AB_QFULL = 1, AB_QEMPTY = AB_QFULL + AB_NST,
+              AB_SDP = AB_QEMPTY + AB_NST,     // 2: S^T and dP^T of buffer b computed
+              AB_DS = AB_SDP + 2,              // 2: key threads done with buffer b
+              AB_DQFULL = AB_DS + 2,           // 2: dQ^T in buffer b (and dK, dV done)
+              AB_DQEMPTY = AB_DQFULL + 2,      // 2: dQ^T of buffer b drained
+              AB_LDFULL = AB_DQEMPTY + 2,      // 2: lse / D stage loaded
+              AB_LDEMPTY = AB_LDFULL + 2,      // 2: lse / D stage read
+              AB_DONE = AB_LDEMPTY + 2;
+static_assert(AB_DONE < AB_NUM_BARS, "barrier count");
 
 struct AttnBwdParams {
   int seq, batch, hps, causal, nq;
@@ -75,20 +91,18 @@ struct AttnBwdParams {
   int ld_bulk;        // lse / D rows 16-byte aligned: copied by the TMA warp
   const float* lse;   // [N * hps][stride], base 2, by token
   const float* dsum;  // D, same layout
-  float* dq_acc;      // [N * hps][d / 4][stride][4]
+  float* dq_acc;      // [N * hps][stride][128] fp32
   uint16_t* dqkv;     // [N][M][3 hs]
   unsigned* err;
 };
 
-__device__ __forceinline__ void red_add_v4(float* addr, uint32_t a, uint32_t b, uint32_t c,
-                                           uint32_t d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(__uint_as_float(a)),
-               "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
-               : "memory");
+__device__ __forceinline__ void red_add_f32(float* addr, uint32_t v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(__uint_as_float(v)) : "memory");
 }
 
 __global__ void __launch_bounds__(AB_THREADS, 1)
-    attention_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv,
+    attention_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
+                            const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_do, const AttnBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -108,27 +122,32 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
   const int j = blockIdx.y;  // key block
   const int kv0 = j * AB_BK;
   const int row_base = sidx * p.seq;
-  const int i_first = p.causal ? j : 0;  // query blocks that see this key block
+  // first query block that sees a key of this block (causal: queries >= kv0)
+  const int i_first = p.causal ? kv0 / AB_BQ : 0;
   const int n_it = p.nq - i_first;
   const int64_t hb = static_cast<int64_t>(g) * p.hps + head;  // (shard, head)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(AB_KV), 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(AB_QFULL + b), 1);
-      mbar_init(bar(AB_QEMPTY + b), 1);
+    for (int s = 0; s < AB_NST; ++s) {
+      mbar_init(bar(AB_QFULL + s), 1);
+      mbar_init(bar(AB_QEMPTY + s), 1);
     }
-    mbar_init(bar(AB_SDP), 1);
-    mbar_init(bar(AB_DS), 8);       // one arrival per compute warp
-    mbar_init(bar(AB_LDFULL), 1);
-    mbar_init(bar(AB_DQFULL), 1);
-    mbar_init(bar(AB_DQEMPTY), 4);  // one arrival per dQ warp
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(AB_SDP + b), 1);
+      mbar_init(bar(AB_DS + b), 8);       // one arrival per key warp
+      mbar_init(bar(AB_DQFULL + b), 1);
+      mbar_init(bar(AB_DQEMPTY + b), 4);  // one arrival per drain warp
+      mbar_init(bar(AB_LDFULL + b), 1);
+      mbar_init(bar(AB_LDEMPTY + b), 8);  // one arrival per key warp
+    }
     mbar_init(bar(AB_DONE), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_qkv);
+    tma_prefetch_desc(&tm_kv);
+    tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_do);
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_holder), 512);
@@ -141,40 +160,40 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     // ------------------------------------------------------------ TMA
     bool ok = true;
     const int kcol = p.hs + head * AB_D, vcol = 2 * p.hs + head * AB_D;
-    mbar_arrive_expect_tx(bar(AB_KV), 2 * AB_TILE);
-    tma_load_3d(s0 + AOFF_K, &tm_qkv, bar(AB_KV), kcol, row_base + kv0, g);
-    tma_load_3d(s0 + AOFF_K + AB_SUB, &tm_qkv, bar(AB_KV), kcol + 64, row_base + kv0, g);
-    tma_load_3d(s0 + AOFF_V, &tm_qkv, bar(AB_KV), vcol, row_base + kv0, g);
-    tma_load_3d(s0 + AOFF_V + AB_SUB, &tm_qkv, bar(AB_KV), vcol + 64, row_base + kv0, g);
-    int issued = 0, ld_issued = 0;
+    mbar_arrive_expect_tx(bar(AB_KV), 2 * AB_KTILE);
+    tma_load_3d(s0 + AOFF_K, &tm_kv, bar(AB_KV), kcol, row_base + kv0, g);
+    tma_load_3d(s0 + AOFF_K + AB_KSUB, &tm_kv, bar(AB_KV), kcol + 64, row_base + kv0, g);
+    tma_load_3d(s0 + AOFF_V, &tm_kv, bar(AB_KV), vcol, row_base + kv0, g);
+    tma_load_3d(s0 + AOFF_V + AB_KSUB, &tm_kv, bar(AB_KV), vcol + 64, row_base + kv0, g);
     const float* lse_h = p.lse + hb * p.stride + row_base;
     const float* d_h = p.dsum + hb * p.stride + row_base;
+    int issued = 0, ld_issued = 0;
     for (int it = 0; it < n_it; ++it) {
-      const int st = it & 1;
-      const uint32_t ph = (it >> 1) & 1;
+      const int st = it % AB_NST;
+      const uint32_t ph = (it / AB_NST) & 1;
       if (!mbar_wait(bar(AB_QEMPTY + st), ph ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
       const int q0 = (i_first + it) * AB_BQ;
       const int qrow = row_base + q0;
-      const uint32_t qd = s0 + AOFF_Q + st * AB_TILE, dd = s0 + AOFF_DO + st * AB_TILE;
-      mbar_arrive_expect_tx(bar(AB_QFULL + st), 2 * AB_TILE);
-      tma_load_3d(qd, &tm_qkv, bar(AB_QFULL + st), head * AB_D, qrow, g);
-      tma_load_3d(qd + AB_SUB, &tm_qkv, bar(AB_QFULL + st), head * AB_D + 64, qrow, g);
+      const uint32_t qd = s0 + AOFF_Q + st * AB_QTILE, dd = s0 + AOFF_DO + st * AB_QTILE;
+      mbar_arrive_expect_tx(bar(AB_QFULL + st), 2 * AB_QTILE);
+      tma_load_3d(qd, &tm_q, bar(AB_QFULL + st), head * AB_D, qrow, g);
+      tma_load_3d(qd + AB_QSUB, &tm_q, bar(AB_QFULL + st), head * AB_D + 64, qrow, g);
       tma_load_3d(dd, &tm_do, bar(AB_QFULL + st), head * AB_D, qrow, g);
-      tma_load_3d(dd + AB_SUB, &tm_do, bar(AB_QFULL + st), head * AB_D + 64, qrow, g);
+      tma_load_3d(dd + AB_QSUB, &tm_do, bar(AB_QFULL + st), head * AB_D + 64, qrow, g);
       ++issued;
       if (p.ld_bulk) {
-        // the single lse / D buffer is free once the compute warps are done
-        // with the previous query block
-        if (it > 0 && !mbar_wait(bar(AB_DS), (it - 1) & 1, abort_flag)) {
+        const int ls = it & 1;
+        if (!mbar_wait(bar(AB_LDEMPTY + ls), ((it >> 1) & 1) ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(AB_LDFULL), 2 * AB_BQ * 4);
-        bulk_load(s0 + AOFF_LD, lse_h + q0, AB_BQ * 4, bar(AB_LDFULL));
-        bulk_load(s0 + AOFF_LD + AB_BQ * 4, d_h + q0, AB_BQ * 4, bar(AB_LDFULL));
+        const uint32_t ld = s0 + AOFF_LD + ls * (2 * AB_BQ * 4);
+        mbar_arrive_expect_tx(bar(AB_LDFULL + ls), 2 * AB_BQ * 4);
+        bulk_load(ld, lse_h + q0, AB_BQ * 4, bar(AB_LDFULL + ls));
+        bulk_load(ld + AB_BQ * 4, d_h + q0, AB_BQ * 4, bar(AB_LDFULL + ls));
         ++ld_issued;
       }
     }
@@ -185,72 +204,78 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     // every load issued must land before the CTA exits
     int never = 0;
     if (!mbar_wait(bar(AB_KV), 0, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
-    for (int ii = (issued >= 2 ? issued - 2 : 0); ii < issued; ++ii)
-      if (!mbar_wait(bar(AB_QFULL + (ii & 1)), (ii >> 1) & 1, &never))
+    for (int ii = (issued >= AB_NST ? issued - AB_NST : 0); ii < issued; ++ii)
+      if (!mbar_wait(bar(AB_QFULL + ii % AB_NST), (ii / AB_NST) & 1, &never))
         atomicOr(p.err, ERR_WAIT_DRAIN);
-    if (ld_issued > 0 && !mbar_wait(bar(AB_LDFULL), (ld_issued - 1) & 1, &never))
-      atomicOr(p.err, ERR_WAIT_DRAIN);
+    for (int ii = (ld_issued >= 2 ? ld_issued - 2 : 0); ii < ld_issued; ++ii)
+      if (!mbar_wait(bar(AB_LDFULL + (ii & 1)), (ii >> 1) & 1, &never))
+        atomicOr(p.err, ERR_WAIT_DRAIN);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA
-    constexpr uint32_t idesc_kk = umma_idesc_bf16_f32(AB_BK, AB_BQ);        // A, B K-major
-    constexpr uint32_t idesc_kmn = umma_idesc_bf16_f32_bmn(AB_BK, AB_D);    // B MN-major
-    constexpr uint32_t idesc_mnmn = idesc_kmn | (1u << 15);                 // A, B MN-major
-    const uint32_t sK = s0 + AOFF_K, sV = s0 + AOFF_V, sDS = s0 + AOFF_DS;
+    constexpr uint32_t idesc_s = umma_idesc_bf16_f32(AB_BK, AB_BQ);          // A, B K-major
+    constexpr uint32_t idesc_kmn = umma_idesc_bf16_f32_bmn(AB_BK, AB_D);     // B MN-major
+    constexpr uint32_t idesc_dq =
+        umma_idesc_bf16_f32_bmn(AB_D, AB_BQ) | (1u << 15);                   // A, B MN-major
+    const uint32_t sK = s0 + AOFF_K, sV = s0 + AOFF_V;
+    // S^T and dP^T of query block k into buffer k & 1
+    auto issue_sdp = [&](int k) -> bool {
+      const int st = k % AB_NST, b = k & 1;
+      if (!mbar_wait(bar(AB_QFULL + st), (k / AB_NST) & 1, abort_flag)) return false;
+      // the buffer's dQ^T of block k - 2 must be drained (its S^T / P^T and
+      // dP^T were consumed before that dQ^T was computed)
+      if (k >= 2 && !mbar_wait(bar(AB_DQEMPTY + b), ((k - 2) >> 1) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sQ = s0 + AOFF_Q + st * AB_QTILE, sdO = s0 + AOFF_DO + st * AB_QTILE;
+      const uint32_t tS = tmem + 128u * b, tP = tS + 64u;
+#pragma unroll
+      for (int kk = 0; kk < AB_D / 16; ++kk) {   // contraction over d
+        const uint32_t ka = (kk >> 2) * AB_KSUB + (kk & 3) * 32;
+        const uint32_t qa = (kk >> 2) * AB_QSUB + (kk & 3) * 32;
+        umma_bf16(tS, umma_desc_sw128(sK + ka), umma_desc_sw128(sQ + qa), idesc_s, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < AB_D / 16; ++kk) {
+        const uint32_t ka = (kk >> 2) * AB_KSUB + (kk & 3) * 32;
+        const uint32_t qa = (kk >> 2) * AB_QSUB + (kk & 3) * 32;
+        umma_bf16(tP, umma_desc_sw128(sV + ka), umma_desc_sw128(sdO + qa), idesc_s, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(bar(AB_SDP + b));
+      return true;
+    };
     bool ok = mbar_wait(bar(AB_KV), 0, abort_flag);
+    if (ok && n_it > 0) ok = issue_sdp(0);
     for (int it = 0; ok && it < n_it; ++it) {
-      const int st = it & 1;
-      const uint32_t ph = (it >> 1) & 1;
-      if (!mbar_wait(bar(AB_QFULL + st), ph, abort_flag)) {
+      const int st = it % AB_NST, b = it & 1;
+      if (it + 1 < n_it && !issue_sdp(it + 1)) {
+        ok = false;
+        break;
+      }
+      if (!mbar_wait(bar(AB_DS + b), (it >> 1) & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t sQ = s0 + AOFF_Q + st * AB_TILE, sdO = s0 + AOFF_DO + st * AB_TILE;
-      // S^T = K Q^T: rows = keys, columns = queries, contraction over d
-#pragma unroll
-      for (int kk = 0; kk < AB_D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * AB_SUB + (kk & 3) * 32;
-        umma_bf16(tmem + TC_S, umma_desc_sw128(sK + off), umma_desc_sw128(sQ + off), idesc_kk,
-                  kk > 0 ? 1u : 0u);
-      }
-      // dP^T = V dO^T, into the columns the previous dQ occupied
-      if (it > 0) {
-        if (!mbar_wait(bar(AB_DQEMPTY), (it - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-      }
-#pragma unroll
-      for (int kk = 0; kk < AB_D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * AB_SUB + (kk & 3) * 32;
-        umma_bf16(tmem + TC_DP, umma_desc_sw128(sV + off), umma_desc_sw128(sdO + off), idesc_kk,
-                  kk > 0 ? 1u : 0u);
-      }
-      umma_commit(bar(AB_SDP));
-      if (!mbar_wait(bar(AB_DS), it & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // dV += P^T dO (P^T from TMEM, contraction over queries)
+      const uint32_t sQ = s0 + AOFF_Q + st * AB_QTILE, sdO = s0 + AOFF_DO + st * AB_QTILE;
+      const uint32_t sDS = s0 + AOFF_DS + b * AB_DSTILE;
+      const uint32_t tS = tmem + 128u * b, tP = tS + 64u;
+      // dV += P^T dO: P^T (keys x queries, bf16 pairs) from TMEM
 #pragma unroll
       for (int kk = 0; kk < AB_BQ / 16; ++kk)
-        umma_bf16_tmem_a(tmem + TC_DV, tmem + TC_S + kk * 8 + (kk >= 4 ? 32 : 0),
-                         umma_desc_sw128_mn(sdO + kk * 2048, AB_SUB), idesc_kmn,
-                         (it > 0 || kk > 0) ? 1u : 0u);
+        umma_bf16_tmem_a(tmem + 256u, tS + kk * 8 + (kk >= 2 ? 16 : 0),
+                         umma_desc_sw128_mn(sdO + kk * 2048, AB_QSUB),
+                         idesc_kmn, (it > 0 || kk > 0) ? 1u : 0u);
       // dK += dS^T Q
 #pragma unroll
       for (int kk = 0; kk < AB_BQ / 16; ++kk)
-        umma_bf16(tmem + TC_DK, umma_desc_sw128(sDS + (kk >> 2) * AB_SUB + (kk & 3) * 32),
-                  umma_desc_sw128_mn(sQ + kk * 2048, AB_SUB), idesc_kmn,
+        umma_bf16(tmem + 384u, umma_desc_sw128(sDS + kk * 32),
+                  umma_desc_sw128_mn(sQ + kk * 2048, AB_QSUB), idesc_kmn,
                   (it > 0 || kk > 0) ? 1u : 0u);
-      // dQ = dS K (dS read MN-major from the same tile; contraction over keys)
+      // dQ^T = K^T dS^T (head dim x queries), contraction over the keys
 #pragma unroll
       for (int kk = 0; kk < AB_BK / 16; ++kk)
-        umma_bf16(tmem + TC_DP, umma_desc_sw128_mn(sDS + kk * 2048, AB_SUB),
-                  umma_desc_sw128_mn(sK + kk * 2048, AB_SUB), idesc_mnmn, kk > 0 ? 1u : 0u);
-      umma_commit(bar(AB_DQFULL));
+        umma_bf16(tP, umma_desc_sw128_mn(sK + kk * 2048, AB_KSUB),
+                  umma_desc_sw128_mn(sDS + kk * 2048, AB_QSUB), idesc_dq, kk > 0 ? 1u : 0u);
+      umma_commit(bar(AB_DQFULL + b));
       umma_commit(bar(AB_QEMPTY + st));
     }
     if (!ok) {
@@ -261,24 +286,23 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     umma_commit(bar(AB_DONE));
     int never = 0;
     if (!mbar_wait(bar(AB_DONE), 0, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ P^T, dS^T, dQ
+  } else if ((warp >= 4 && warp < 8) || warp >= 12) {
+    // ------------------------------------------------------------ P^T, dS^T
     const int rq = warp & 3;
-    const int grp = (warp - 4) >> 2;  // which half of the block's queries
-    const int row = rq * 32 + lane;   // key within the block (= TMEM lane)
+    const int grp = warp >= 12 ? 1 : 0;  // queries [32 grp, 32 grp + 32) of each block
+    const int row = rq * 32 + lane;      // key within the block (= TMEM lane)
     const int key = kv0 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(rq * 32) << 16;
     const float sl2 = p.scale_log2;
     const float* lse_h = p.lse + hb * p.stride + row_base;
     const float* d_h = p.dsum + hb * p.stride + row_base;
-    const float* s_lse = reinterpret_cast<const float*>(sm + AOFF_LD);
-    const float* s_d = s_lse + AB_BQ;
-    const uint32_t ds_row = s0 + AOFF_DS + static_cast<uint32_t>(row) * 128u;
-    float* acc_h = p.dq_acc + hb * (static_cast<int64_t>(AB_D) * p.stride) + row_base * 4LL;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      if (!mbar_wait(bar(AB_SDP), it & 1, abort_flag) ||
-          (p.ld_bulk && !mbar_wait(bar(AB_LDFULL), it & 1, abort_flag))) {
+      const int b = it & 1;
+      if (!mbar_wait(bar(AB_SDP + b), (it >> 1) & 1, abort_flag) ||
+          (p.ld_bulk && !mbar_wait(bar(AB_LDFULL + b), (it >> 1) & 1, abort_flag)) ||
+          // dS^T buffer b is free once dK and dQ^T of block it - 2 are done
+          (it >= 2 && !mbar_wait(bar(AB_DQFULL + b), ((it - 2) >> 1) & 1, abort_flag))) {
         ok = false;
         break;
       }
@@ -286,24 +310,28 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       const int i = i_first + it;
       const int q0 = i * AB_BQ;
       const bool need_mask =
-          (p.causal && i == j) || q0 + AB_BQ > p.seq || kv0 + AB_BK > p.seq;
+          (p.causal && q0 < kv0 + AB_BK) || q0 + AB_BQ > p.seq || kv0 + AB_BK > p.seq;
+      const uint32_t tS = tmem + lane_addr + 128u * b, tP = tS + 64u;
+      const float* s_lse = reinterpret_cast<const float*>(sm + AOFF_LD + b * (2 * AB_BQ * 4));
+      const float* s_d = s_lse + AB_BQ;
+      const uint32_t ds_row = s0 + AOFF_DS + b * AB_DSTILE + static_cast<uint32_t>(row) * 128u;
 #pragma unroll 1
-      for (int c = 2 * grp; c < 2 * grp + 2; ++c) {
-        uint32_t sv[32], dv[32];
-        tmem_ld_32x32b_x32(tmem + lane_addr + TC_S + c * 32, sv);
-        tmem_ld_32x32b_x32(tmem + lane_addr + TC_DP + c * 32, dv);
+      for (int c = 2 * grp; c < 2 * grp + 2; ++c) {  // 16 queries at a time
+        uint32_t sv[16], dv[16];
+        tmem_ld_32x32b_x16(tS + c * 16, sv);
+        tmem_ld_32x32b_x16(tP + c * 16, dv);
         tmem_ld_wait();
-        uint32_t pk[16], dk[16];
+        uint32_t pk[8], dk[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
+        for (int e = 0; e < 16; e += 4) {
           // lse and D of these 4 queries: the same for every key thread
           float4 l4, d4;
           if (p.ld_bulk) {
-            l4 = *reinterpret_cast<const float4*>(s_lse + c * 32 + e);
-            d4 = *reinterpret_cast<const float4*>(s_d + c * 32 + e);
+            l4 = *reinterpret_cast<const float4*>(s_lse + c * 16 + e);
+            d4 = *reinterpret_cast<const float4*>(s_d + c * 16 + e);
           } else {
-            const float* lp = lse_h + q0 + c * 32 + e;
-            const float* dp = d_h + q0 + c * 32 + e;
+            const float* lp = lse_h + q0 + c * 16 + e;
+            const float* dp = d_h + q0 + c * 16 + e;
             l4 = make_float4(__ldg(lp), __ldg(lp + 1), __ldg(lp + 2), __ldg(lp + 3));
             d4 = make_float4(__ldg(dp), __ldg(dp + 1), __ldg(dp + 2), __ldg(dp + 3));
           }
@@ -315,7 +343,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
             const float pv = ex2_approx(fmaf(__uint_as_float(sv[e + u]), sl2, -lq[u]));
             const float dsv = pv * (__uint_as_float(dv[e + u]) - dq[u]);
             if (need_mask) {
-              const int q = q0 + c * 32 + e + u;
+              const int q = q0 + c * 16 + e + u;
               const bool valid = key < p.seq && q < p.seq && (!p.causal || q >= key);
               pp[u] = valid ? pv : 0.f;
               ds[u] = valid ? dsv : 0.f;
@@ -329,16 +357,15 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
           dk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
           dk[(e >> 1) + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        // P^T of queries [32 c, 32 c + 32) into 16 columns this thread has
-        // already read: [16 c, 16 c + 16) + 32 for the second half
-        tmem_st_32x32b_x16(tmem + lane_addr + TC_S + c * 16 + grp * 32, pk);
-        // dS^T row `row`, queries [32 c, 32 c + 32): 128-byte swizzled rows,
-        // queries 0-63 in the first 16 KB half, 64-127 in the second
-        const uint32_t half = ds_row + static_cast<uint32_t>(c >> 1) * AB_SUB;
+        // P^T of queries [16 c, 16 c + 16) into 8 columns of S^T this thread
+        // has already read: [8 c, 8 c + 8), + 16 for the second group
+        tmem_st_32x32b_x8(tS + c * 8 + grp * 16, pk);
+        // dS^T row `row`, queries [16 c, 16 c + 16): two 16-byte chunks of
+        // the 128-byte swizzled row
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t chunk = static_cast<uint32_t>((c & 1) * 4 + u);
-          st_shared_v4(half + ((chunk ^ (static_cast<uint32_t>(row) & 7u)) << 4), dk[4 * u],
+        for (int u = 0; u < 2; ++u) {
+          const uint32_t chunk = static_cast<uint32_t>(c * 2 + u);
+          st_shared_v4(ds_row + ((chunk ^ (static_cast<uint32_t>(row) & 7u)) << 4), dk[4 * u],
                        dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
       }
@@ -346,31 +373,9 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       fence_proxy_async_shared();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(AB_DS));
-      if (grp == 1) {
-        // drain this block's dQ (one thread per query = TMEM lane)
-        if (!mbar_wait(bar(AB_DQFULL), it & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t v[AB_D];
-#pragma unroll
-        for (int c = 0; c < AB_D / 32; ++c)
-          tmem_ld_32x32b_x32(tmem + lane_addr + TC_DP + c * 32, &v[c * 32]);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(AB_DQEMPTY));  // the columns may be overwritten now
-        const int q = q0 + row;
-        if (q < p.seq) {
-          // layout [d / 4][stride][4]: a warp's 32 queries are 512 contiguous bytes
-          float* a = acc_h + static_cast<int64_t>(q) * 4;
-#pragma unroll
-          for (int u = 0; u < AB_D / 4; ++u)
-            red_add_v4(a + static_cast<int64_t>(u) * p.stride * 4, v[4 * u], v[4 * u + 1],
-                       v[4 * u + 2], v[4 * u + 3]);
-        }
+      if (lane == 0) {
+        mbar_arrive(bar(AB_DS + b));
+        if (p.ld_bulk) mbar_arrive(bar(AB_LDEMPTY + b));
       }
     }
     if (!ok) {
@@ -383,14 +388,14 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       uint16_t* base = p.dqkv + (static_cast<int64_t>(g) * p.M + row_base + key) * (3 * p.hs) +
                        head * AB_D;
 #pragma unroll 1
-      for (int c = 2 * grp; c < 2 * grp + 2; ++c) {
-        uint32_t kv[32], vv[32];
-        tmem_ld_32x32b_x32(tmem + lane_addr + TC_DK + c * 32, kv);
-        tmem_ld_32x32b_x32(tmem + lane_addr + TC_DV + c * 32, vv);
+      for (int c = 4 * grp; c < 4 * grp + 4; ++c) {  // 16 columns at a time
+        uint32_t kv[16], vv[16];
+        tmem_ld_32x32b_x16(tmem + lane_addr + 384u + c * 16, kv);
+        tmem_ld_32x32b_x16(tmem + lane_addr + 256u + c * 16, vv);
         tmem_ld_wait();
         if (key < p.seq) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int e = 0; e < 2; ++e) {
             uint4 wk, wv;
             wk.x = pack_bf16x2(__uint_as_float(kv[8 * e + 0]) * p.scale,
                                __uint_as_float(kv[8 * e + 1]) * p.scale);
@@ -404,12 +409,46 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
             wv.y = pack_bf16x2(__uint_as_float(vv[8 * e + 2]), __uint_as_float(vv[8 * e + 3]));
             wv.z = pack_bf16x2(__uint_as_float(vv[8 * e + 4]), __uint_as_float(vv[8 * e + 5]));
             wv.w = pack_bf16x2(__uint_as_float(vv[8 * e + 6]), __uint_as_float(vv[8 * e + 7]));
-            *reinterpret_cast<uint4*>(base + p.hs + c * 32 + 8 * e) = wk;
-            *reinterpret_cast<uint4*>(base + 2 * p.hs + c * 32 + 8 * e) = wv;
+            *reinterpret_cast<uint4*>(base + p.hs + c * 16 + 8 * e) = wk;
+            *reinterpret_cast<uint4*>(base + 2 * p.hs + c * 16 + 8 * e) = wv;
           }
         }
       }
     } else {
+      if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
+      *abort_flag = 1;
+    }
+  } else if (warp >= 8 && warp < 12) {
+    // ------------------------------------------------------------ dQ^T
+    const int rq = warp & 3;
+    const int dcol = rq * 32 + lane;  // head-dimension column (= TMEM lane)
+    const uint32_t lane_addr = static_cast<uint32_t>(rq * 32) << 16;
+    // accumulator rows [stride][128]: a warp's 32 lanes cover 128 contiguous bytes
+    float* acc_h = p.dq_acc + (hb * p.stride + row_base) * AB_D + dcol;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int b = it & 1;
+      if (!mbar_wait(bar(AB_DQFULL + b), (it >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[AB_BQ];
+      const uint32_t tP = tmem + lane_addr + 128u * b + 64u;
+      tmem_ld_32x32b_x32(tP, &v[0]);
+      tmem_ld_32x32b_x32(tP + 32, &v[32]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(AB_DQEMPTY + b));  // the columns may be overwritten now
+      const int q0 = (i_first + it) * AB_BQ;
+      const int nq_valid = min(AB_BQ, p.seq - q0);
+      float* a = acc_h + static_cast<int64_t>(q0) * AB_D;
+#pragma unroll
+      for (int q = 0; q < AB_BQ; ++q)
+        if (q < nq_valid) red_add_f32(a + static_cast<int64_t>(q) * AB_D, v[q]);
+    }
+    if (!ok) {
       if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
       *abort_flag = 1;
     }
@@ -454,23 +493,23 @@ __global__ void __launch_bounds__(256) zero_f32x4_kernel(float4* __restrict__ p,
     p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dQ (bf16, scaled) into the Q columns of dQKV from the [d/4][stride][4]
-// accumulator; thread = ((shard, head), 8 columns, token), tokens fastest.
+// dQ (bf16, scaled) into the Q columns of dQKV from the [stride][128]
+// accumulator; thread = ((shard, head), token, 8 columns), columns fastest.
 __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float* __restrict__ acc,
                                                           uint16_t* __restrict__ dqkv, int64_t n,
                                                           int64_t M, int64_t stride, int hps,
                                                           int hs, float scale) {
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (i >= n) return;
-  const int64_t tok = i % M;
-  const int64_t r = i / M;
-  const int c8 = static_cast<int>(r % (AB_D / 8));
-  const int64_t hb = r / (AB_D / 8);
+  const int c8 = static_cast<int>(i % (AB_D / 8));
+  const int64_t r = i / (AB_D / 8);
+  const int64_t tok = r % M;
+  const int64_t hb = r / M;
   const int head = static_cast<int>(hb % hps);
   const int64_t g = hb / hps;
-  const float* a = acc + (hb * (AB_D / 4) + 2 * c8) * stride * 4 + tok * 4;
+  const float* a = acc + (hb * stride + tok) * AB_D + c8 * 8;
   const float4 x = *reinterpret_cast<const float4*>(a);
-  const float4 y = *reinterpret_cast<const float4*>(a + stride * 4);
+  const float4 y = *reinterpret_cast<const float4*>(a + 4);
   uint4 w;
   w.x = pack_bf16x2(x.x * scale, x.y * scale);
   w.y = pack_bf16x2(x.z * scale, x.w * scale);
@@ -497,12 +536,12 @@ static PFN_cuTensorMapEncodeTiled_v12000 bwd_map_encoder() {
 }
 
 static bool encode_rows(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base,
-                        int64_t cols, int64_t rows, int shards) {
+                        int64_t cols, int64_t rows, int shards, uint32_t box_rows) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(shards)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols * 2),
                            static_cast<cuuint64_t>(rows * cols * 2)};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -519,9 +558,10 @@ int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const f
   const int64_t stride = M + 128;
   auto enc = bwd_map_encoder();
   if (enc == nullptr) return 1;
-  CUtensorMap tm_qkv, tm_do;
-  if (!encode_rows(enc, &tm_qkv, QKV, 3 * hs, M, n_shards)) return 1;
-  if (!encode_rows(enc, &tm_do, dO, hs, M, n_shards)) return 1;
+  CUtensorMap tm_kv, tm_q, tm_do;
+  if (!encode_rows(enc, &tm_kv, QKV, 3 * hs, M, n_shards, AB_BK)) return 1;
+  if (!encode_rows(enc, &tm_q, QKV, 3 * hs, M, n_shards, AB_BQ)) return 1;
+  if (!encode_rows(enc, &tm_do, dO, hs, M, n_shards, AB_BQ)) return 1;
 
   const int64_t heads_total = static_cast<int64_t>(n_shards) * hps;
   // dQ accumulator to zero, D = rowsum(dO * O)
@@ -555,9 +595,9 @@ int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const f
                        AB_SMEM);
   const dim3 grid(static_cast<unsigned>(heads_total * batch),
                   static_cast<unsigned>((seq + AB_BK - 1) / AB_BK));
-  attention_bwd_tc_kernel<<<grid, AB_THREADS, AB_SMEM, s>>>(tm_qkv, tm_do, p);
+  attention_bwd_tc_kernel<<<grid, AB_THREADS, AB_SMEM, s>>>(tm_kv, tm_q, tm_do, p);
 
-  const int64_t n = heads_total * (AB_D / 8) * M;
+  const int64_t n = heads_total * M * (AB_D / 8);
   attn_bwd_dq_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
       dq_acc, static_cast<uint16_t*>(dQKV), n, M, stride, hps, static_cast<int>(hs), p.scale);
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
