@@ -217,6 +217,9 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     constexpr uint32_t idesc_dq =
         umma_idesc_bf16_f32_bmn(AB_D, AB_BQ) | (1u << 15);                   // A, B MN-major
     const uint32_t sK = s0 + AOFF_K, sV = s0 + AOFF_V;
+    // descriptors built once; each MMA moves them by a constant offset
+    const uint64_t dK = umma_desc_sw128(sK), dV = umma_desc_sw128(sV);
+    const uint64_t dK_mn = umma_desc_sw128_mn(sK, AB_KSUB);
     // S^T and dP^T of query block k into buffer k & 1
     auto issue_sdp = [&](int k) -> bool {
       const int st = k % AB_NST, b = k & 1;
@@ -225,19 +228,20 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       // dP^T were consumed before that dQ^T was computed)
       if (k >= 2 && !mbar_wait(bar(AB_DQEMPTY + b), ((k - 2) >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
-      const uint32_t sQ = s0 + AOFF_Q + st * AB_QTILE, sdO = s0 + AOFF_DO + st * AB_QTILE;
+      const uint64_t dQ = umma_desc_sw128(s0 + AOFF_Q + st * AB_QTILE);
+      const uint64_t dO = umma_desc_sw128(s0 + AOFF_DO + st * AB_QTILE);
       const uint32_t tS = tmem + 128u * b, tP = tS + 64u;
 #pragma unroll
       for (int kk = 0; kk < AB_D / 16; ++kk) {   // contraction over d
         const uint32_t ka = (kk >> 2) * AB_KSUB + (kk & 3) * 32;
         const uint32_t qa = (kk >> 2) * AB_QSUB + (kk & 3) * 32;
-        umma_bf16(tS, umma_desc_sw128(sK + ka), umma_desc_sw128(sQ + qa), idesc_s, kk > 0 ? 1u : 0u);
+        umma_bf16(tS, desc_advance(dK, ka), desc_advance(dQ, qa), idesc_s, kk > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int kk = 0; kk < AB_D / 16; ++kk) {
         const uint32_t ka = (kk >> 2) * AB_KSUB + (kk & 3) * 32;
         const uint32_t qa = (kk >> 2) * AB_QSUB + (kk & 3) * 32;
-        umma_bf16(tP, umma_desc_sw128(sV + ka), umma_desc_sw128(sdO + qa), idesc_s, kk > 0 ? 1u : 0u);
+        umma_bf16(tP, desc_advance(dV, ka), desc_advance(dO, qa), idesc_s, kk > 0 ? 1u : 0u);
       }
       umma_commit(bar(AB_SDP + b));
       return true;
@@ -255,26 +259,28 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t sQ = s0 + AOFF_Q + st * AB_QTILE, sdO = s0 + AOFF_DO + st * AB_QTILE;
-      const uint32_t sDS = s0 + AOFF_DS + b * AB_DSTILE;
+      const uint64_t dQ_mn = umma_desc_sw128_mn(s0 + AOFF_Q + st * AB_QTILE, AB_QSUB);
+      const uint64_t dO_mn = umma_desc_sw128_mn(s0 + AOFF_DO + st * AB_QTILE, AB_QSUB);
+      const uint64_t dS_k = umma_desc_sw128(s0 + AOFF_DS + b * AB_DSTILE);
+      const uint64_t dS_mn = umma_desc_sw128_mn(s0 + AOFF_DS + b * AB_DSTILE, AB_QSUB);
       const uint32_t tS = tmem + 128u * b, tP = tS + 64u;
       // dV += P^T dO: P^T (keys x queries, bf16 pairs) from TMEM
 #pragma unroll
       for (int kk = 0; kk < AB_BQ / 16; ++kk)
-        umma_bf16_tmem_a(tmem + 256u, tS + kk * 8 + (kk >= 2 ? 16 : 0),
-                         umma_desc_sw128_mn(sdO + kk * 2048, AB_QSUB),
+        umma_bf16_tmem_a(tmem + 256u, tS + kk * 8 + (kk >= 2 ? 16 : 0),  // P^T of queries 16 kk..
+                         desc_advance(dO_mn, kk * 2048),
                          idesc_kmn, (it > 0 || kk > 0) ? 1u : 0u);
       // dK += dS^T Q
 #pragma unroll
       for (int kk = 0; kk < AB_BQ / 16; ++kk)
-        umma_bf16(tmem + 384u, umma_desc_sw128(sDS + kk * 32),
-                  umma_desc_sw128_mn(sQ + kk * 2048, AB_QSUB), idesc_kmn,
+        umma_bf16(tmem + 384u, desc_advance(dS_k, kk * 32), desc_advance(dQ_mn, kk * 2048),
+                  idesc_kmn,
                   (it > 0 || kk > 0) ? 1u : 0u);
       // dQ^T = K^T dS^T (head dim x queries), contraction over the keys
 #pragma unroll
       for (int kk = 0; kk < AB_BK / 16; ++kk)
-        umma_bf16(tP, umma_desc_sw128_mn(sK + kk * 2048, AB_KSUB),
-                  umma_desc_sw128_mn(sDS + kk * 2048, AB_QSUB), idesc_dq, kk > 0 ? 1u : 0u);
+        umma_bf16(tP, desc_advance(dK_mn, kk * 2048), desc_advance(dS_mn, kk * 2048), idesc_dq,
+                  kk > 0 ? 1u : 0u);
       umma_commit(bar(AB_DQFULL + b));
       umma_commit(bar(AB_QEMPTY + st));
     }
@@ -312,26 +318,26 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       const bool need_mask =
           (p.causal && q0 < kv0 + AB_BK) || q0 + AB_BQ > p.seq || kv0 + AB_BK > p.seq;
       const uint32_t tS = tmem + lane_addr + 128u * b, tP = tS + 64u;
-      const float* s_lse = reinterpret_cast<const float*>(sm + AOFF_LD + b * (2 * AB_BQ * 4));
-      const float* s_d = s_lse + AB_BQ;
+      const uint32_t s_lse = s0 + AOFF_LD + b * (2 * AB_BQ * 4), s_d = s_lse + AB_BQ * 4;
       const uint32_t ds_row = s0 + AOFF_DS + b * AB_DSTILE + static_cast<uint32_t>(row) * 128u;
-#pragma unroll 1
-      for (int c = 2 * grp; c < 2 * grp + 2; ++c) {  // 16 queries at a time
-        uint32_t sv[16], dv[16];
-        tmem_ld_32x32b_x16(tS + c * 16, sv);
-        tmem_ld_32x32b_x16(tP + c * 16, dv);
+      {
+        // this thread's 32 queries [32 grp, 32 grp + 32): one TMEM round trip
+        const int c = grp;
+        uint32_t sv[32], dv[32];
+        tmem_ld_32x32b_x32(tS + c * 32, sv);
+        tmem_ld_32x32b_x32(tP + c * 32, dv);
         tmem_ld_wait();
-        uint32_t pk[8], dk[8];
+        uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
+        for (int e = 0; e < 32; e += 4) {
           // lse and D of these 4 queries: the same for every key thread
           float4 l4, d4;
           if (p.ld_bulk) {
-            l4 = *reinterpret_cast<const float4*>(s_lse + c * 16 + e);
-            d4 = *reinterpret_cast<const float4*>(s_d + c * 16 + e);
+            l4 = ld_shared_v4f(s_lse + (c * 32 + e) * 4);
+            d4 = ld_shared_v4f(s_d + (c * 32 + e) * 4);
           } else {
-            const float* lp = lse_h + q0 + c * 16 + e;
-            const float* dp = d_h + q0 + c * 16 + e;
+            const float* lp = lse_h + q0 + c * 32 + e;
+            const float* dp = d_h + q0 + c * 32 + e;
             l4 = make_float4(__ldg(lp), __ldg(lp + 1), __ldg(lp + 2), __ldg(lp + 3));
             d4 = make_float4(__ldg(dp), __ldg(dp + 1), __ldg(dp + 2), __ldg(dp + 3));
           }
@@ -343,7 +349,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
             const float pv = ex2_approx(fmaf(__uint_as_float(sv[e + u]), sl2, -lq[u]));
             const float dsv = pv * (__uint_as_float(dv[e + u]) - dq[u]);
             if (need_mask) {
-              const int q = q0 + c * 16 + e + u;
+              const int q = q0 + c * 32 + e + u;
               const bool valid = key < p.seq && q < p.seq && (!p.causal || q >= key);
               pp[u] = valid ? pv : 0.f;
               ds[u] = valid ? dsv : 0.f;
@@ -357,14 +363,13 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
           dk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
           dk[(e >> 1) + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        // P^T of queries [16 c, 16 c + 16) into 8 columns of S^T this thread
-        // has already read: [8 c, 8 c + 8), + 16 for the second group
-        tmem_st_32x32b_x8(tS + c * 8 + grp * 16, pk);
-        // dS^T row `row`, queries [16 c, 16 c + 16): two 16-byte chunks of
+        // P^T of the 32 queries into 16 columns of S^T this thread has read
+        tmem_st_32x32b_x16(tS + c * 32, pk);
+        // dS^T row `row`, queries [32 c, 32 c + 32): four 16-byte chunks of
         // the 128-byte swizzled row
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const uint32_t chunk = static_cast<uint32_t>(c * 2 + u);
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t chunk = static_cast<uint32_t>(c * 4 + u);
           st_shared_v4(ds_row + ((chunk ^ (static_cast<uint32_t>(row) & 7u)) << 4), dk[4 * u],
                        dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
