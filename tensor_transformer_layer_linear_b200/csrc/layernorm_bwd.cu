@@ -43,7 +43,7 @@ __device__ __forceinline__ void unpack8(const uint4& b, float (&a)[8]) {
 }
 
 template <int CH, int NS>
-__global__ void __launch_bounds__(kLnbThreads) rows_sum_ln_bwd_kernel(
+__global__ void __launch_bounds__(kLnbThreads, (CH <= 2 ? 3 : 1)) rows_sum_ln_bwd_kernel(
     const float* __restrict__ P, int n_shards, int64_t stride, int64_t rows, int h,
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ gamma,
     const uint16_t* __restrict__ res, float eps, uint16_t* __restrict__ dx,
@@ -164,10 +164,20 @@ __global__ void __launch_bounds__(kLnbThreads) rows_sum_ln_bwd_kernel(
   }
 }
 
+// CTAs resident per SM: three for rows of up to 4096 columns (register
+// budget), else one
 template <int CH>
-static void launch_lnb_ch(const float* P, int n_shards, int64_t rows, int h, const void* x,
-                          const void* gamma, const void* res, float eps, void* dx, float* dg_part,
-                          float* db_part, int ctas, cudaStream_t s) {
+constexpr int lnb_ctas_per_sm() {
+  return CH <= 2 ? 3 : 1;
+}
+
+template <int CH>
+static int launch_lnb_ch(const float* P, int n_shards, int64_t rows, int h, const void* x,
+                         const void* gamma, const void* res, float eps, void* dx, float* dg_part,
+                         float* db_part, int max_ctas, int num_sms, cudaStream_t s) {
+  int ctas = lnb_ctas_per_sm<CH>() * num_sms;
+  if (ctas > max_ctas) ctas = max_ctas;
+  if (ctas > rows) ctas = static_cast<int>(rows);
   auto X = static_cast<const uint16_t*>(x);
   auto G = static_cast<const uint16_t*>(gamma);
   auto R = static_cast<const uint16_t*>(res);
@@ -188,6 +198,7 @@ static void launch_lnb_ch(const float* P, int n_shards, int64_t rows, int h, con
     case 8: rows_sum_ln_bwd_kernel<CH, 8><<<ctas, kLnbThreads, smem, s>>>(P, 8, stride, rows, h, X, G, R, eps, D, dg_part, db_part); break;
     default: rows_sum_ln_bwd_kernel<CH, 0><<<ctas, kLnbThreads, smem, s>>>(P, n_shards, stride, rows, h, X, G, R, eps, D, dg_part, db_part); break;
   }
+  return ctas;
 }
 
 int launch_rows_sum_ln_bwd(const float* P, int n_shards, int64_t rows, int64_t h, const void* x,
@@ -195,21 +206,19 @@ int launch_rows_sum_ln_bwd(const float* P, int n_shards, int64_t rows, int64_t h
                            float* dgamma, float* dbeta, float* part, int max_ctas,
                            cudaStream_t s, int num_sms) {
   if (rows <= 0) return 0;
-  int ctas = 4 * num_sms;
-  if (ctas > max_ctas) ctas = max_ctas;
-  if (ctas > rows) ctas = static_cast<int>(rows);
   float* dg_part = part;
   float* db_part = part + static_cast<int64_t>(max_ctas) * h;
   const int hh = static_cast<int>(h);
   const int64_t nch = h / 8;
+  int ctas;
   if (nch <= kLnbThreads)
-    launch_lnb_ch<1>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, ctas, s);
+    ctas = launch_lnb_ch<1>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s);
   else if (nch <= 2 * kLnbThreads)
-    launch_lnb_ch<2>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, ctas, s);
+    ctas = launch_lnb_ch<2>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s);
   else if (nch <= 4 * kLnbThreads)
-    launch_lnb_ch<4>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, ctas, s);
+    ctas = launch_lnb_ch<4>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s);
   else
-    launch_lnb_ch<8>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, ctas, s);
+    ctas = launch_lnb_ch<8>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s);
   if (launch_slab_sum(dg_part, ctas, hh, dgamma, s) != 0) return 2;
   if (launch_slab_sum(db_part, ctas, hh, dbeta, s) != 0) return 2;
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
