@@ -684,6 +684,84 @@ def gqa_self_attention_sharded(X, Wqkv, bqkv, Wo, bo, residual, batch: int,
     return reduce_partials(row_parallel_linear(O_i, Wo, n_shards), bo, residual)
 
 
+def gqa_attention_heads_backward(Q, K, V, dO, batch: int, seq: int, n_q: int,
+                                 n_kv: int, causal: bool) -> tuple:
+    """attention_head_backward for every (sequence, query head); query head j
+    uses key/value head j // (n_q / n_kv), so a key/value head's gradient is
+    the sum over the query heads of its group. Returns (dQ, dK, dV)."""
+    d = Q.shape[1] // n_q
+    g = n_q // n_kv
+    dQ, dK, dV = np.zeros_like(Q, dtype=np.float64), np.zeros_like(K, dtype=np.float64), \
+        np.zeros_like(V, dtype=np.float64)
+    for s in range(batch):
+        r = slice(s * seq, (s + 1) * seq)
+        for j in range(n_q):
+            c = slice(j * d, (j + 1) * d)
+            kc = slice((j // g) * d, (j // g + 1) * d)
+            dq, dk, dv = attention_head_backward(Q[r, c], K[r, kc], V[r, kc], dO[r, c], causal)
+            dQ[r, c] = dq
+            dK[r, kc] += dk
+            dV[r, kc] += dv
+    return dQ, dK, dV
+
+
+def gqa_self_attention_backward(X, Wqkv, bqkv, Wo, bo, dY, batch: int, seq: int,
+                                n_q: int, n_kv: int, causal: bool = True,
+                                residual: bool = True) -> dict:
+    """Gradients of the unsharded GQA block given dY: dX, dWqkv, dbqkv, dWo, dbo."""
+    d = Wo.shape[0] // n_q
+    QKV = linear(X, Wqkv, bqkv)
+    Q = QKV[:, :n_q * d]
+    K = QKV[:, n_q * d:(n_q + n_kv) * d]
+    V = QKV[:, (n_q + n_kv) * d:]
+    O = gqa_attention_heads(Q, K, V, batch, seq, n_q, n_kv, causal)
+    dO = dY @ Wo.T
+    dQ, dK, dV = gqa_attention_heads_backward(Q, K, V, dO, batch, seq, n_q, n_kv, causal)
+    dQKV = np.concatenate([dQ, dK, dV], axis=1)
+    dX = dQKV @ Wqkv.T
+    if residual:
+        dX = dX + dY
+    return dict(dX=dX, dWqkv=X.T @ dQKV, dbqkv=dQKV.sum(axis=0), dWo=O.T @ dY,
+                dbo=dY.sum(axis=0))
+
+
+def gqa_self_attention_backward_sharded(X, Wqkv, bqkv, Wo, bo, dY, batch: int,
+                                        seq: int, n_q: int, n_kv: int,
+                                        n_shards: int, causal: bool = True,
+                                        residual: bool = True) -> dict:
+    """The tensor-parallel GQA backward: as self_attention_backward_sharded,
+    with each shard's key/value heads (duplicated when N > n_kv) receiving the
+    gradient of its own query heads. A duplicated head's weight gradient is the
+    sum over its replicas (the gradient of a replicated parameter); the
+    per-shard gradients, packed like the shards, are returned as well."""
+    d = Wo.shape[0] // n_q
+    qs, kvl = n_q // n_shards, gqa_kv_local(n_kv, n_shards)
+    hs = qs * d
+    Wo_i = shard_matrices(Wo, SPLIT_ROW, n_shards)
+    parts, dqkv_shards, dW_shards, db_shards = [], [], [], []
+    dWqkv, dbqkv = np.zeros(Wqkv.shape), np.zeros(Wqkv.shape[1])
+    dWo = np.zeros(Wo.shape)
+    for i, cols in enumerate(gqa_shard_columns(n_q, n_kv, d, n_shards)):
+        W = Wqkv[:, cols]
+        q = linear(X, W, None if bqkv is None else bqkv[cols])
+        Q, K, V = q[:, :hs], q[:, hs:hs + kvl * d], q[:, hs + kvl * d:]
+        O = gqa_attention_heads(Q, K, V, batch, seq, qs, kvl, causal)
+        dO = dY @ Wo_i[i].T
+        dQ, dK, dV = gqa_attention_heads_backward(Q, K, V, dO, batch, seq, qs, kvl, causal)
+        dQKV = np.concatenate([dQ, dK, dV], axis=1)
+        dqkv_shards.append(dQKV)
+        parts.append(dQKV @ W.T)
+        dW_shards.append((X.T @ dQKV).T)       # packed like the shard: [cols][h_in]
+        db_shards.append(dQKV.sum(axis=0))
+        np.add.at(dWqkv.T, cols, (X.T @ dQKV).T)
+        np.add.at(dbqkv, cols, dQKV.sum(axis=0))
+        dWo[i * hs:(i + 1) * hs, :] = O.T @ dY
+    dX = reduce_partials(parts, None, dY if residual else None)
+    return dict(dX=dX, dWqkv=dWqkv, dbqkv=dbqkv, dWo=dWo, dbo=dY.sum(axis=0),
+                dX_partials=parts, dQKV_shards=dqkv_shards,
+                dWqkv_packed=np.stack(dW_shards), dbqkv_packed=np.stack(db_shards))
+
+
 # --------------------------------------------------------------------------
 # sequence parallelism ([TP-LLM] "Sequence Parallelism")
 # --------------------------------------------------------------------------

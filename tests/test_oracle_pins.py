@@ -781,3 +781,41 @@ def test_attention_logsumexp_closed_forms():
     q = np.array([[2.0, 0.0]])                     # d = 2: scores k . q / sqrt 2
     k = np.array([[0.0, 0.0], [math.log(3) * math.sqrt(2) / 2, 0.0]])
     assert O.attention_logsumexp(q, k, False)[0] == pytest.approx(math.log(4.0), abs=1e-14)
+
+
+def test_gqa_attention_backward_matches_finite_differences():
+    rng = np.random.default_rng(37)
+    b, s, d, nq, nkv = 1, 4, 2, 4, 2
+    h = nq * d
+    X = rng.standard_normal((b * s, h))
+    Wqkv = rng.standard_normal((h, (nq + 2 * nkv) * d)) * .4
+    bqkv = rng.standard_normal((nq + 2 * nkv) * d) * .1
+    Wo, bo = rng.standard_normal((h, h)) * .4, rng.standard_normal(h) * .1
+    dY = rng.standard_normal((b * s, h))
+    g = O.gqa_self_attention_backward(X, Wqkv, bqkv, Wo, bo, dY, b, s, nq, nkv)
+    loss = lambda: float(np.sum(O.gqa_self_attention(X, Wqkv, bqkv, Wo, bo, X, b, s, nq, nkv) * dY))  # noqa: E731
+    for name, arr in (("dX", X), ("dWqkv", Wqkv), ("dbqkv", bqkv), ("dWo", Wo), ("dbo", bo)):
+        np.testing.assert_allclose(g[name], _num_grad(loss, arr), rtol=1e-6, atol=1e-8,
+                                   err_msg=name)
+
+
+@pytest.mark.parametrize("n,nkv", [(1, 2), (2, 2), (4, 2), (8, 2), (4, 4), (2, 8)])
+def test_gqa_attention_backward_sharded_equals_unsharded(n, nkv):
+    """Whole groups per shard (N <= n_kv) and duplicated kv heads (N > n_kv):
+    the replicas' weight gradients sum to the logical ones."""
+    rng = np.random.default_rng(38 + n)
+    b, s, d, nq = 2, 5, 2, 8
+    h = nq * d
+    X = rng.standard_normal((b * s, h))
+    Wqkv = rng.standard_normal((h, (nq + 2 * nkv) * d)) * .3
+    bqkv = rng.standard_normal((nq + 2 * nkv) * d) * .1
+    Wo, bo = rng.standard_normal((h, h)) * .3, rng.standard_normal(h) * .1
+    dY = rng.standard_normal((b * s, h))
+    ref = O.gqa_self_attention_backward(X, Wqkv, bqkv, Wo, bo, dY, b, s, nq, nkv)
+    got = O.gqa_self_attention_backward_sharded(X, Wqkv, bqkv, Wo, bo, dY, b, s, nq, nkv, n)
+    for k in ("dX", "dWqkv", "dbqkv", "dWo", "dbo"):
+        np.testing.assert_allclose(got[k], ref[k], rtol=1e-11, atol=1e-11, err_msg=k)
+    # with n_kv = n_q GQA is multi-head attention
+    if nkv == nq:
+        mha = O.self_attention_backward(X, Wqkv, bqkv, Wo, bo, dY, b, s, nq)
+        np.testing.assert_allclose(ref["dX"], mha["dX"], rtol=1e-12, atol=1e-12)
