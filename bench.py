@@ -105,6 +105,10 @@ def work(cfg: dict) -> dict:
         if kind in ("attn", "layer"):
             gb += 16.0 * M * h * h
             ab = 2.0 * fl["attention"]
+        if kind == "attn_gqa":
+            qkv = (cfg["n_heads"] + 2 * cfg["n_kv_heads"]) * (h // cfg["n_heads"])
+            gb += 4.0 * M * h * h + 4.0 * M * qkv * h   # dO, dW_O; dX, dW_QKV
+            ab = 2.0 * fl["attention"]
         fl = {"gemm_backward": gb, "attention_backward": ab, "gemm_column_parallel": 0.0,
               "gemm_row_parallel": 0.0, "attention": 0.0}
         if kind == "layer":
@@ -209,6 +213,12 @@ def oracle_sample(cfg: dict, inp: dict, tokens: int):
             p = {k: f64(v) for k, v in inp.items() if k != "X"}
             O.transformer_layer_backward(x, p, dY, 1, T, cfg["n_heads"], cfg["n_shards"],
                                          cfg.get("ln_eps", 1e-5))
+        elif cfg["kind"] == "attn_gqa":
+            O.gqa_self_attention_backward_sharded(x, f64(inp["Wqkv"]), f64(inp["bqkv"]),
+                                                  f64(inp["Wo"]), f64(inp["bo"]), dY, 1, T,
+                                                  cfg["n_heads"], cfg["n_kv_heads"],
+                                                  cfg["n_shards"], cfg.get("causal", True),
+                                                  bool(cfg.get("residual")))
         elif cfg["kind"] == "attn":
             O.self_attention_backward_sharded(x, f64(inp["Wqkv"]), f64(inp["bqkv"]),
                                               f64(inp["Wo"]), f64(inp["bo"]), dY, 1, T,
@@ -354,6 +364,10 @@ class Model:
         if kind == "mlp":
             self.dA, self.dB, self.db1, self.db2 = f32(h * F), f32(h * F), f32(F), f32(h)
             wsk = tp.TP_WS_MLP_BWD
+        elif kind == "attn_gqa":
+            self.dWqkv, self.dbqkv = f32(self.qkv_cols * h), f32(self.qkv_cols)
+            self.dWo, self.dbo = f32(h * h), f32(h)
+            wsk = tp.TP_WS_ATTN_BWD
         elif kind == "attn":
             self.dWqkv, self.dbqkv, self.dWo, self.dbo = f32(3 * h * h), f32(3 * h), f32(h * h), f32(h)
             wsk = tp.TP_WS_ATTN_BWD
@@ -377,6 +391,12 @@ class Model:
                 tp.tp_mlp_backward(X, self.M, h, cfg["ffn"], n, self.A, self.b1, self.B, self.dY,
                                    cfg.get("residual", False), self.ws_bwd, self.ws_bwd_bytes, dX,
                                    self.dA, self.db1, self.dB, self.db2)
+            elif kind == "attn_gqa":
+                tp.tp_attn_backward_gqa(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"],
+                                        cfg["n_kv_heads"], cfg.get("causal", True), n, self.Wqkv,
+                                        self.bqkv, self.Wo, self.dY, cfg.get("residual", False),
+                                        self.ws_bwd, self.ws_bwd_bytes, dX, self.dWqkv,
+                                        self.dbqkv, self.dWo, self.dbo)
             elif kind == "attn":
                 tp.tp_attn_backward(X, cfg["batch"], cfg["seq"], h, cfg["n_heads"],
                                     cfg.get("causal", True), n, self.Wqkv, self.bqkv, self.Wo,
@@ -660,8 +680,8 @@ def main():
     if args.shards:
         cfg["n_shards"] = args.shards
     if args.backward:
-        if cfg["kind"] not in ("mlp", "attn", "layer"):
-            ap.error("--backward applies to the MLP, attention and layer workloads")
+        if cfg["kind"] not in ("mlp", "attn", "attn_gqa", "layer"):
+            ap.error("--backward applies to the MLP, attention, GQA and layer workloads")
         cfg["backward"] = True
     if args.sequence_parallel:
         if cfg["kind"] != "layer":

@@ -361,6 +361,47 @@ tp_status tp_layer_backward(const uint16_t* X, int64_t batch, int64_t seq,
                             size_t ws_bytes, uint16_t* dX,
                             const tp_layer_grads* g, void* stream);
 
+/* tp_attention_gqa_lse - tp_attention_gqa that also writes the base-2
+ * log-sum-exp of every query's scaled scores, laid out as in
+ * tp_attention_lse (n_q*(batch*seq + 128) floats, query heads in shard
+ * order). */
+tp_status tp_attention_gqa_lse(const uint16_t* QKV_shards, int64_t batch,
+                               int64_t seq, int64_t n_q, int64_t n_kv,
+                               int64_t head_dim, int causal, int n_shards,
+                               uint16_t* O_shards, float* lse, void* stream);
+
+/* tp_attention_gqa_backward - tp_attention_backward for grouped-query QKV
+ * shards (the layout of tp_shard_qkv_gqa): a key/value head's dK and dV are
+ * summed over the local query heads of its group ([TP-LLM] "Grouped-Query
+ * Attention (GQA) Constraints"). When N > n_kv each shard's duplicated
+ * key/value head receives the gradient of that shard's query heads only; the
+ * gradient of the logical head is the sum over its replicas. dQKV_shards is
+ * packed like QKV_shards. ws >= tp_workspace_bytes(TP_WS_ATTN_CORE_BWD, M,
+ * n_q*head_dim, 0, N). */
+tp_status tp_attention_gqa_backward(const uint16_t* QKV_shards,
+                                    const uint16_t* O_shards,
+                                    const uint16_t* dO_shards, const float* lse,
+                                    int64_t batch, int64_t seq, int64_t n_q,
+                                    int64_t n_kv, int64_t head_dim, int causal,
+                                    int n_shards, void* ws, size_t ws_bytes,
+                                    uint16_t* dQKV_shards, void* stream);
+
+/* tp_attn_backward_gqa - tp_attn_backward for the grouped-query block of
+ * tp_attn_forward_gqa (h = n_q * 128). dWqkv_shards and dbqkv_shards are
+ * packed like the GQA shards ([N][(n_q/N + 2 kv_local) 128][h] and
+ * [N][(n_q/N + 2 kv_local) 128]); a duplicated key/value head's columns hold
+ * that shard's share of its gradient. ws >= tp_workspace_bytes(TP_WS_ATTN_BWD,
+ * M, h, 0, N). */
+tp_status tp_attn_backward_gqa(const uint16_t* X, int64_t batch, int64_t seq,
+                               int64_t h, int64_t n_q, int64_t n_kv, int causal,
+                               int n_shards, const uint16_t* Wqkv_shards,
+                               const uint16_t* bqkv_shards,
+                               const uint16_t* Wo_shards, const uint16_t* dY,
+                               int residual, void* ws, size_t ws_bytes,
+                               uint16_t* dX, float* dWqkv_shards,
+                               float* dbqkv_shards, float* dWo_shards,
+                               float* dbo, void* stream);
+
 /* tp_attn_forward - Y = concat_heads(attention) W_O + b_O + residual by the
  * tensor-parallel route: QKV column-parallel by whole heads (+ bias), local
  * attention per shard, W_O row-parallel into N partials, one sum

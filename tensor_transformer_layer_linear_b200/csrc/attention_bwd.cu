@@ -10,8 +10,10 @@
 //   dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d),
 // where P is rebuilt from the forward's log-sum-exp.
 //
-// One CTA per (shard, sequence, head, 128-key block), 16 warps, stepping
-// through the sequence's 64-query blocks:
+// One CTA per (shard, sequence, key/value head, 128-key block), 16 warps,
+// stepping through the 64-query blocks of every query head that uses the
+// key/value head (one for multi-head attention, the group for grouped-query
+// attention: the key block's dK and dV sum over the group):
 //   warp 0     TMA: the key block's K and V once, then each query block's Q
 //              and dO into a 4-deep ring (128-byte swizzle), straight out of
 //              the QKV projection's [shard][token][3h/N] output and dO, and
@@ -84,7 +86,10 @@ static_assert(AB_DONE < AB_NUM_BARS, "barrier count");
 
 struct AttnBwdParams {
   int seq, batch, hps, causal, nq;
-  int hs;        // columns of one projection per shard (hps x 128)
+  int kvl;       // key/value heads per shard
+  int group;     // local query heads per local key/value head
+  int q_w;       // query columns per shard (hps x 128)
+  int ld;        // QKV row width per shard: q_w + 2 kvl x 128
   long long M;   // tokens per shard
   long long stride;  // M + 128: per-head row length of lse, D and dq_acc
   float scale_log2, scale;
@@ -116,16 +121,22 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int y = blockIdx.x;
-  const int head = y % p.hps;
-  const int sidx = (y / p.hps) % p.batch;
-  const int g = y / (p.hps * p.batch);
+  const int kvh = y % p.kvl;  // local key/value head
+  const int sidx = (y / p.kvl) % p.batch;
+  const int g = y / (p.kvl * p.batch);
   const int j = blockIdx.y;  // key block
   const int kv0 = j * AB_BK;
   const int row_base = sidx * p.seq;
   // first query block that sees a key of this block (causal: queries >= kv0)
   const int i_first = p.causal ? kv0 / AB_BQ : 0;
-  const int n_it = p.nq - i_first;
-  const int64_t hb = static_cast<int64_t>(g) * p.hps + head;  // (shard, head)
+  const int n_qb = p.nq - i_first;  // query blocks per query head
+  const int n_it = p.group * n_qb;  // (query head of the group, query block) steps
+  // step t: query head kvh * group + t / n_qb (local), query block i_first + t % n_qb
+  auto step_head = [&](int t) { return kvh * p.group + t / n_qb; };
+  auto step_block = [&](int t) { return i_first + t % n_qb; };
+  auto head_row = [&](int t) {  // (shard, query head) row of lse, D and dq_acc
+    return static_cast<int64_t>(g) * p.hps + step_head(t);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(AB_KV), 1);
@@ -159,14 +170,12 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA
     bool ok = true;
-    const int kcol = p.hs + head * AB_D, vcol = 2 * p.hs + head * AB_D;
+    const int kcol = p.q_w + kvh * AB_D, vcol = p.q_w + p.kvl * AB_D + kvh * AB_D;
     mbar_arrive_expect_tx(bar(AB_KV), 2 * AB_KTILE);
     tma_load_3d(s0 + AOFF_K, &tm_kv, bar(AB_KV), kcol, row_base + kv0, g);
     tma_load_3d(s0 + AOFF_K + AB_KSUB, &tm_kv, bar(AB_KV), kcol + 64, row_base + kv0, g);
     tma_load_3d(s0 + AOFF_V, &tm_kv, bar(AB_KV), vcol, row_base + kv0, g);
     tma_load_3d(s0 + AOFF_V + AB_KSUB, &tm_kv, bar(AB_KV), vcol + 64, row_base + kv0, g);
-    const float* lse_h = p.lse + hb * p.stride + row_base;
-    const float* d_h = p.dsum + hb * p.stride + row_base;
     int issued = 0, ld_issued = 0;
     for (int it = 0; it < n_it; ++it) {
       const int st = it % AB_NST;
@@ -175,14 +184,15 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         ok = false;
         break;
       }
-      const int q0 = (i_first + it) * AB_BQ;
+      const int q0 = step_block(it) * AB_BQ;
       const int qrow = row_base + q0;
+      const int qcol = step_head(it) * AB_D;
       const uint32_t qd = s0 + AOFF_Q + st * AB_QTILE, dd = s0 + AOFF_DO + st * AB_QTILE;
       mbar_arrive_expect_tx(bar(AB_QFULL + st), 2 * AB_QTILE);
-      tma_load_3d(qd, &tm_q, bar(AB_QFULL + st), head * AB_D, qrow, g);
-      tma_load_3d(qd + AB_QSUB, &tm_q, bar(AB_QFULL + st), head * AB_D + 64, qrow, g);
-      tma_load_3d(dd, &tm_do, bar(AB_QFULL + st), head * AB_D, qrow, g);
-      tma_load_3d(dd + AB_QSUB, &tm_do, bar(AB_QFULL + st), head * AB_D + 64, qrow, g);
+      tma_load_3d(qd, &tm_q, bar(AB_QFULL + st), qcol, qrow, g);
+      tma_load_3d(qd + AB_QSUB, &tm_q, bar(AB_QFULL + st), qcol + 64, qrow, g);
+      tma_load_3d(dd, &tm_do, bar(AB_QFULL + st), qcol, qrow, g);
+      tma_load_3d(dd + AB_QSUB, &tm_do, bar(AB_QFULL + st), qcol + 64, qrow, g);
       ++issued;
       if (p.ld_bulk) {
         const int ls = it & 1;
@@ -191,9 +201,10 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
           break;
         }
         const uint32_t ld = s0 + AOFF_LD + ls * (2 * AB_BQ * 4);
+        const int64_t lrow = head_row(it) * p.stride + row_base + q0;
         mbar_arrive_expect_tx(bar(AB_LDFULL + ls), 2 * AB_BQ * 4);
-        bulk_load(ld, lse_h + q0, AB_BQ * 4, bar(AB_LDFULL + ls));
-        bulk_load(ld + AB_BQ * 4, d_h + q0, AB_BQ * 4, bar(AB_LDFULL + ls));
+        bulk_load(ld, p.lse + lrow, AB_BQ * 4, bar(AB_LDFULL + ls));
+        bulk_load(ld + AB_BQ * 4, p.dsum + lrow, AB_BQ * 4, bar(AB_LDFULL + ls));
         ++ld_issued;
       }
     }
@@ -300,11 +311,11 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     const int key = kv0 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(rq * 32) << 16;
     const float sl2 = p.scale_log2;
-    const float* lse_h = p.lse + hb * p.stride + row_base;
-    const float* d_h = p.dsum + hb * p.stride + row_base;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int b = it & 1;
+      const float* lse_h = p.lse + head_row(it) * p.stride + row_base;
+      const float* d_h = p.dsum + head_row(it) * p.stride + row_base;
       if (!mbar_wait(bar(AB_SDP + b), (it >> 1) & 1, abort_flag) ||
           (p.ld_bulk && !mbar_wait(bar(AB_LDFULL + b), (it >> 1) & 1, abort_flag)) ||
           // dS^T buffer b is free once dK and dQ^T of block it - 2 are done
@@ -313,7 +324,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int i = i_first + it;
+      const int i = step_block(it);
       const int q0 = i * AB_BQ;
       const bool need_mask =
           (p.causal && q0 < kv0 + AB_BK) || q0 + AB_BQ > p.seq || kv0 + AB_BK > p.seq;
@@ -390,8 +401,8 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       tc_fence_after();
       // tcgen05.ld is warp-collective: every lane loads, only rows inside
       // the sequence are stored; each group writes half of the 128 columns
-      uint16_t* base = p.dqkv + (static_cast<int64_t>(g) * p.M + row_base + key) * (3 * p.hs) +
-                       head * AB_D;
+      uint16_t* base = p.dqkv + (static_cast<int64_t>(g) * p.M + row_base + key) * p.ld +
+                       p.q_w + kvh * AB_D;  // dK here, dV kvl x 128 columns further
 #pragma unroll 1
       for (int c = 4 * grp; c < 4 * grp + 4; ++c) {  // 16 columns at a time
         uint32_t kv[16], vv[16];
@@ -414,8 +425,8 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
             wv.y = pack_bf16x2(__uint_as_float(vv[8 * e + 2]), __uint_as_float(vv[8 * e + 3]));
             wv.z = pack_bf16x2(__uint_as_float(vv[8 * e + 4]), __uint_as_float(vv[8 * e + 5]));
             wv.w = pack_bf16x2(__uint_as_float(vv[8 * e + 6]), __uint_as_float(vv[8 * e + 7]));
-            *reinterpret_cast<uint4*>(base + p.hs + c * 16 + 8 * e) = wk;
-            *reinterpret_cast<uint4*>(base + 2 * p.hs + c * 16 + 8 * e) = wv;
+            *reinterpret_cast<uint4*>(base + c * 16 + 8 * e) = wk;
+            *reinterpret_cast<uint4*>(base + p.kvl * AB_D + c * 16 + 8 * e) = wv;
           }
         }
       }
@@ -429,7 +440,6 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     const int dcol = rq * 32 + lane;  // head-dimension column (= TMEM lane)
     const uint32_t lane_addr = static_cast<uint32_t>(rq * 32) << 16;
     // accumulator rows [stride][128]: a warp's 32 lanes cover 128 contiguous bytes
-    float* acc_h = p.dq_acc + (hb * p.stride + row_base) * AB_D + dcol;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int b = it & 1;
@@ -446,9 +456,9 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(AB_DQEMPTY + b));  // the columns may be overwritten now
-      const int q0 = (i_first + it) * AB_BQ;
+      const int q0 = step_block(it) * AB_BQ;
       const int nq_valid = min(AB_BQ, p.seq - q0);
-      float* a = acc_h + static_cast<int64_t>(q0) * AB_D;
+      float* a = p.dq_acc + (head_row(it) * p.stride + row_base + q0) * AB_D + dcol;
 #pragma unroll
       for (int q = 0; q < AB_BQ; ++q)
         if (q < nq_valid) red_add_f32(a + static_cast<int64_t>(q) * AB_D, v[q]);
@@ -503,7 +513,7 @@ __global__ void __launch_bounds__(256) zero_f32x4_kernel(float4* __restrict__ p,
 __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float* __restrict__ acc,
                                                           uint16_t* __restrict__ dqkv, int64_t n,
                                                           int64_t M, int64_t stride, int hps,
-                                                          int hs, float scale) {
+                                                          int ld, float scale) {
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (i >= n) return;
   const int c8 = static_cast<int>(i % (AB_D / 8));
@@ -520,7 +530,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const float* __restric
   w.y = pack_bf16x2(x.z * scale, x.w * scale);
   w.z = pack_bf16x2(y.x * scale, y.y * scale);
   w.w = pack_bf16x2(y.z * scale, y.w * scale);
-  *reinterpret_cast<uint4*>(dqkv + (g * M + tok) * (3 * static_cast<int64_t>(hs)) + head * AB_D +
+  *reinterpret_cast<uint4*>(dqkv + (g * M + tok) * static_cast<int64_t>(ld) + head * AB_D +
                             c8 * 8) = w;
 }
 
@@ -554,19 +564,21 @@ static bool encode_rows(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, c
 }
 
 int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const float* lse,
-                         int64_t batch, int64_t seq, int64_t n_heads, int n_shards, int causal,
-                         void* dQKV, float* dsum, float* dq_acc, cudaStream_t s, unsigned* err,
-                         int num_sms) {
-  const int hps = static_cast<int>(n_heads / n_shards);
-  const int64_t hs = static_cast<int64_t>(hps) * AB_D;
+                         int64_t batch, int64_t seq, int64_t n_q, int64_t kv_local, int n_shards,
+                         int causal, void* dQKV, float* dsum, float* dq_acc, cudaStream_t s,
+                         unsigned* err, int num_sms) {
+  const int hps = static_cast<int>(n_q / n_shards);
+  const int kvl = static_cast<int>(kv_local);
+  const int64_t q_w = static_cast<int64_t>(hps) * AB_D;
+  const int64_t ld = q_w + 2LL * kvl * AB_D;  // QKV row width per shard
   const int64_t M = batch * seq;
   const int64_t stride = M + 128;
   auto enc = bwd_map_encoder();
   if (enc == nullptr) return 1;
   CUtensorMap tm_kv, tm_q, tm_do;
-  if (!encode_rows(enc, &tm_kv, QKV, 3 * hs, M, n_shards, AB_BK)) return 1;
-  if (!encode_rows(enc, &tm_q, QKV, 3 * hs, M, n_shards, AB_BQ)) return 1;
-  if (!encode_rows(enc, &tm_do, dO, hs, M, n_shards, AB_BQ)) return 1;
+  if (!encode_rows(enc, &tm_kv, QKV, ld, M, n_shards, AB_BK)) return 1;
+  if (!encode_rows(enc, &tm_q, QKV, ld, M, n_shards, AB_BQ)) return 1;
+  if (!encode_rows(enc, &tm_do, dO, q_w, M, n_shards, AB_BQ)) return 1;
 
   const int64_t heads_total = static_cast<int64_t>(n_shards) * hps;
   // dQ accumulator to zero, D = rowsum(dO * O)
@@ -585,7 +597,10 @@ int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const f
   p.hps = hps;
   p.causal = causal;
   p.nq = static_cast<int>((seq + AB_BQ - 1) / AB_BQ);
-  p.hs = static_cast<int>(hs);
+  p.kvl = kvl;
+  p.group = hps / kvl;
+  p.q_w = static_cast<int>(q_w);
+  p.ld = static_cast<int>(ld);
   p.M = M;
   p.stride = stride;
   p.scale = 1.0f / sqrtf(static_cast<float>(AB_D));
@@ -598,13 +613,13 @@ int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const f
   p.err = err;
   cudaFuncSetAttribute(attention_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        AB_SMEM);
-  const dim3 grid(static_cast<unsigned>(heads_total * batch),
+  const dim3 grid(static_cast<unsigned>(static_cast<int64_t>(n_shards) * kvl * batch),
                   static_cast<unsigned>((seq + AB_BK - 1) / AB_BK));
   attention_bwd_tc_kernel<<<grid, AB_THREADS, AB_SMEM, s>>>(tm_kv, tm_q, tm_do, p);
 
   const int64_t n = heads_total * M * (AB_D / 8);
   attn_bwd_dq_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
-      dq_acc, static_cast<uint16_t*>(dQKV), n, M, stride, hps, static_cast<int>(hs), p.scale);
+      dq_acc, static_cast<uint16_t*>(dQKV), n, M, stride, hps, static_cast<int>(ld), p.scale);
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
 

@@ -931,8 +931,9 @@ tp_status tp_attention_backward(const uint16_t* QKV_shards, const uint16_t* O_sh
                                            round256(static_cast<size_t>(h) / 128 * rows * 4));
   TraceScope ts(tpk::KID_ATTENTION_BWD, as_stream(stream));
   const int rc = tpk::launch_attention_bwd(QKV_shards, O_shards, dO_shards, lse, batch, seq,
-                                           n_heads, n_shards, causal ? 1 : 0, dQKV_shards, dsum,
-                                           dq_acc, as_stream(stream), d.err, d.num_sms);
+                                           n_heads, n_heads / n_shards, n_shards, causal ? 1 : 0,
+                                           dQKV_shards, dsum, dq_acc, as_stream(stream), d.err,
+                                           d.num_sms);
   return rc == 0 ? TP_OK : TP_ERR_CUDA;
 }
 
@@ -966,34 +967,43 @@ static AttnBwdBufs attn_bwd_layout(void* ws, size_t M, size_t H, size_t N) {
 // the weight and bias gradients, and last the N partials
 // dX_i = dQKV_i W_QKV,i^T in b.part.
 static tp_status attn_backward_core(const DevInfo& d, void* stream, const uint16_t* X,
-                                    int64_t batch, int64_t seq, int64_t h, int64_t n_heads,
-                                    int causal, int n_shards, const uint16_t* Wqkv_shards,
-                                    const uint16_t* Wo_shards, const uint16_t* dY,
-                                    const AttnBwdBufs& b, float* dWqkv_shards, float* dbqkv_shards,
-                                    float* dWo_shards, float* dbo) {
+                                    int64_t batch, int64_t seq, int64_t h, int64_t n_q,
+                                    int64_t n_kv, int causal, int n_shards,
+                                    const uint16_t* Wqkv_shards, const uint16_t* Wo_shards,
+                                    const uint16_t* dY, const AttnBwdBufs& b, float* dWqkv_shards,
+                                    float* dbqkv_shards, float* dWo_shards, float* dbo) {
   cudaStream_t s = as_stream(stream);
   const int M = static_cast<int>(batch * seq), H = static_cast<int>(h);
-  const int hs = H / n_shards;
+  const int hs = H / n_shards;  // query (and output) columns per shard
+  const int64_t kvl = gqa_kv_local(n_kv, n_shards);
+  const int qkv_w = hs + 2 * static_cast<int>(kvl) * 128;  // QKV columns per shard
   // dO_i = dY W_O,i^T; Wo_shards[i] = W_O,i^T is the MN-major operand
   tp_status st = bwd_gemm(d, s, n_shards, dY, false, false, Wo_shards, true, true, b.dO, M, hs,
                           H, false);
   if (st != TP_OK) return st;
-  st = tp_attention_backward(b.qkv, b.o, b.dO, b.lse, batch, seq, h, n_heads, causal, n_shards,
-                             b.core, attn_core_bwd_bytes(M, H), b.dqkv, stream);
-  if (st != TP_OK) return st;
+  {
+    const size_t rows = static_cast<size_t>(M) + 128;
+    float* dsum = static_cast<float*>(b.core);
+    float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(b.core) +
+                                             round256(static_cast<size_t>(n_q) * rows * 4));
+    TraceScope ts(tpk::KID_ATTENTION_BWD, s);
+    if (tpk::launch_attention_bwd(b.qkv, b.o, b.dO, b.lse, batch, seq, n_q, kvl, n_shards,
+                                  causal ? 1 : 0, b.dqkv, dsum, dq_acc, s, d.err, d.num_sms) != 0)
+      return TP_ERR_CUDA;
+  }
   // dW_QKV,i^T = dQKV_i^T X (packed like Wqkv_shards), dW_O,i^T = dY^T O_i (like Wo_shards)
-  st = bwd_gemm(d, s, n_shards, b.dqkv, true, true, X, false, true, dWqkv_shards, 3 * hs, H, M,
+  st = bwd_gemm(d, s, n_shards, b.dqkv, true, true, X, false, true, dWqkv_shards, qkv_w, H, M,
                 true);
   if (st != TP_OK) return st;
   st = bwd_gemm(d, s, n_shards, dY, false, true, b.o, true, true, dWo_shards, H, hs, M, true);
   if (st != TP_OK) return st;
-  st = bwd_colsum(d, s, b.dqkv, n_shards, M, 3 * hs, b.slabs, dbqkv_shards);
+  st = bwd_colsum(d, s, b.dqkv, n_shards, M, qkv_w, b.slabs, dbqkv_shards);
   if (st != TP_OK) return st;
   st = bwd_colsum(d, s, dY, 1, M, H, b.slabs, dbo);
   if (st != TP_OK) return st;
   // dX partials: dQKV_i W_QKV,i^T; Wqkv_shards[i] = W_QKV,i^T is the MN-major operand
   return bwd_gemm(d, s, n_shards, b.dqkv, true, false, Wqkv_shards, true, true, b.part, M, H,
-                  3 * hs, true);
+                  qkv_w, true);
 }
 
 static bool attn_bwd_shape_ok(int64_t batch, int64_t seq, int64_t h, int64_t n_heads,
@@ -1031,8 +1041,9 @@ tp_status tp_attn_backward(const uint16_t* X, int64_t batch, int64_t seq, int64_
   if (st != TP_OK) return st;
   st = tp_attention_lse(b.qkv, batch, seq, h, n_heads, causal, n_shards, b.o, b.lse, stream);
   if (st != TP_OK) return st;
-  st = attn_backward_core(d, stream, X, batch, seq, h, n_heads, causal, n_shards, Wqkv_shards,
-                          Wo_shards, dY, b, dWqkv_shards, dbqkv_shards, dWo_shards, dbo);
+  st = attn_backward_core(d, stream, X, batch, seq, h, n_heads, n_heads, causal, n_shards,
+                          Wqkv_shards, Wo_shards, dY, b, dWqkv_shards, dbqkv_shards, dWo_shards,
+                          dbo);
   if (st != TP_OK) return st;
   // the one reduction of the block's backward: dX = sum_i dX_i (+ dY)
   return tp_reduce_partials(b.part, n_shards, M, h, nullptr, residual ? dY : nullptr, dX, stream);
@@ -1143,13 +1154,105 @@ tp_status tp_layer_backward(const uint16_t* X, int64_t batch, int64_t seq, int64
   if (st != TP_OK) return st;
   // attention block: gradients and the partials of dx1; its one reduction is
   // fused with LN1's backward and the residual: dX = dh1 + LN1'(X)^T sum_i dx1_i
-  st = attn_backward_core(d, stream, x1, batch, seq, h, n_heads, 1, n_shards, w->Wqkv_shards,
-                          w->Wo_shards, dh1, ab, g->Wqkv_shards, g->bqkv_shards, g->Wo_shards,
-                          g->bo);
+  st = attn_backward_core(d, stream, x1, batch, seq, h, n_heads, n_heads, 1, n_shards,
+                          w->Wqkv_shards, w->Wo_shards, dh1, ab, g->Wqkv_shards, g->bqkv_shards,
+                          g->Wo_shards, g->bo);
   if (st != TP_OK) return st;
   return tp_reduce_partials_layernorm_backward(ab.part, n_shards, M, h, X, w->ln1_gamma, dh1,
                                                ln_eps, lnb, lnb_bytes, dX, g->ln1_gamma,
                                                g->ln1_beta, stream);
 }
 
+
+tp_status tp_attention_gqa_lse(const uint16_t* QKV_shards, int64_t batch, int64_t seq,
+                               int64_t n_q, int64_t n_kv, int64_t head_dim, int causal,
+                               int n_shards, uint16_t* O_shards, float* lse, void* stream) {
+  if (QKV_shards == nullptr || O_shards == nullptr || lse == nullptr) return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || !gqa_ok(n_q, n_kv, n_shards)) return TP_ERR_SHAPE;
+  if (head_dim != 128) return TP_ERR_UNSUPPORTED;
+  if (batch * seq > kIntMax || seq > kIntMax) return TP_ERR_SHAPE;
+  if (static_cast<int64_t>(n_shards) * batch * (n_q / n_shards) > 65535) return TP_ERR_SHAPE;
+  if (!al16(QKV_shards) || !al16(O_shards) || !al16(lse)) return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
+  const int rc = tpk::launch_attention(QKV_shards, batch, seq, n_q, gqa_kv_local(n_kv, n_shards),
+                                       n_shards, causal ? 1 : 0, O_shards, as_stream(stream),
+                                       d.err, lse);
+  return rc == 0 ? TP_OK : (rc == 3 ? TP_ERR_UNSUPPORTED : TP_ERR_CUDA);
+}
+
+tp_status tp_attention_gqa_backward(const uint16_t* QKV_shards, const uint16_t* O_shards,
+                                    const uint16_t* dO_shards, const float* lse, int64_t batch,
+                                    int64_t seq, int64_t n_q, int64_t n_kv, int64_t head_dim,
+                                    int causal, int n_shards, void* ws, size_t ws_bytes,
+                                    uint16_t* dQKV_shards, void* stream) {
+  if (QKV_shards == nullptr || O_shards == nullptr || dO_shards == nullptr || lse == nullptr ||
+      dQKV_shards == nullptr || ws == nullptr)
+    return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || !gqa_ok(n_q, n_kv, n_shards)) return TP_ERR_SHAPE;
+  if (head_dim != 128) return TP_ERR_UNSUPPORTED;
+  if (batch * seq > kIntMax || seq > kIntMax) return TP_ERR_SHAPE;
+  const int64_t M = batch * seq;
+  const int64_t hq = n_q * head_dim;  // query columns over all shards
+  if (ws_bytes < tp_workspace_bytes(TP_WS_ATTN_CORE_BWD, M, hq, 0, n_shards))
+    return TP_ERR_WORKSPACE;
+  if (!al16(QKV_shards) || !al16(O_shards) || !al16(dO_shards) || !al16(lse) ||
+      !al16(dQKV_shards) || !al16(ws))
+    return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  const size_t rows = static_cast<size_t>(M) + 128;
+  float* dsum = static_cast<float*>(ws);
+  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                           round256(static_cast<size_t>(n_q) * rows * 4));
+  TraceScope ts(tpk::KID_ATTENTION_BWD, as_stream(stream));
+  const int rc = tpk::launch_attention_bwd(QKV_shards, O_shards, dO_shards, lse, batch, seq, n_q,
+                                           gqa_kv_local(n_kv, n_shards), n_shards,
+                                           causal ? 1 : 0, dQKV_shards, dsum, dq_acc,
+                                           as_stream(stream), d.err, d.num_sms);
+  return rc == 0 ? TP_OK : TP_ERR_CUDA;
+}
+
+tp_status tp_attn_backward_gqa(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
+                               int64_t n_q, int64_t n_kv, int causal, int n_shards,
+                               const uint16_t* Wqkv_shards, const uint16_t* bqkv_shards,
+                               const uint16_t* Wo_shards, const uint16_t* dY, int residual,
+                               void* ws, size_t ws_bytes, uint16_t* dX, float* dWqkv_shards,
+                               float* dbqkv_shards, float* dWo_shards, float* dbo,
+                               void* stream) {
+  if (X == nullptr || Wqkv_shards == nullptr || Wo_shards == nullptr || dY == nullptr ||
+      dX == nullptr || dWqkv_shards == nullptr || dbqkv_shards == nullptr ||
+      dWo_shards == nullptr || dbo == nullptr || ws == nullptr)
+    return TP_ERR_NULL;
+  if (batch <= 0 || seq <= 0 || h <= 0 || !gqa_ok(n_q, n_kv, n_shards)) return TP_ERR_SHAPE;
+  if (h % n_q || h / n_q != 128) return TP_ERR_UNSUPPORTED;
+  if (batch * seq > kIntMax || seq > kIntMax) return TP_ERR_SHAPE;
+  if (static_cast<int64_t>(n_shards) * batch * (n_q / n_shards) > 65535) return TP_ERR_SHAPE;
+  const int64_t M = batch * seq;
+  // the attention workspace holds 3h QKV columns, which covers GQA (N <= n_q)
+  if (ws_bytes < tp_workspace_bytes(TP_WS_ATTN_BWD, M, h, 0, n_shards)) return TP_ERR_WORKSPACE;
+  if (!al16(ws) || !al16(X) || !al16(Wqkv_shards) || !al16(Wo_shards) || !al16(dY) ||
+      !al16(dX) || !al16(dWqkv_shards) || !al16(dbqkv_shards) || !al16(dWo_shards) ||
+      !al16(dbo) || (bqkv_shards && !al16(bqkv_shards)))
+    return TP_ERR_ALIGN;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  const AttnBwdBufs b = attn_bwd_layout(ws, M, h, n_shards);
+  const int64_t qkv_cols = n_shards * (n_q / n_shards + 2 * gqa_kv_local(n_kv, n_shards)) * 128;
+  // recompute the forward: QKV_i, O_i and the lse
+  st = tp_column_linear(X, M, h, Wqkv_shards, bqkv_shards, qkv_cols, n_shards, TP_ACT_NONE,
+                        b.qkv, stream);
+  if (st != TP_OK) return st;
+  st = tp_attention_gqa_lse(b.qkv, batch, seq, n_q, n_kv, 128, causal, n_shards, b.o, b.lse,
+                            stream);
+  if (st != TP_OK) return st;
+  st = attn_backward_core(d, stream, X, batch, seq, h, n_q, n_kv, causal, n_shards, Wqkv_shards,
+                          Wo_shards, dY, b, dWqkv_shards, dbqkv_shards, dWo_shards, dbo);
+  if (st != TP_OK) return st;
+  return tp_reduce_partials(b.part, n_shards, M, h, nullptr, residual ? dY : nullptr, dX, stream);
+}
 }  // extern "C"

@@ -91,14 +91,15 @@ int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, i
                      int n_shards, int causal, void* O, cudaStream_t s, unsigned* err,
                      float* lse = nullptr);
 
-// Attention backward of every shard's heads (n_kv = n_q, head_dim 128):
-// dQKV [N][M][3 hs] (packed like QKV) from QKV, O, dO [N][M][hs] and the
-// forward's lse. dsum [n_heads][M + 128] fp32 and dq_acc
-// [n_heads][128][M + 128] fp32 are scratch.
+// Attention backward of every shard's heads (head_dim 128; n_q/N query heads
+// and kv_local key/value heads per shard, laid out like the forward's QKV):
+// dQKV (packed like QKV) from QKV, O, dO [N][M][n_q/N x 128] and the
+// forward's lse. dsum [n_q][M + 128] fp32 and dq_acc [n_q][M + 128][128]
+// fp32 are scratch.
 int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const float* lse,
-                         int64_t batch, int64_t seq, int64_t n_heads, int n_shards, int causal,
-                         void* dQKV, float* dsum, float* dq_acc, cudaStream_t s, unsigned* err,
-                         int num_sms);
+                         int64_t batch, int64_t seq, int64_t n_q, int64_t kv_local, int n_shards,
+                         int causal, void* dQKV, float* dsum, float* dq_acc, cudaStream_t s,
+                         unsigned* err, int num_sms);
 
 // out[i][c][r] = W[row(i, r)][col(i, c)] for the split kinds (kind 4: GQA
 // QKV with n_q query and n_kv key/value heads of head_dim).

@@ -89,6 +89,12 @@ _SIGS = {
     "tp_layer_backward": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32,
                                  ctypes.POINTER(tp_layer_weights), _f32, _vp, _vp, _sz, _vp,
                                  ctypes.POINTER(tp_layer_grads), _vp]),
+    "tp_attention_gqa_lse": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp,
+                                    _vp]),
+    "tp_attention_gqa_backward": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i32,
+                                         _i32, _vp, _sz, _vp, _vp]),
+    "tp_attn_backward_gqa": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp,
+                                    _vp, _i32, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _vp]),
     "tp_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "tp_get_last_error": (_i32, [_vp]),
     "tp_status_string": (ctypes.c_char_p, [_i32]),
@@ -341,6 +347,31 @@ def tp_layer_backward(X, batch, seq, h, n_heads, ffn, n_shards, weights: tp_laye
     _check(lib.tp_layer_backward(_p(X), batch, seq, h, n_heads, ffn, n_shards,
                                  ctypes.byref(weights), ln_eps, _p(dY), _p(ws), ws_bytes, _p(dX),
                                  ctypes.byref(grads), _s(stream)), "tp_layer_backward")
+
+
+def tp_attention_gqa_lse(QKV_shards, batch, seq, n_q, n_kv, head_dim, causal, n_shards, O_shards,
+                         lse, stream=None):
+    _check(lib.tp_attention_gqa_lse(_p(QKV_shards), batch, seq, n_q, n_kv, head_dim,
+                                    int(bool(causal)), n_shards, _p(O_shards), _p(lse), _s(stream)),
+           "tp_attention_gqa_lse")
+
+
+def tp_attention_gqa_backward(QKV_shards, O_shards, dO_shards, lse, batch, seq, n_q, n_kv,
+                              head_dim, causal, n_shards, ws, ws_bytes, dQKV_shards, stream=None):
+    _check(lib.tp_attention_gqa_backward(_p(QKV_shards), _p(O_shards), _p(dO_shards), _p(lse),
+                                         batch, seq, n_q, n_kv, head_dim, int(bool(causal)),
+                                         n_shards, _p(ws), ws_bytes, _p(dQKV_shards), _s(stream)),
+           "tp_attention_gqa_backward")
+
+
+def tp_attn_backward_gqa(X, batch, seq, h, n_q, n_kv, causal, n_shards, Wqkv_shards, bqkv_shards,
+                         Wo_shards, dY, residual, ws, ws_bytes, dX, dWqkv_shards, dbqkv_shards,
+                         dWo_shards, dbo, stream=None):
+    _check(lib.tp_attn_backward_gqa(_p(X), batch, seq, h, n_q, n_kv, int(bool(causal)), n_shards,
+                                    _p(Wqkv_shards), _p(bqkv_shards), _p(Wo_shards), _p(dY),
+                                    int(bool(residual)), _p(ws), ws_bytes, _p(dX),
+                                    _p(dWqkv_shards), _p(dbqkv_shards), _p(dWo_shards), _p(dbo),
+                                    _s(stream)), "tp_attn_backward_gqa")
 
 
 def tp_get_last_error(stream=None) -> int:

@@ -10,7 +10,7 @@ import pytest
 from oracle import tp_oracle as O
 from tensor_transformer_layer_linear_b200 import synth
 
-from helpers import assert_parity, f64, from_dev_bf16, to_dev
+from helpers import BWD_FRO_REL, assert_parity, f64, from_dev_bf16, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -117,3 +117,84 @@ def test_gqa_rejects_bad_group_split(tp):
     with pytest.raises(tp.TPError) as e:
         tp.tp_shard_qkv_gqa(X, 8, 8, 4, 16, 6, X)              # N = 6 vs n_kv = 4
     assert e.value.status == tp.TP_ERR_SHAPE
+
+
+# ---------------------------------------------------------------- backward
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("n_q,n_kv,n,seq", [(4, 2, 1, 256), (4, 2, 2, 200), (4, 2, 4, 192),
+                                            (4, 1, 2, 130), (8, 2, 2, 128)])
+def test_gqa_attention_backward_kernel(tp, n_q, n_kv, n, seq, causal):
+    """Per shard, against the oracle's grouped backward on the shard's own
+    query and (possibly duplicated) key/value heads."""
+    rng = np.random.default_rng(1400 + n_q + n_kv + n + seq)
+    batch, d = 2, 128
+    qs, kvl = n_q // n, _kvl(n_kv, n)
+    M = batch * seq
+    QKV = _bits(rng, (n, M, (qs + 2 * kvl) * d))
+    dO = _bits(rng, (n, M, qs * d))
+    O_ = torch.empty((n, M, qs * d), dtype=torch.int16, device="cuda")
+    lse = torch.empty(n_q * (M + 128), dtype=torch.float32, device="cuda")
+    qkv_d = to_dev(QKV)
+    tp.tp_attention_gqa_lse(qkv_d, batch, seq, n_q, n_kv, d, causal, n, O_, lse)
+    nb = tp.tp_workspace_bytes(tp.TP_WS_ATTN_CORE_BWD, M, n_q * d, 0, n)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    dQKV = torch.empty_like(qkv_d)
+    tp.tp_attention_gqa_backward(qkv_d, O_, to_dev(dO), lse, batch, seq, n_q, n_kv, d, causal, n,
+                                 ws, nb, dQKV)
+    assert tp.tp_get_last_error() == tp.TP_OK
+    got = from_dev_bf16(dQKV)
+    for i in range(n):
+        q = f64(QKV[i][:, :qs * d])
+        k = f64(QKV[i][:, qs * d:(qs + kvl) * d])
+        v = f64(QKV[i][:, (qs + kvl) * d:])
+        dq, dk, dv = O.gqa_attention_heads_backward(q, k, v, f64(dO[i]), batch, seq, qs, kvl, causal)
+        assert_parity(got[i][:, :qs * d], dq, f"dQ shard {i}")
+        assert_parity(got[i][:, qs * d:(qs + kvl) * d], dk, f"dK shard {i}")
+        assert_parity(got[i][:, (qs + kvl) * d:], dv, f"dV shard {i}")
+
+
+@pytest.mark.parametrize("n_q,n_kv,n", [(4, 2, 1), (4, 2, 2), (4, 2, 4), (8, 2, 4), (4, 4, 2)])
+def test_gqa_block_backward(tp, n_q, n_kv, n):
+    """The grouped-query block's backward against the oracle: dX, dW_O, the
+    biases, the packed per-shard QKV weight gradients, and (N > n_kv) the sum
+    over the replicas of a duplicated key/value head."""
+    rng = np.random.default_rng(1500 + n_q + n_kv + n)
+    batch, seq, d = 2, 192, 128
+    h = n_q * d
+    M = batch * seq
+    cfg = dict(kind="attn_gqa", batch=batch, seq=seq, h=h, n_heads=n_q, n_kv_heads=n_kv,
+               x_std=1.0, w_std=0.05, b_std=0.05)
+    inp = synth.make_inputs(cfg, seed=20 + n)
+    dY = _bits(rng, (M, h))
+    Wqkv_s, cols = _pack(tp, inp["Wqkv"], h, n_q, n_kv, d, n)
+    bqkv_s, _ = _pack(tp, inp["bqkv"].reshape(1, -1), 1, n_q, n_kv, d, n)
+    Wo_s = torch.empty(h * h, dtype=torch.int16, device="cuda")
+    tp.tp_shard_weights(to_dev(inp["Wo"]), h, h, n, 1, 0, Wo_s)
+    nb = tp.tp_workspace_bytes(tp.TP_WS_ATTN_BWD, M, h, 0, n)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    dX = torch.empty((M, h), dtype=torch.int16, device="cuda")
+    dW = torch.empty((n, cols, h), dtype=torch.float32, device="cuda")
+    db = torch.empty((n, cols), dtype=torch.float32, device="cuda")
+    dWo = torch.empty((n, h, h // n), dtype=torch.float32, device="cuda")
+    dbo = torch.empty(h, dtype=torch.float32, device="cuda")
+    tp.tp_attn_backward_gqa(to_dev(inp["X"]), batch, seq, h, n_q, n_kv, True, n, Wqkv_s, bqkv_s,
+                            Wo_s, to_dev(dY), True, ws, nb, dX, dW, db, dWo, dbo)
+    assert tp.tp_get_last_error() == tp.TP_OK
+    ref = O.gqa_self_attention_backward_sharded(f64(inp["X"]), f64(inp["Wqkv"]), f64(inp["bqkv"]),
+                                                f64(inp["Wo"]), f64(inp["bo"]), f64(dY), batch,
+                                                seq, n_q, n_kv, n)
+    # backward gate: grouped key/value gradients add the group's rounding
+    assert_parity(from_dev_bf16(dX), ref["dX"], "dX", fro_rel=BWD_FRO_REL)
+    gW = dW.cpu().numpy().astype(np.float64)
+    gb = db.cpu().numpy().astype(np.float64)
+    assert_parity(gW, ref["dWqkv_packed"], "dWqkv (per shard)", fro_rel=BWD_FRO_REL)
+    assert_parity(gb, ref["dbqkv_packed"], "dbqkv (per shard)", fro_rel=BWD_FRO_REL)
+    assert_parity(dWo.cpu().numpy().astype(np.float64), O.packed_shards(ref["dWo"], O.SPLIT_ROW, n),
+                  "dWo")
+    assert_parity(dbo.cpu().numpy().astype(np.float64), ref["dbo"], "dbo")
+    # the replicas' shares add up to the logical gradient
+    logical = np.zeros_like(ref["dWqkv"])
+    for i, c in enumerate(O.gqa_shard_columns(n_q, n_kv, d, n)):
+        np.add.at(logical.T, c, gW[i])
+    assert_parity(logical, ref["dWqkv"], "dWqkv (replicas summed)", fro_rel=BWD_FRO_REL)
