@@ -97,7 +97,8 @@ typedef enum {
 
 typedef enum {
     TP_WS_MLP = 0, TP_WS_ATTN = 1, TP_WS_LAYER = 2, TP_WS_LAYER_SP = 3, TP_WS_MLP_BWD = 4,
-    TP_WS_ATTN_CORE_BWD = 5, TP_WS_ATTN_BWD = 6, TP_WS_LAYER_BWD = 7, TP_WS_LN_BWD = 8
+    TP_WS_ATTN_CORE_BWD = 5, TP_WS_ATTN_BWD = 6, TP_WS_LAYER_BWD = 7, TP_WS_LN_BWD = 8,
+    TP_WS_LAYER_BWD_SP = 9
 } tp_ws_kind;
 
 /* Weights of one pre-LN layer, all device pointers in the packed shard
@@ -402,6 +403,21 @@ tp_status tp_attn_backward_gqa(const uint16_t* X, int64_t batch, int64_t seq,
                                float* dbqkv_shards, float* dWo_shards,
                                float* dbo, void* stream);
 
+/* tp_layer_backward_sp - tp_layer_backward under sequence parallelism: X,
+ * dY and dX in the sequence-sharded layout [N][batch][seq/N][h] of
+ * tp_layer_forward_sp ([TP-LLM] "Sequence Parallelism"). The backward swaps
+ * the forward's collectives: dY and dh1 are all-gathered before each block,
+ * and each block's one reduction is a reduce-scatter fused with the LN
+ * backward and the residual. Gradients as tp_layer_backward.
+ * ws >= tp_workspace_bytes(TP_WS_LAYER_BWD_SP, batch*seq, h, F, N). */
+tp_status tp_layer_backward_sp(const uint16_t* X_shards, int64_t batch,
+                               int64_t seq, int64_t h, int64_t n_heads,
+                               int64_t ffn, int n_shards,
+                               const tp_layer_weights* w, float ln_eps,
+                               const uint16_t* dY_shards, void* ws,
+                               size_t ws_bytes, uint16_t* dX_shards,
+                               const tp_layer_grads* g, void* stream);
+
 /* tp_attn_forward - Y = concat_heads(attention) W_O + b_O + residual by the
  * tensor-parallel route: QKV column-parallel by whole heads (+ bias), local
  * attention per shard, W_O row-parallel into N partials, one sum
@@ -537,7 +553,8 @@ tp_status tp_mlp_forward_noalloc(const uint16_t* X, int64_t B, int64_t h,
  * (TP_WS_ATTN, ffn ignored), tp_layer_forward (TP_WS_LAYER),
  * tp_layer_forward_sp (TP_WS_LAYER_SP), tp_mlp_backward (TP_WS_MLP_BWD),
  * tp_attention_backward (TP_WS_ATTN_CORE_BWD, ffn ignored), tp_attn_backward
- * (TP_WS_ATTN_BWD, ffn ignored), tp_layer_backward (TP_WS_LAYER_BWD) or
+ * (TP_WS_ATTN_BWD, ffn ignored), tp_layer_backward (TP_WS_LAYER_BWD),
+ * tp_layer_backward_sp (TP_WS_LAYER_BWD_SP) or
  * tp_reduce_partials_layernorm_backward (TP_WS_LN_BWD, tokens and ffn ignored).
  * tokens = batch * seq. Returns 0 for invalid arguments. */
 size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn,

@@ -823,6 +823,63 @@ def transformer_layer_sp(X_slices: list, p: dict, batch: int, seq: int,
     return reduce_scatter_partials(P_i, batch, seq, n_shards, p["b2"], h1)
 
 
+def transformer_layer_sp_backward(X_slices: list, p: dict, dY_slices: list,
+                                  batch: int, seq: int, n_heads: int,
+                                  n_shards: int, eps: float = 1e-5,
+                                  causal: bool = True) -> dict:
+    """Backward of transformer_layer_sp: each forward all-gather becomes a
+    reduce-scatter and each reduce-scatter an all-gather. dY's slices are
+    all-gathered for the MLP block; its partial input gradients are
+    reduce-scattered into the slices, where LN2's backward and the residual
+    give dh1; dh1 is all-gathered for the attention block, whose partials are
+    reduce-scattered, LN1's backward applied on the slices and dh1 added.
+    Returns dX as N slices and every parameter gradient."""
+    x1 = [layernorm(x, p["ln1_g"], p["ln1_b"], eps) for x in X_slices]
+    X1 = all_gather_sequence(x1, batch, seq)
+    h1 = transformer_layer_sp_block_out(X_slices, p, batch, seq, n_heads, n_shards, eps, causal)
+    x2 = [layernorm(x, p["ln2_g"], p["ln2_b"], eps) for x in h1]
+    X2 = all_gather_sequence(x2, batch, seq)
+    dYg = all_gather_sequence(dY_slices, batch, seq)
+    gm = mlp_backward_sharded(X2, p["A"], p["b1"], p["B"], dYg, n_shards, residual=False)
+    g2 = sequence_shard(reduce_partials(gm["dX_partials"]), batch, seq, n_shards)
+    h = X_slices[0].shape[-1]
+    dh1, dg2, db2n = [], 0.0, 0.0
+    for hs_, gs_, dys in zip(h1, g2, dY_slices):   # slices [b][S/N][h]: rows of h
+        dx, dg, db = layernorm_backward(hs_.reshape(-1, h), p["ln2_g"], gs_.reshape(-1, h), eps)
+        dh1.append(dys + dx.reshape(dys.shape))
+        dg2, db2n = dg2 + dg, db2n + db
+    dh1g = all_gather_sequence(dh1, batch, seq)
+    ga = self_attention_backward_sharded(X1, p["Wqkv"], p["bqkv"], p["Wo"], p["bo"], dh1g,
+                                         batch, seq, n_heads, n_shards, causal, residual=False)
+    g1 = sequence_shard(reduce_partials(ga["dX_partials"]), batch, seq, n_shards)
+    dX, dg1, db1n = [], 0.0, 0.0
+    for xs_, gs_, dhs in zip(X_slices, g1, dh1):
+        dx, dg, db = layernorm_backward(xs_.reshape(-1, h), p["ln1_g"], gs_.reshape(-1, h), eps)
+        dX.append(dhs + dx.reshape(dhs.shape))
+        dg1, db1n = dg1 + dg, db1n + db
+    return dict(dX=dX, dWqkv=ga["dWqkv"], dbqkv=ga["dbqkv"], dWo=ga["dWo"], dbo=ga["dbo"],
+                dA=gm["dA"], db1=gm["db1"], dB=gm["dB"], db2=gm["db2"],
+                dln1_g=dg1, dln1_b=db1n, dln2_g=dg2, dln2_b=db2n)
+
+
+def transformer_layer_sp_block_out(X_slices: list, p: dict, batch: int, seq: int,
+                                   n_heads: int, n_shards: int, eps: float = 1e-5,
+                                   causal: bool = True) -> list:
+    """h1 = X + Attn(LN1(X)) of the sequence-parallel layer, as slices."""
+    h = X_slices[0].shape[-1]
+    d = h // n_heads
+    hs = h // n_shards
+    x1 = [layernorm(x, p["ln1_g"], p["ln1_b"], eps) for x in X_slices]
+    X1 = all_gather_sequence(x1, batch, seq)
+    QKV_i = column_parallel_linear(X1, p["Wqkv"], p["bqkv"], n_shards,
+                                   kind=SPLIT_QKV_HEADS, head_dim=d)
+    O_i = [attention_heads(q[:, :hs], q[:, hs:2 * hs], q[:, 2 * hs:],
+                           batch, seq, n_heads // n_shards, causal)
+           for q in QKV_i]
+    P_i = row_parallel_linear(O_i, p["Wo"], n_shards)
+    return reduce_scatter_partials(P_i, batch, seq, n_shards, p["bo"], X_slices)
+
+
 # --------------------------------------------------------------------------
 # the same definitions restricted to a subset of output token rows
 # (used to check full-size workloads on sampled rows)

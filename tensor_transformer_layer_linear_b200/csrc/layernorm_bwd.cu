@@ -13,7 +13,9 @@
 // block reductions per row. Each CTA keeps its column sums of g x_hat and g
 // in shared memory (every column owned by one thread) and writes them once;
 // a second pass adds the CTAs' sums in a fixed order, so dgamma and dbeta
-// are deterministic.
+// are deterministic. With a sequence-shard map (sequence parallelism) the
+// partials stay in token order while x, the residual gradient and dx use the
+// sequence-sharded layout: the reduce-scatter of the backward.
 #include "tp_device.cuh"
 #include "tp_internal.h"
 
@@ -47,7 +49,7 @@ __global__ void __launch_bounds__(kLnbThreads, (CH <= 2 ? 3 : 1)) rows_sum_ln_bw
     const float* __restrict__ P, int n_shards, int64_t stride, int64_t rows, int h,
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ gamma,
     const uint16_t* __restrict__ res, float eps, uint16_t* __restrict__ dx,
-    float* __restrict__ dg_part, float* __restrict__ db_part) {
+    float* __restrict__ dg_part, float* __restrict__ db_part, SeqShard sp) {
   __shared__ float red[kLnbThreads / 32];
   extern __shared__ float colsums[];  // [2][h]: sums of g x_hat, then of g
   const int nch = h >> 3;
@@ -56,7 +58,8 @@ __global__ void __launch_bounds__(kLnbThreads, (CH <= 2 ? 3 : 1)) rows_sum_ln_bw
   // (the barriers of the first row's block reductions order this before any
   // thread adds to its columns; every CTA has at least one row)
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    const int64_t off = r * h;
+    const int64_t off = r * h;                      // partials: token order
+    const int64_t soff = seq_shard_row(sp, r) * h;  // x, residual, dx
     float xv[CH][8], gv[CH][8], gm[CH][8];
     float s = 0.f;
 #pragma unroll
@@ -64,7 +67,7 @@ __global__ void __launch_bounds__(kLnbThreads, (CH <= 2 ? 3 : 1)) rows_sum_ln_bw
       const int ch = threadIdx.x + c * kLnbThreads;
       if (ch < nch) {
         const int64_t e = off + (ch << 3);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(x + e)), xv[c]);
+        unpack8(__ldg(reinterpret_cast<const uint4*>(x + soff + (ch << 3))), xv[c]);
         // the gradient reaching the LN output: sum of the partials in shard order
         if constexpr (NS > 0) {
           float4 v[NS][2];
@@ -131,7 +134,7 @@ __global__ void __launch_bounds__(kLnbThreads, (CH <= 2 ? 3 : 1)) rows_sum_ln_bw
     for (int c = 0; c < CH; ++c) {
       const int ch = threadIdx.x + c * kLnbThreads;
       if (ch < nch) {
-        const int64_t e = off + (ch << 3);
+        const int64_t e = soff + (ch << 3);
         float rv[8];
         if (res != nullptr) {
           unpack8(__ldg(reinterpret_cast<const uint4*>(res + e)), rv);
@@ -174,7 +177,8 @@ constexpr int lnb_ctas_per_sm() {
 template <int CH>
 static int launch_lnb_ch(const float* P, int n_shards, int64_t rows, int h, const void* x,
                          const void* gamma, const void* res, float eps, void* dx, float* dg_part,
-                         float* db_part, int max_ctas, int num_sms, cudaStream_t s) {
+                         float* db_part, int max_ctas, int num_sms, cudaStream_t s,
+                         SeqShard sp) {
   int ctas = lnb_ctas_per_sm<CH>() * num_sms;
   if (ctas > max_ctas) ctas = max_ctas;
   if (ctas > rows) ctas = static_cast<int>(rows);
@@ -192,11 +196,11 @@ static int launch_lnb_ch(const float* P, int n_shards, int64_t rows, int h, cons
     cudaFuncSetAttribute(rows_sum_ln_bwd_kernel<CH, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   }
   switch (n_shards) {
-    case 1: rows_sum_ln_bwd_kernel<CH, 1><<<ctas, kLnbThreads, smem, s>>>(P, 1, stride, rows, h, X, G, R, eps, D, dg_part, db_part); break;
-    case 2: rows_sum_ln_bwd_kernel<CH, 2><<<ctas, kLnbThreads, smem, s>>>(P, 2, stride, rows, h, X, G, R, eps, D, dg_part, db_part); break;
-    case 4: rows_sum_ln_bwd_kernel<CH, 4><<<ctas, kLnbThreads, smem, s>>>(P, 4, stride, rows, h, X, G, R, eps, D, dg_part, db_part); break;
-    case 8: rows_sum_ln_bwd_kernel<CH, 8><<<ctas, kLnbThreads, smem, s>>>(P, 8, stride, rows, h, X, G, R, eps, D, dg_part, db_part); break;
-    default: rows_sum_ln_bwd_kernel<CH, 0><<<ctas, kLnbThreads, smem, s>>>(P, n_shards, stride, rows, h, X, G, R, eps, D, dg_part, db_part); break;
+    case 1: rows_sum_ln_bwd_kernel<CH, 1><<<ctas, kLnbThreads, smem, s>>>(P, 1, stride, rows, h, X, G, R, eps, D, dg_part, db_part, sp); break;
+    case 2: rows_sum_ln_bwd_kernel<CH, 2><<<ctas, kLnbThreads, smem, s>>>(P, 2, stride, rows, h, X, G, R, eps, D, dg_part, db_part, sp); break;
+    case 4: rows_sum_ln_bwd_kernel<CH, 4><<<ctas, kLnbThreads, smem, s>>>(P, 4, stride, rows, h, X, G, R, eps, D, dg_part, db_part, sp); break;
+    case 8: rows_sum_ln_bwd_kernel<CH, 8><<<ctas, kLnbThreads, smem, s>>>(P, 8, stride, rows, h, X, G, R, eps, D, dg_part, db_part, sp); break;
+    default: rows_sum_ln_bwd_kernel<CH, 0><<<ctas, kLnbThreads, smem, s>>>(P, n_shards, stride, rows, h, X, G, R, eps, D, dg_part, db_part, sp); break;
   }
   return ctas;
 }
@@ -204,21 +208,22 @@ static int launch_lnb_ch(const float* P, int n_shards, int64_t rows, int h, cons
 int launch_rows_sum_ln_bwd(const float* P, int n_shards, int64_t rows, int64_t h, const void* x,
                            const void* gamma, const void* residual, float eps, void* dx,
                            float* dgamma, float* dbeta, float* part, int max_ctas,
-                           cudaStream_t s, int num_sms) {
+                           cudaStream_t s, int num_sms, int sp_n, int sp_batch, int sp_seq) {
   if (rows <= 0) return 0;
+  const SeqShard sp{sp_n, sp_batch, sp_seq};
   float* dg_part = part;
   float* db_part = part + static_cast<int64_t>(max_ctas) * h;
   const int hh = static_cast<int>(h);
   const int64_t nch = h / 8;
   int ctas;
   if (nch <= kLnbThreads)
-    ctas = launch_lnb_ch<1>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s);
+    ctas = launch_lnb_ch<1>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s, sp);
   else if (nch <= 2 * kLnbThreads)
-    ctas = launch_lnb_ch<2>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s);
+    ctas = launch_lnb_ch<2>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s, sp);
   else if (nch <= 4 * kLnbThreads)
-    ctas = launch_lnb_ch<4>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s);
+    ctas = launch_lnb_ch<4>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s, sp);
   else
-    ctas = launch_lnb_ch<8>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s);
+    ctas = launch_lnb_ch<8>(P, n_shards, rows, hh, x, gamma, residual, eps, dx, dg_part, db_part, max_ctas, num_sms, s, sp);
   if (launch_slab_sum(dg_part, ctas, hh, dgamma, s) != 0) return 2;
   if (launch_slab_sum(db_part, ctas, hh, dbeta, s) != 0) return 2;
   return cudaGetLastError() == cudaSuccess ? 0 : 2;

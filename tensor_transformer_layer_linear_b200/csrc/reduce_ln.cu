@@ -65,24 +65,6 @@ __device__ __forceinline__ void sum_partials8(const float* __restrict__ P, int n
   }
 }
 
-// Row m = b S + s of the token-ordered [batch][S] rows, stored in the
-// sequence-sharded layout [N][batch][S/N]: shard s / (S/N) keeps positions
-// [i S/N, (i+1) S/N) of every sequence ("Sequence Parallelism"). sp.n == 0
-// means the identity.
-struct SeqShard {
-  int n;      // shards (0: no permutation)
-  int batch;
-  int seq;
-};
-__device__ __forceinline__ int64_t seq_shard_row(const SeqShard& sp, int64_t m) {
-  if (sp.n == 0) return m;
-  const int ss = sp.seq / sp.n;
-  const int64_t b = m / sp.seq;
-  const int s = static_cast<int>(m - b * sp.seq);
-  const int i = s / ss;
-  return (static_cast<int64_t>(i) * sp.batch + b) * ss + (s - i * ss);
-}
-
 // Y = sum_i P_i + bias + residual. With sp.n > 0 the residual is read from,
 // and Y written to, the sequence-sharded layout (the reduce-scatter).
 template <int NS>

@@ -451,14 +451,16 @@ size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int 
   if (kind == TP_WS_ATTN_CORE_BWD) return attn_core_bwd_bytes(M, H);
   if (kind == TP_WS_ATTN_BWD) return attn_bwd_bytes(M, H, N);
   if (kind == TP_WS_LN_BWD) return ln_bwd_bytes(H);
-  if (kind == TP_WS_LAYER_BWD) {
+  if (kind == TP_WS_LAYER_BWD || kind == TP_WS_LAYER_BWD_SP) {
     if (ffn <= 0) return 0;
     // x1, h1, x2, dh1 + the attention part (its own partials and slabs
     // reused by the MLP) + G, H, dZ of the MLP + LN-backward column sums
     const size_t F = static_cast<size_t>(ffn);
     const size_t slabs = round256(static_cast<size_t>(kColsumSlabs) * (F + 4 * H) * 4);
+    // (+ the gathered dY and dh1 under sequence parallelism)
+    const size_t gathered = (kind == TP_WS_LAYER_BWD_SP) ? 2 * round256(M * H * 2) : 0;
     return 4 * round256(M * H * 2) + attn_bwd_bytes(M, H, N) + 3 * round256(M * F * 2) + slabs +
-           ln_bwd_bytes(H);
+           ln_bwd_bytes(H) + gathered;
   }
   if (kind == TP_WS_LAYER || kind == TP_WS_LAYER_SP) {
     if (ffn <= 0) return 0;
@@ -1075,10 +1077,14 @@ tp_status tp_reduce_partials_layernorm_backward(const float* partials, int n_sha
              : TP_ERR_CUDA;
 }
 
-tp_status tp_layer_backward(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
-                            int64_t n_heads, int64_t ffn, int n_shards, const tp_layer_weights* w,
-                            float ln_eps, const uint16_t* dY, void* ws, size_t ws_bytes,
-                            uint16_t* dX, const tp_layer_grads* g, void* stream) {
+// The layer backward for token-ordered (sp == false) or sequence-sharded
+// (sp == true) X, dY and dX; the GEMM and attention work always runs on
+// token-ordered activations (all-gathered under sequence parallelism).
+static tp_status layer_backward_impl(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
+                                     int64_t n_heads, int64_t ffn, int n_shards,
+                                     const tp_layer_weights* w, float ln_eps, const uint16_t* dY,
+                                     void* ws, size_t ws_bytes, uint16_t* dX,
+                                     const tp_layer_grads* g, void* stream, bool sp) {
   if (X == nullptr || w == nullptr || dY == nullptr || dX == nullptr || g == nullptr ||
       ws == nullptr)
     return TP_ERR_NULL;
@@ -1092,11 +1098,13 @@ tp_status tp_layer_backward(const uint16_t* X, int64_t batch, int64_t seq, int64
       g->b1_shards == nullptr || g->B_shards == nullptr || g->b2 == nullptr)
     return TP_ERR_NULL;
   if (!attn_bwd_shape_ok(batch, seq, h, n_heads, n_shards) || ffn <= 0 || ffn % n_shards ||
-      (ffn / n_shards) % 8 || h % 8 || h > 16384 || ffn > kIntMax)
+      (ffn / n_shards) % 8 || h % 8 || h > 16384 || ffn > kIntMax || (sp && seq % n_shards))
     return TP_ERR_SHAPE;
   if (h / n_heads != 128) return TP_ERR_UNSUPPORTED;
   const int64_t M = batch * seq;
-  if (ws_bytes < tp_workspace_bytes(TP_WS_LAYER_BWD, M, h, ffn, n_shards)) return TP_ERR_WORKSPACE;
+  if (ws_bytes < tp_workspace_bytes(sp ? TP_WS_LAYER_BWD_SP : TP_WS_LAYER_BWD, M, h, ffn,
+                                    n_shards))
+    return TP_ERR_WORKSPACE;
   if (!al16(ws) || !al16(X) || !al16(dY) || !al16(dX)) return TP_ERR_ALIGN;
   const float* grads[] = {g->ln1_gamma, g->ln1_beta, g->Wqkv_shards, g->bqkv_shards,
                           g->Wo_shards, g->bo, g->ln2_gamma, g->ln2_beta, g->A_shards,
@@ -1111,10 +1119,10 @@ tp_status tp_layer_backward(const uint16_t* X, int64_t batch, int64_t seq, int64
   const size_t F = static_cast<size_t>(ffn);
   const size_t act_b = round256(Mz * H * 2);
   uint8_t* p = static_cast<uint8_t*>(ws);
-  uint16_t* x1 = reinterpret_cast<uint16_t*>(p); p += act_b;
-  uint16_t* h1 = reinterpret_cast<uint16_t*>(p); p += act_b;
-  uint16_t* x2 = reinterpret_cast<uint16_t*>(p); p += act_b;
-  uint16_t* dh1 = reinterpret_cast<uint16_t*>(p); p += act_b;
+  uint16_t* x1 = reinterpret_cast<uint16_t*>(p); p += act_b;   // token order
+  uint16_t* h1 = reinterpret_cast<uint16_t*>(p); p += act_b;   // layout of X
+  uint16_t* x2 = reinterpret_cast<uint16_t*>(p); p += act_b;   // token order
+  uint16_t* dh1 = reinterpret_cast<uint16_t*>(p); p += act_b;  // layout of X
   AttnBwdBufs ab = attn_bwd_layout(p, Mz, H, n_shards);
   p += attn_bwd_bytes(Mz, H, n_shards);
   MlpBwdBufs mb;
@@ -1124,14 +1132,30 @@ tp_status tp_layer_backward(const uint16_t* X, int64_t batch, int64_t seq, int64
   float* slabs = reinterpret_cast<float*>(p);
   p += round256(static_cast<size_t>(kColsumSlabs) * (F + 4 * H) * 4);
   float* lnb = reinterpret_cast<float*>(p);
+  p += ln_bwd_bytes(H);
+  // token-ordered dY and dh1 (all-gathered under sequence parallelism)
+  const uint16_t* dYg = dY;
+  const uint16_t* dh1g = dh1;
+  uint16_t* gather_dY = nullptr;
+  uint16_t* gather_dh1 = nullptr;
+  if (sp) {
+    gather_dY = reinterpret_cast<uint16_t*>(p); p += act_b;
+    gather_dh1 = reinterpret_cast<uint16_t*>(p); p += act_b;
+    dYg = gather_dY;
+    dh1g = gather_dh1;
+  }
   mb.part = ab.part;  // the two blocks' partials are used one after the other
   mb.slabs = slabs;
   ab.slabs = slabs;
-  const size_t lnb_bytes = ln_bwd_bytes(H);
+  const int spn = sp ? n_shards : 0, sb = static_cast<int>(batch), sq = static_cast<int>(seq);
 
   // forward recompute: x1 = LN1(X), QKV, O, lse, h1 = X + Attn(x1), x2 = LN2(h1)
-  st = tp_layernorm(X, M, h, w->ln1_gamma, w->ln1_beta, ln_eps, x1, stream);
-  if (st != TP_OK) return st;
+  {
+    TraceScope ts(tpk::KID_LAYERNORM, s);
+    if (tpk::launch_rows_sum_ln(nullptr, 0, M, h, nullptr, X, w->ln1_gamma, w->ln1_beta, ln_eps,
+                                nullptr, x1, s, spn, sb, sq, 1) != 0)
+      return TP_ERR_CUDA;
+  }
   st = tp_column_linear(x1, M, h, w->Wqkv_shards, w->bqkv_shards, 3 * h, n_shards, TP_ACT_NONE,
                         ab.qkv, stream);
   if (st != TP_OK) return st;
@@ -1139,30 +1163,66 @@ tp_status tp_layer_backward(const uint16_t* X, int64_t batch, int64_t seq, int64
   if (st != TP_OK) return st;
   st = tp_row_linear(ab.o, M, h, w->Wo_shards, h, n_shards, ab.part, stream);
   if (st != TP_OK) return st;
-  st = tp_reduce_partials_layernorm(ab.part, n_shards, M, h, w->bo, X, w->ln2_gamma, w->ln2_beta,
-                                    ln_eps, h1, x2, stream);
-  if (st != TP_OK) return st;
+  {
+    TraceScope ts(tpk::KID_REDUCE_LN, s);
+    if (tpk::launch_rows_sum_ln(ab.part, n_shards, M, h, w->bo, X, w->ln2_gamma, w->ln2_beta,
+                                ln_eps, h1, x2, s, spn, sb, sq, 1) != 0)
+      return TP_ERR_CUDA;
+  }
+  if (sp) {  // the backward of the forward's last reduce-scatter: gather dY
+    TraceScope ts(tpk::KID_ALL_GATHER, s);
+    if (tpk::launch_all_gather_sequence(dY, n_shards, sb, sq, h, gather_dY, s, d.num_sms) != 0)
+      return TP_ERR_CUDA;
+  }
   // MLP block: gradients and the partials of dx2; its one reduction is fused
   // with LN2's backward and the residual: dh1 = dY + LN2'(h1)^T sum_i dx2_i
+  // (a reduce-scatter into the slices under sequence parallelism)
   st = mlp_backward_core(d, s, x2, static_cast<int>(M), static_cast<int>(h),
                          static_cast<int>(ffn), n_shards, w->A_shards, w->b1_shards, w->B_shards,
-                         dY, mb, g->A_shards, g->b1_shards, g->B_shards, g->b2);
+                         dYg, mb, g->A_shards, g->b1_shards, g->B_shards, g->b2);
   if (st != TP_OK) return st;
-  st = tp_reduce_partials_layernorm_backward(mb.part, n_shards, M, h, h1, w->ln2_gamma, dY,
-                                             ln_eps, lnb, lnb_bytes, dh1, g->ln2_gamma,
-                                             g->ln2_beta, stream);
-  if (st != TP_OK) return st;
+  {
+    TraceScope ts(tpk::KID_LAYERNORM_BWD, s);
+    if (tpk::launch_rows_sum_ln_bwd(mb.part, n_shards, M, h, h1, w->ln2_gamma, dY, ln_eps, dh1,
+                                    g->ln2_gamma, g->ln2_beta, lnb, kLnBwdMaxCtas, s, d.num_sms,
+                                    spn, sb, sq) != 0)
+      return TP_ERR_CUDA;
+  }
+  if (sp) {  // the attention block's input gradient is needed in token order
+    TraceScope ts(tpk::KID_ALL_GATHER, s);
+    if (tpk::launch_all_gather_sequence(dh1, n_shards, sb, sq, h, gather_dh1, s, d.num_sms) != 0)
+      return TP_ERR_CUDA;
+  }
   // attention block: gradients and the partials of dx1; its one reduction is
   // fused with LN1's backward and the residual: dX = dh1 + LN1'(X)^T sum_i dx1_i
   st = attn_backward_core(d, stream, x1, batch, seq, h, n_heads, n_heads, 1, n_shards,
-                          w->Wqkv_shards, w->Wo_shards, dh1, ab, g->Wqkv_shards, g->bqkv_shards,
+                          w->Wqkv_shards, w->Wo_shards, dh1g, ab, g->Wqkv_shards, g->bqkv_shards,
                           g->Wo_shards, g->bo);
   if (st != TP_OK) return st;
-  return tp_reduce_partials_layernorm_backward(ab.part, n_shards, M, h, X, w->ln1_gamma, dh1,
-                                               ln_eps, lnb, lnb_bytes, dX, g->ln1_gamma,
-                                               g->ln1_beta, stream);
+  TraceScope ts(tpk::KID_LAYERNORM_BWD, s);
+  return tpk::launch_rows_sum_ln_bwd(ab.part, n_shards, M, h, X, w->ln1_gamma, dh1, ln_eps, dX,
+                                     g->ln1_gamma, g->ln1_beta, lnb, kLnBwdMaxCtas, s, d.num_sms,
+                                     spn, sb, sq) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
 }
 
+tp_status tp_layer_backward(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
+                            int64_t n_heads, int64_t ffn, int n_shards, const tp_layer_weights* w,
+                            float ln_eps, const uint16_t* dY, void* ws, size_t ws_bytes,
+                            uint16_t* dX, const tp_layer_grads* g, void* stream) {
+  return layer_backward_impl(X, batch, seq, h, n_heads, ffn, n_shards, w, ln_eps, dY, ws,
+                             ws_bytes, dX, g, stream, false);
+}
+
+tp_status tp_layer_backward_sp(const uint16_t* X_shards, int64_t batch, int64_t seq, int64_t h,
+                               int64_t n_heads, int64_t ffn, int n_shards,
+                               const tp_layer_weights* w, float ln_eps, const uint16_t* dY_shards,
+                               void* ws, size_t ws_bytes, uint16_t* dX_shards,
+                               const tp_layer_grads* g, void* stream) {
+  return layer_backward_impl(X_shards, batch, seq, h, n_heads, ffn, n_shards, w, ln_eps,
+                             dY_shards, ws, ws_bytes, dX_shards, g, stream, true);
+}
 
 tp_status tp_attention_gqa_lse(const uint16_t* QKV_shards, int64_t batch, int64_t seq,
                                int64_t n_q, int64_t n_kv, int64_t head_dim, int causal,

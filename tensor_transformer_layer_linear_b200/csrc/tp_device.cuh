@@ -406,6 +406,24 @@ __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Row m = b S + s of the token-ordered [batch][S] rows, stored in the
+// sequence-sharded layout [N][batch][S/N]: shard s / (S/N) keeps positions
+// [i S/N, (i+1) S/N) of every sequence ("Sequence Parallelism"). sp.n == 0
+// means the identity.
+struct SeqShard {
+  int n;      // shards (0: no permutation)
+  int batch;
+  int seq;
+};
+__device__ __forceinline__ int64_t seq_shard_row(const SeqShard& sp, int64_t m) {
+  if (sp.n == 0) return m;
+  const int ss = sp.seq / sp.n;
+  const int64_t b = m / sp.seq;
+  const int s = static_cast<int>(m - b * sp.seq);
+  const int i = s / ss;
+  return (static_cast<int64_t>(i) * sp.batch + b) * ss + (s - i * ss);
+}
+
 // ---------------------------------------------------------------- misc
 // 2^x with the special-function unit's approximation (flush-to-zero): the
 // PTX ex2.approx.ftz instruction.

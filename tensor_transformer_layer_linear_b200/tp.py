@@ -32,7 +32,7 @@ TP_ERR_WORKSPACE, TP_ERR_UNSUPPORTED, TP_ERR_CUDA, TP_ERR_TIMEOUT = 4, 5, 6, 7
 TP_SPLIT_COLUMN, TP_SPLIT_ROW, TP_SPLIT_QKV_HEADS, TP_SPLIT_GATE_UP = 0, 1, 2, 3
 TP_ACT_NONE, TP_ACT_GELU_ERF, TP_ACT_SWIGLU = 0, 1, 2
 TP_WS_MLP, TP_WS_ATTN, TP_WS_LAYER, TP_WS_LAYER_SP, TP_WS_MLP_BWD = 0, 1, 2, 3, 4
-TP_WS_ATTN_CORE_BWD, TP_WS_ATTN_BWD, TP_WS_LAYER_BWD, TP_WS_LN_BWD = 5, 6, 7, 8
+TP_WS_ATTN_CORE_BWD, TP_WS_ATTN_BWD, TP_WS_LAYER_BWD, TP_WS_LN_BWD, TP_WS_LAYER_BWD_SP = 5, 6, 7, 8, 9
 
 _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
@@ -95,6 +95,9 @@ _SIGS = {
                                          _i32, _vp, _sz, _vp, _vp]),
     "tp_attn_backward_gqa": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp,
                                     _vp, _i32, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "tp_layer_backward_sp": (_i32, [_vp, _i64, _i64, _i64, _i64, _i64, _i32,
+                                    ctypes.POINTER(tp_layer_weights), _f32, _vp, _vp, _sz, _vp,
+                                    ctypes.POINTER(tp_layer_grads), _vp]),
     "tp_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "tp_get_last_error": (_i32, [_vp]),
     "tp_status_string": (ctypes.c_char_p, [_i32]),
@@ -372,6 +375,15 @@ def tp_attn_backward_gqa(X, batch, seq, h, n_q, n_kv, causal, n_shards, Wqkv_sha
                                     int(bool(residual)), _p(ws), ws_bytes, _p(dX),
                                     _p(dWqkv_shards), _p(dbqkv_shards), _p(dWo_shards), _p(dbo),
                                     _s(stream)), "tp_attn_backward_gqa")
+
+
+def tp_layer_backward_sp(X_shards, batch, seq, h, n_heads, ffn, n_shards,
+                         weights: tp_layer_weights, ln_eps, dY_shards, ws, ws_bytes, dX_shards,
+                         grads: tp_layer_grads, stream=None):
+    _check(lib.tp_layer_backward_sp(_p(X_shards), batch, seq, h, n_heads, ffn, n_shards,
+                                    ctypes.byref(weights), ln_eps, _p(dY_shards), _p(ws), ws_bytes,
+                                    _p(dX_shards), ctypes.byref(grads), _s(stream)),
+           "tp_layer_backward_sp")
 
 
 def tp_get_last_error(stream=None) -> int:

@@ -819,3 +819,33 @@ def test_gqa_attention_backward_sharded_equals_unsharded(n, nkv):
     if nkv == nq:
         mha = O.self_attention_backward(X, Wqkv, bqkv, Wo, bo, dY, b, s, nq)
         np.testing.assert_allclose(ref["dX"], mha["dX"], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("n", [1, 2, 4])
+def test_transformer_layer_sp_backward_is_the_sharded_layer_backward(n):
+    """Sequence parallelism only moves rows: the SP backward's dX slices are
+    the slices of the standard layer backward's dX and every parameter
+    gradient is the same (up to summation order)."""
+    rng = np.random.default_rng(39 + n)
+    b, s, h, nh, F = 2, 8, 8, 4, 16
+    X = rng.standard_normal((b * s, h))
+    p = dict(Wqkv=rng.standard_normal((h, 3 * h)) * .4, bqkv=rng.standard_normal(3 * h) * .1,
+             Wo=rng.standard_normal((h, h)) * .4, bo=rng.standard_normal(h) * .1,
+             A=rng.standard_normal((h, F)) * .4, b1=rng.standard_normal(F) * .1,
+             B=rng.standard_normal((F, h)) * .4, b2=rng.standard_normal(h) * .1,
+             ln1_g=1 + rng.standard_normal(h) * .1, ln1_b=rng.standard_normal(h) * .1,
+             ln2_g=1 + rng.standard_normal(h) * .1, ln2_b=rng.standard_normal(h) * .1)
+    dY = rng.standard_normal((b * s, h))
+    ref = O.transformer_layer_backward(X, p, dY, b, s, nh, n)
+    got = O.transformer_layer_sp_backward(O.sequence_shard(X, b, s, n), p,
+                                          O.sequence_shard(dY, b, s, n), b, s, nh, n)
+    np.testing.assert_allclose(O.all_gather_sequence(got["dX"], b, s), ref["dX"], rtol=1e-12,
+                               atol=1e-12)
+    for k in ("dWqkv", "dbqkv", "dWo", "dbo", "dA", "db1", "dB", "db2", "dln1_g", "dln1_b",
+              "dln2_g", "dln2_b"):
+        np.testing.assert_allclose(got[k], ref[k], rtol=1e-12, atol=1e-12, err_msg=k)
+    # and the SP forward's h1 is the standard layer's h1, sliced
+    h1 = O.transformer_layer_sp_block_out(O.sequence_shard(X, b, s, n), p, b, s, nh, n)
+    x1 = O.layernorm(X, p["ln1_g"], p["ln1_b"])
+    ref_h1 = O.self_attention(x1, p["Wqkv"], p["bqkv"], p["Wo"], p["bo"], X, b, s, nh)
+    np.testing.assert_allclose(O.all_gather_sequence(h1, b, s), ref_h1, rtol=1e-12, atol=1e-12)
