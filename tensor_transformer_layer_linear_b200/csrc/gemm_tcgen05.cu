@@ -42,24 +42,17 @@ constexpr int BK = 64;             // 64 bf16 = 128 bytes = one swizzle row
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, each half the columns
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 
-// Epilogue kinds: bf16 + bias + activation (column-parallel), fp32 partials
-// (row-parallel), gated SiLU(gate) * up over interleaved 128-column blocks,
-// the GeLU backward bf16(acc * GeLU'(Z)) with GeLU'(Z) read from aux, and the
-// backward's recompute of the column layer: bf16 GeLU(Z) out, GeLU'(Z) to
-// aux_out (Z = acc + bias).
-enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU = 2, EPI_MUL_AUX = 3, EPI_GELU_AUX = 4 };
-
-template <int BN, int CTAS, int EPI>
+template <int BN, int CTAS>
 struct GemmCfg {
   static constexpr int kTileM = BM * CTAS;       // rows of a tile
   static constexpr int kBRows = BN / CTAS;       // B^T rows held per CTA
   static constexpr int kABytes = BM * BK * 2;
   static constexpr int kBBytes = kBRows * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr bool kWideStore = (CTAS == 2) && (EPI == EPI_F32);
-  static constexpr int kStages = (CTAS == 2) ? (kWideStore ? 5 : 6) : ((BN == 256) ? 4 : 6);
+  static constexpr int kStages = (CTAS == 2) ? 6 : ((BN == 256) ? 4 : 6);
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kStagingBufs = kWideStore ? 2 : 1;
+  // epilogue staging: per epilogue warp, kStagingBufs buffers of 32 rows x 128 bytes
+  static constexpr int kStagingBufs = 1;
   static constexpr int kStagingBytes = kEpiWarps * kStagingBufs * 4096;
   static constexpr int kNumBars = 2 * kStages + 5;
   static constexpr int kSmemBytes =
@@ -79,6 +72,12 @@ struct GemmParams {
   unsigned* err;
 };
 
+// Epilogue kinds: bf16 + bias + activation (column-parallel), fp32 partials
+// (row-parallel), gated SiLU(gate) * up over interleaved 128-column blocks,
+// the GeLU backward bf16(acc * GeLU'(Z)) with GeLU'(Z) read from aux, and the
+// backward's recompute of the column layer: bf16 GeLU(Z) out, GeLU'(Z) to
+// aux_out (Z = acc + bias).
+enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU = 2, EPI_MUL_AUX = 3, EPI_GELU_AUX = 4 };
 
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + __expf(-x)); }
 
@@ -92,7 +91,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmD,
                         const __grid_constant__ CUtensorMap tmE, const GemmParams p) {
-  using C = GemmCfg<BN, CTAS, EPI>;
+  using C = GemmCfg<BN, CTAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* tiles = smem_raw + pad;
@@ -515,7 +514,7 @@ static bool encode_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1
 
 template <int BN, int EPI, int CTAS, bool A_MN = false, bool B_MN = false>
 static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, int num_sms) {
-  using C = GemmCfg<BN, CTAS, EPI>;
+  using C = GemmCfg<BN, CTAS>;
   constexpr bool OUT_F32 = EPI == EPI_F32;
   CUtensorMap tmA, tmB, tmD, tmE;
   const uint64_t ga = pr.a_batched ? pr.G : 1, gb = pr.b_batched ? pr.G : 1;

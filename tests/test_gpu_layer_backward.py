@@ -171,3 +171,96 @@ def test_layer_backward_workload(tp):
                                        cfg["ln_eps"])
     assert_parity(got["dX"][:s], ref["dX"], "dX of sequence 0", fro_rel=BWD_FRO_REL)
     np.testing.assert_allclose(got["b2"], f64(dY).sum(axis=0), rtol=1e-5, atol=1e-3)
+
+
+# ---------------------------------------------------------------- sequence parallelism
+
+def _slices(bits, batch, seq, n):
+    h = bits.shape[-1]
+    return np.ascontiguousarray(np.stack(O.sequence_shard(bits.reshape(batch * seq, h), batch, seq, n)))
+
+
+# gradients that do not depend on dQ (whose fp32 accumulation order varies
+# between runs) are bit-identical between the two layouts
+EXACT = ("ln2_gamma", "ln2_beta", "A_shards", "b1_shards", "B_shards", "b2", "Wo_shards", "bo")
+
+
+def _same_as_standard(sp, std, b, s):
+    """The same kernels on permuted rows: the MLP side and W_O bit-identical,
+    the rest equal up to dQ's accumulation order."""
+    for k in EXACT:
+        assert np.array_equal(sp[k], std[k]), k
+    got = synth.bf16_bits_to_f64(O.all_gather_sequence(list(sp["dX_bits"]), b, s))
+    assert_parity(got, std["dX"], "dX vs standard", max_rel=2e-3, fro_rel=1e-4)
+    for k in ("Wqkv_shards", "bqkv_shards", "ln1_gamma", "ln1_beta"):
+        assert_parity(sp[k], std[k], k + " vs standard", max_rel=2e-3, fro_rel=1e-4)
+
+
+def run_layer_backward_sp(tp, inp, dY_bits, cfg, n):
+    """tp_layer_backward_sp on the slices of X and dY; returns dX slices and
+    the gradients (same packing as run_layer_backward)."""
+    b, s, h, nh, F = cfg["batch"], cfg["seq"], cfg["h"], cfg["n_heads"], cfg["ffn"]
+    M = b * s
+    dev = {k: to_dev(v) for k, v in inp.items()}
+    keep = dict(
+        ln1_gamma=dev["ln1_g"], ln1_beta=dev["ln1_b"],
+        Wqkv_shards=_shard(tp, dev["Wqkv"], h, 3 * h, 2, n, 128),
+        bqkv_shards=_shard(tp, dev["bqkv"], 1, 3 * h, 2, n, 128),
+        Wo_shards=_shard(tp, dev["Wo"], h, h, 1, n), bo=dev["bo"],
+        ln2_gamma=dev["ln2_g"], ln2_beta=dev["ln2_b"],
+        A_shards=_shard(tp, dev["A"], h, F, 0, n), b1_shards=dev["b1"],
+        B_shards=_shard(tp, dev["B"], F, h, 1, n), b2=dev["b2"])
+    w = tp.make_layer_weights(**keep)
+    sizes = dict(ln1_gamma=h, ln1_beta=h, Wqkv_shards=3 * h * h, bqkv_shards=3 * h,
+                 Wo_shards=h * h, bo=h, ln2_gamma=h, ln2_beta=h, A_shards=h * F, b1_shards=F,
+                 B_shards=F * h, b2=h)
+    gt = {k: torch.empty(v, dtype=torch.float32, device="cuda") for k, v in sizes.items()}
+    g = tp.make_layer_grads(**gt)
+    ws, nb = _ws(tp, tp.TP_WS_LAYER_BWD_SP, M, h, F, n)
+    dXs = torch.empty((n, b, s // n, h), dtype=torch.int16, device="cuda")
+    tp.tp_layer_backward_sp(to_dev(_slices(inp["X"], b, s, n)), b, s, h, nh, F, n, w,
+                            cfg.get("ln_eps", 1e-5), to_dev(_slices(dY_bits, b, s, n)), ws, nb,
+                            dXs, g)
+    assert tp.tp_get_last_error() == tp.TP_OK
+    out = {k: v.cpu().numpy().astype(np.float64) for k, v in gt.items()}
+    out["dX_bits"] = dXs.cpu().numpy().view(np.uint16)
+    return out
+
+
+@pytest.mark.parametrize("n", [1, 2, 4])
+def test_layer_backward_sp_small(tp, n):
+    cfg = dict(kind="layer", batch=2, seq=160, h=512, n_heads=4, ffn=2048, x_std=1.0,
+               w_std=0.05, b_std=0.05, ln_eps=1e-5)
+    inp = synth.make_inputs(cfg, seed=12)
+    rng = np.random.default_rng(1700)
+    for k in ("ln1_g", "ln2_g"):
+        inp[k] = _bits(rng, (cfg["h"],), 0.2, 1.0)
+    for k in ("ln1_b", "ln2_b"):
+        inp[k] = _bits(rng, (cfg["h"],), 0.1)
+    b, s = cfg["batch"], cfg["seq"]
+    dY = _bits(rng, (b * s, cfg["h"]))
+    sp = run_layer_backward_sp(tp, inp, dY, cfg, n)
+    std = run_layer_backward(tp, inp, dY, cfg, n)
+    _same_as_standard(sp, std, b, s)
+    # and against the oracle's sequence-parallel backward
+    p = {k: f64(v) for k, v in inp.items() if k != "X"}
+    ref = O.transformer_layer_sp_backward(O.sequence_shard(f64(inp["X"]), b, s, n), p,
+                                          O.sequence_shard(f64(dY), b, s, n), b, s,
+                                          cfg["n_heads"], n, cfg["ln_eps"])
+    for i in range(n):
+        assert_parity(synth.bf16_bits_to_f64(sp["dX_bits"][i]), ref["dX"][i], f"dX slice {i}",
+                      fro_rel=BWD_FRO_REL)
+    for k, v in _packed_ref(ref, n, cfg["h"], cfg["ffn"]).items():
+        assert_parity(sp[k], v, k, fro_rel=BWD_FRO_REL)
+
+
+def test_layer_backward_sp_workload(tp):
+    """The layer workload under sequence parallelism: bit-identical to the
+    standard layer backward up to the row permutation."""
+    cfg = synth.config("layer_2x2048_h4096_32x128_f16384_n8")
+    inp = synth.make_inputs(cfg)
+    b, s, n = cfg["batch"], cfg["seq"], cfg["n_shards"]
+    dY = _bits(np.random.default_rng(1800), (b * s, cfg["h"]))
+    sp = run_layer_backward_sp(tp, inp, dY, cfg, n)
+    std = run_layer_backward(tp, inp, dY, cfg, n)
+    _same_as_standard(sp, std, b, s)
