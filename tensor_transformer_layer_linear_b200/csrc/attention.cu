@@ -189,45 +189,51 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       // ---------------------------------------------------------- MMA
       constexpr uint32_t idesc_s = umma_idesc_bf16_f32(FA_BM, FA_BN);
       constexpr uint32_t idesc_o = umma_idesc_bf16_f32_bmn(FA_BM, FA_D);
-      auto qk = [&](int T, uint32_t kb) {
-        const uint32_t qb = s0 + OFF_Q + T * FA_TILE;
+      // descriptors built once; each MMA moves them by a constant offset
+      // (the issuing thread shares its sub-partition with softmax warps, so
+      // fewer instructions per MMA keep the tensor pipe fed)
+      const uint64_t dq0 = umma_desc_sw128(s0 + OFF_Q), dq1 = umma_desc_sw128(s0 + OFF_Q + FA_TILE);
+      const uint64_t dk0 = umma_desc_sw128(s0 + OFF_K), dk1 = umma_desc_sw128(s0 + OFF_K + FA_TILE);
+      const uint64_t dv0 = umma_desc_sw128_mn(s0 + OFF_V, FA_SUB);
+      const uint64_t dv1 = umma_desc_sw128_mn(s0 + OFF_V + FA_TILE, FA_SUB);
+      auto qk = [&](int T, int b) {
+        const uint64_t dq = T ? dq1 : dq0, dk = b ? dk1 : dk0;
 #pragma unroll
         for (int kk = 0; kk < FA_D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * FA_SUB + (kk & 3) * 32;
-          umma_bf16(tmem + T * FA_BN, umma_desc_sw128(qb + off), umma_desc_sw128(kb + off),
-                    idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16(tmem + T * FA_BN, desc_advance(dq, off), desc_advance(dk, off), idesc_s,
+                    kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(B_SFULL + T));
       };
-      auto pv = [&](int T, uint32_t vb, bool first) {
+      auto pv = [&](int T, int b, bool first) {
+        const uint64_t dv = b ? dv1 : dv0;
 #pragma unroll
         for (int kk = 0; kk < FA_BN / 16; ++kk) {
           umma_bf16_tmem_a(tmem + 2 * FA_BN + T * FA_D, tmem + T * FA_BN + kk * 8,
-                           umma_desc_sw128_mn(vb + kk * 2048, FA_SUB), idesc_o,
-                           (!first || kk > 0) ? 1u : 0u);
+                           desc_advance(dv, kk * 2048), idesc_o, (!first || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
       for (int j = 0; ok && j < nb; ++j) {
         const int b = j & 1;
         const uint32_t ph = (j >> 1) & 1;
-        const uint32_t kb = s0 + OFF_K + b * FA_TILE;
         if (!mbar_wait(bar(B_KFULL + b), ph, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        qk(0, kb);                                              // S_j^0
+        qk(0, b);                                               // S_j^0
         if (j >= 1) {                                           // O_1 += P_{j-1}^1 V_{j-1}
           if (!mbar_wait(bar(B_PFULL + 1), (j - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          pv(1, s0 + OFF_V + ((j - 1) & 1) * FA_TILE, j - 1 == 0);
+          pv(1, (j - 1) & 1, j - 1 == 0);
           umma_commit(bar(B_VEMPTY + ((j - 1) & 1)));
         }
-        qk(1, kb);                                              // S_j^1
+        qk(1, b);                                               // S_j^1
         umma_commit(bar(B_KEMPTY + b));
         if (!mbar_wait(bar(B_VFULL + b), ph, abort_flag) ||     // O_0 += P_j^0 V_j
             !mbar_wait(bar(B_PFULL + 0), j & 1, abort_flag)) {
@@ -235,13 +241,13 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
           break;
         }
         tc_fence_after();
-        pv(0, s0 + OFF_V + b * FA_TILE, j == 0);
+        pv(0, b, j == 0);
       }
       if (ok) {                                                 // O_1 += P_last^1 V_last
         const int jl = nb - 1;
         if (mbar_wait(bar(B_PFULL + 1), jl & 1, abort_flag)) {
           tc_fence_after();
-          pv(1, s0 + OFF_V + (jl & 1) * FA_TILE, jl == 0);
+          pv(1, jl & 1, jl == 0);
           umma_commit(bar(B_VEMPTY + (jl & 1)));
         } else {
           ok = false;
@@ -322,8 +328,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float a = exp2f(fmaf(__uint_as_float(v[c * 32 + e]), sl2, -base));
-          const float bb = exp2f(fmaf(__uint_as_float(v[c * 32 + e + 1]), sl2, -base));
+          const float a = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e]), sl2, -base));
+          const float bb = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e + 1]), sl2, -base));
           s8[(e >> 1) & 7] += a + bb;
           pk[e >> 1] = pack_bf16x2(a, bb);
         }

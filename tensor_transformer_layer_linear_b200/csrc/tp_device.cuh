@@ -254,7 +254,8 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t 
 // A shared-memory descriptor moved `bytes` further (16-byte units in the
 // start-address field; shared addresses stay below 256 KB, so no carry).
 __device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t bytes) {
-  return d + (bytes >> 4);
+  const uint32_t lo = static_cast<uint32_t>(d) + (bytes >> 4);  // a 32-bit add
+  return (d & 0xFFFFFFFF00000000ull) | lo;
 }
 
 // Instruction descriptor, kind::f16, bf16 in, fp32 accumulate, A K-major and
