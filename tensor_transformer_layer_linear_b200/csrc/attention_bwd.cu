@@ -455,7 +455,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(AB_DQEMPTY + b));  // the columns may be overwritten now
+      if (lane == 0) mbar_arrive_relaxed(bar(AB_DQEMPTY + b));  // the columns may be overwritten now
       const int q0 = step_block(it) * AB_BQ;
       const int nq_valid = min(AB_BQ, p.seq - q0);
       float* a = p.dq_acc + (head_row(it) * p.stride + row_base + q0) * AB_D + dcol;

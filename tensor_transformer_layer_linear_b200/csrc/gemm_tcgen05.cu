@@ -69,6 +69,8 @@ struct GemmParams {
   const uint16_t* bias;
   const uint16_t* aux;  // EPI_MUL_AUX: the factor GeLU'(Z) [G][M][Nc] bf16
   uint16_t* aux_out;    // EPI_GELU_AUX: receives GeLU'(Z) [G][M][Nc] bf16
+  float* out_f32;       // EPI_F32 with direct_store: D [G][M][Nc] fp32
+  int direct_store;     // EPI_F32: write rows with coalesced st.global instead of TMA stores
   unsigned* err;
 };
 
@@ -349,21 +351,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else {
-      uint32_t r[2][CW];
-      tmem_ld_32x32b_x32(tbase, &r[0][0]);
-      if constexpr (!OUT_F32) tmem_ld_32x32b_x32(tbase + 32, &r[0][32]);
+      // fp32 partials: the whole 32 x 128 slice goes to registers at once and
+      // the accumulator is handed back to the MMA before any store is issued,
+      // so the next-but-one tile's MMAs overlap this tile's (long) stores.
+      uint32_t r[OUT_F32 ? NCH : 2][CW];
+      if constexpr (OUT_F32) {
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) tmem_ld_32x32b_x32(tbase + c * CW, &r[c][0]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (CTAS == 2)
+            mbar_arrive_cluster_relaxed(mapa_shared(tempty_bar(acc), 0));  // the leader's barrier
+          else
+            mbar_arrive_relaxed(tempty_bar(acc));
+        }
+      } else {
+        tmem_ld_32x32b_x32(tbase, &r[0][0]);
+        tmem_ld_32x32b_x32(tbase + 32, &r[0][32]);
+      }
       const bool row_ok = row0 + lane < p.M;
       const int64_t aux_row = (static_cast<int64_t>(g) * p.M + row0 + lane) * p.Nc;
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
-        tmem_ld_wait();  // chunk c has arrived
-        if (c + 1 < NCH) {
-          tmem_ld_32x32b_x32(tbase + (c + 1) * CW, &r[(c + 1) & 1][0]);
-          if constexpr (!OUT_F32) tmem_ld_32x32b_x32(tbase + (c + 1) * CW + 32, &r[(c + 1) & 1][32]);
+        if constexpr (!OUT_F32) {
+          tmem_ld_wait();  // chunk c has arrived
+          if (c + 1 < NCH) {
+            tmem_ld_32x32b_x32(tbase + (c + 1) * CW, &r[(c + 1) & 1][0]);
+            tmem_ld_32x32b_x32(tbase + (c + 1) * CW + 32, &r[(c + 1) & 1][32]);
+          }
         }
         const int col0 = colh + c * CW;
         if (col0 >= p.Nc) continue;  // warp-uniform: the whole chunk is past the edge
-        const uint32_t* rc = r[c & 1];
+        const uint32_t* rc = r[OUT_F32 ? c : (c & 1)];
         uint32_t w[32];  // this thread's 128-byte row of the chunk
         uint32_t wg[(EPI == EPI_GELU_AUX) ? 32 : 1];  // and of GeLU'(Z)
         if constexpr (OUT_F32) {
@@ -414,18 +435,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         const uint32_t sbuf = sbase + (chunk_ctr % C::kStagingBufs) * 4096u;
         ++chunk_ctr;
-        if (lane == 0) bulk_wait_read<C::kStagingBufs - 1>();  // the store that last used sbuf read it
-        __syncwarp();
         const uint32_t row_addr = sbuf + static_cast<uint32_t>(lane) * 128u;
+        if (OUT_F32 && p.direct_store) {
+          // Transpose through the staging rows, then eight st.global.v4 per
+          // lane, each writing four full 128-byte row segments.
+          __syncwarp();  // the previous chunk's reads of sbuf are done
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4), w[4 * j],
-                       w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-        fence_proxy_async_shared();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_3d(&tmD, sbuf, col0, row0, g);
-          bulk_commit();
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4), w[4 * j],
+                         w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          __syncwarp();
+          const int u = lane & 7;
+          const int col = col0 + 4 * u;
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + (lane >> 3);
+            const float4 v = ld_shared_v4f(sbuf + static_cast<uint32_t>(rr) * 128u +
+                                           ((static_cast<uint32_t>(u) ^ (rr & 7u)) << 4));
+            if (row0 + rr < p.M && col < p.Nc)
+              __stcs(reinterpret_cast<float4*>(
+                         p.out_f32 + (static_cast<int64_t>(g) * p.M + row0 + rr) * p.Nc + col),
+                     v);
+          }
+        } else {
+          if (lane == 0) bulk_wait_read<C::kStagingBufs - 1>();  // the store that last used sbuf read it
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(row_addr + ((static_cast<uint32_t>(j) ^ (lane & 7u)) << 4), w[4 * j],
+                         w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmD, sbuf, col0, row0, g);
+            bulk_commit();
+          }
         }
         if constexpr (EPI == EPI_GELU_AUX) {
           // the same staging rows, once the store above has read them
@@ -444,13 +488,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       }  // EPI
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if constexpr (CTAS == 2)
-          mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));  // the leader's barrier
-        else
-          mbar_arrive(tempty_bar(acc));
+      if constexpr (!OUT_F32) {  // (fp32 partials released the accumulator above)
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (CTAS == 2)
+            mbar_arrive_cluster_relaxed(mapa_shared(tempty_bar(acc), 0));  // the leader's barrier
+          else
+            mbar_arrive_relaxed(tempty_bar(acc));
+        }
       }
       if (++acc == 2) {
         acc = 0;
@@ -545,6 +591,11 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
   p.bias = static_cast<const uint16_t*>(pr.bias);
   p.aux = static_cast<const uint16_t*>(pr.aux);
   p.aux_out = static_cast<uint16_t*>(pr.aux_out);
+  p.out_f32 = static_cast<float*>(pr.D);
+  // With K <= 256 a tile's MMAs take under half as long as its fp32 stores;
+  // there the stores from registers, which wait for no staging read-back,
+  // keep more bytes in flight than one TMA store per warp.
+  p.direct_store = (OUT_F32 && pr.K <= 256) ? 1 : 0;
   p.err = err;
   auto kern = gemm_tcgen05_kernel<BN, EPI, CTAS, A_MN, B_MN>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);

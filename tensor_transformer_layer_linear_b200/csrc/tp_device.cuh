@@ -352,6 +352,18 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
+// Arrivals that only report "this warp's TMEM reads are complete" (after
+// tcgen05.wait::ld and tcgen05.fence::before_thread_sync): they publish no
+// memory writes, so they use relaxed semantics. A release arrive would first
+// wait for the warp's global and bulk stores still in flight, which on B200
+// costs thousands of cycles per arrival in a store-heavy epilogue.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
 // TMA tile load into this CTA's shared memory whose completion is counted
 // on an mbarrier that may live in the peer CTA of the pair.
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void* tmap,
