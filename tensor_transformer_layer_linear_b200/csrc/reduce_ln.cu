@@ -195,6 +195,105 @@ __global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
   }
 }
 
+// The plain LayerNorm (no partials to sum): one warp per token row, eight
+// rows per CTA, every 16-byte load of the row issued before the first
+// reduction and warp shuffles only, so that a whole wave of rows streams at
+// once. CHW = 8-element chunks per lane (h <= CHW * 256); lane l holds chunks
+// l, l + 32, ... so each step of the warp reads 512 contiguous bytes. The
+// row value is bias + residual rounded to bf16 (written to Y_sum when given);
+// statistics are taken over the rounded values, population variance.
+template <int CHW>
+__global__ void __launch_bounds__(256) layernorm_rows_warp_kernel(
+    int64_t rows, int h, const uint16_t* __restrict__ bias, const uint16_t* __restrict__ res,
+    const uint16_t* __restrict__ gamma, const uint16_t* __restrict__ beta, float eps,
+    uint16_t* __restrict__ Ysum, uint16_t* __restrict__ Yln, SeqShard sp, int ln_natural) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int64_t row_off = row * h;
+  const int64_t sh_off = seq_shard_row(sp, row) * h;  // same row, sharded layout
+  const int64_t ln_off = ln_natural ? row_off : sh_off;
+  const int nch = h >> 3;
+  uint4 x[CHW];
+#pragma unroll
+  for (int c = 0; c < CHW; ++c) {
+    const int ch = lane + 32 * c;
+    x[c] = make_uint4(0u, 0u, 0u, 0u);
+    if (res != nullptr && ch < nch) x[c] = __ldg(reinterpret_cast<const uint4*>(res + sh_off + (ch << 3)));
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < CHW; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) {
+      float v[8] = {bf16_lo(x[c].x), bf16_hi(x[c].x), bf16_lo(x[c].y), bf16_hi(x[c].y),
+                    bf16_lo(x[c].z), bf16_hi(x[c].z), bf16_lo(x[c].w), bf16_hi(x[c].w)};
+      if (bias != nullptr) {
+        add_bf16x8(v, __ldg(reinterpret_cast<const uint4*>(bias + (ch << 3))));
+        x[c] = to_bf16x8(v);
+        v[0] = bf16_lo(x[c].x); v[1] = bf16_hi(x[c].x);
+        v[2] = bf16_lo(x[c].y); v[3] = bf16_hi(x[c].y);
+        v[4] = bf16_lo(x[c].z); v[5] = bf16_hi(x[c].z);
+        v[6] = bf16_lo(x[c].w); v[7] = bf16_hi(x[c].w);
+      }
+      if (Ysum != nullptr) *reinterpret_cast<uint4*>(Ysum + sh_off + (ch << 3)) = x[c];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s += v[j];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s / static_cast<float>(h);
+  float q = 0.f;
+#pragma unroll
+  for (int c = 0; c < CHW; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) {
+      const float v[8] = {bf16_lo(x[c].x), bf16_hi(x[c].x), bf16_lo(x[c].y), bf16_hi(x[c].y),
+                          bf16_lo(x[c].z), bf16_hi(x[c].z), bf16_lo(x[c].w), bf16_hi(x[c].w)};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float d = v[j] - mean;
+        q += d * d;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  const float rstd = rsqrtf(q / static_cast<float>(h) + eps);
+  if (Yln == nullptr) return;
+#pragma unroll
+  for (int c = 0; c < CHW; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) {
+      const uint4 g = __ldg(reinterpret_cast<const uint4*>(gamma + (ch << 3)));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(beta + (ch << 3)));
+      const float v[8] = {bf16_lo(x[c].x), bf16_hi(x[c].x), bf16_lo(x[c].y), bf16_hi(x[c].y),
+                          bf16_lo(x[c].z), bf16_hi(x[c].z), bf16_lo(x[c].w), bf16_hi(x[c].w)};
+      const float gv[8] = {bf16_lo(g.x), bf16_hi(g.x), bf16_lo(g.y), bf16_hi(g.y),
+                           bf16_lo(g.z), bf16_hi(g.z), bf16_lo(g.w), bf16_hi(g.w)};
+      const float bv[8] = {bf16_lo(b.x), bf16_hi(b.x), bf16_lo(b.y), bf16_hi(b.y),
+                           bf16_lo(b.z), bf16_hi(b.z), bf16_lo(b.w), bf16_hi(b.w)};
+      float y[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[j] = (v[j] - mean) * rstd * gv[j] + bv[j];
+      *reinterpret_cast<uint4*>(Yln + ln_off + (ch << 3)) = to_bf16x8(y);
+    }
+  }
+}
+
+template <int CHW>
+static void launch_ln_warp(int64_t rows, int64_t h, const void* bias, const void* residual,
+                           const void* gamma, const void* beta, float eps, void* Y_sum,
+                           void* Y_ln, cudaStream_t s, SeqShard sp, int ln_nat) {
+  const dim3 grid(static_cast<unsigned>((rows + 7) / 8));
+  layernorm_rows_warp_kernel<CHW><<<grid, 256, 0, s>>>(
+      rows, static_cast<int>(h), static_cast<const uint16_t*>(bias),
+      static_cast<const uint16_t*>(residual), static_cast<const uint16_t*>(gamma),
+      static_cast<const uint16_t*>(beta), eps, static_cast<uint16_t*>(Y_sum),
+      static_cast<uint16_t*>(Y_ln), sp, ln_nat);
+}
+
 int launch_reduce(const float* P, int n_shards, int64_t rows, int64_t h, const void* bias,
                   const void* residual, void* Y, cudaStream_t s, int num_sms, int sp_n,
                   int sp_batch, int sp_seq) {
@@ -258,7 +357,15 @@ int launch_rows_sum_ln(const float* P, int n_shards, int64_t rows, int64_t h, co
                        int sp_seq, int ln_natural) {
   if (rows <= 0) return 0;
   const SeqShard sp{sp_n, sp_batch, sp_seq};
-  if (n_shards == 0)
+  const int64_t nch = h / 8;
+  if (n_shards == 0 && nch <= 32 * 32) {
+    if (nch <= 32) launch_ln_warp<1>(rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_natural);
+    else if (nch <= 64) launch_ln_warp<2>(rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_natural);
+    else if (nch <= 128) launch_ln_warp<4>(rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_natural);
+    else if (nch <= 256) launch_ln_warp<8>(rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_natural);
+    else if (nch <= 512) launch_ln_warp<16>(rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_natural);
+    else launch_ln_warp<32>(rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp, ln_natural);
+  } else if (n_shards == 0)
     launch_rows<128>(P, n_shards, rows, h, bias, residual, gamma, beta, eps, Y_sum, Y_ln, s, sp,
                      ln_natural);
   else
