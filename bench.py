@@ -49,10 +49,12 @@ L2_BYTES = 126 * 1024 * 1024
 # committed ncu captures under profiles/, keyed by (workload, kernel). None
 # until a capture of the current kernel exists.
 NCU_TRAFFIC = {
-    # profiles/gemm_tcgen05_layer_ncu_full.md: QKV 244.1 MB and MLP-up 321.7 MB -> mean per launch
-    (DEFAULT_WORKLOAD, "gemm_column_parallel"): 282.9e6,
-    # same capture: W_O 545.1 MB and MLP-down 769.9 MB -> mean per launch
-    (DEFAULT_WORKLOAD, "gemm_row_parallel"): 657.5e6,
+    # profiles/layer_2x2048_h4096_n8_dram_traffic.md (dram__bytes_read.sum + write.sum per launch)
+    # QKV 244.1 MB and MLP-up 316.2 MB -> mean per launch
+    (DEFAULT_WORKLOAD, "gemm_column_parallel"): 280.2e6,
+    # W_O 540.5 MB and MLP-down 765.1 MB -> mean per launch
+    (DEFAULT_WORKLOAD, "gemm_row_parallel"): 652.8e6,
+    (DEFAULT_WORKLOAD, "attention"): 113.1e6,
 }
 
 
