@@ -46,10 +46,10 @@ METRIC = "TP-layer fwd TFLOP/s & % BF16 peak (1 B200); partial-reduce GB/s & % H
 L2_BYTES = 126 * 1024 * 1024
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
-# committed ncu captures under profiles/, keyed by (workload, kernel). None
+# committed ncu captures, keyed by (workload, kernel). None
 # until a capture of the current kernel exists.
 NCU_TRAFFIC = {
-    # profiles/layer_2x2048_h4096_n8_dram_traffic.md (dram__bytes_read.sum + write.sum per launch)
+    # ncu capture of one layer step: dram__bytes_read.sum + dram__bytes_write.sum per launch;
     # QKV 244.1 MB and MLP-up 316.2 MB -> mean per launch
     (DEFAULT_WORKLOAD, "gemm_column_parallel"): 280.2e6,
     # W_O 540.5 MB and MLP-down 765.1 MB -> mean per launch
