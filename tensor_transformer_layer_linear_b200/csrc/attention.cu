@@ -6,7 +6,8 @@
 // its own heads with no communication. With the shards held on one GPU, one
 // launch covers every (shard, sequence, local head, 128-query tile).
 //
-// One CTA per 128-query tile (d = 128), 8 warps:
+// A persistent kernel: one CTA per SM, each walking a share of the 128-query
+// tiles (d = 128), heaviest first; 8 warps:
 //   warps 0-3  softmax: one thread per query row (= TMEM lane). The row of S
 //              is read from TMEM into registers, masked on diagonal / tail
 //              blocks, its max taken, P = exp2(S scale - m) formed in fp32
@@ -14,25 +15,30 @@
 //              over the S columns. The running max moves lazily: O and the
 //              sum are rescaled only when the max grows by more than 2^8, so
 //              P stays <= 256 and O / l is unchanged (the same max scales
-//              numerator and denominator).
-//   warp 4     TMA: the Q tile once, then 128-key K blocks into a 2-deep ring
-//              straight out of the QKV projection's [shard][token][3h/N]
-//              output (128-byte swizzle).
+//              numerator and denominator). After a tile's last block they
+//              normalise O, store it and start on the next tile.
+//   warp 4     TMA: each tile's Q into a 2-deep ring (the next tile's Q loads
+//              while the current one runs), then 128-key K blocks into a
+//              2-deep ring straight out of the QKV projection's
+//              [shard][token][3h/N] output (128-byte swizzle).
 //   warp 6     TMA: the V blocks into their own 2-deep ring.
 //   warp 5     TMEM owner and the single MMA-issuing thread.
 // S is double-buffered in TMEM, so the MMAs of a key block overlap the
-// softmax of the previous one. MMA issue order:
+// softmax of the previous one. Blocks are numbered over the CTA's whole work
+// list, and the MMA order is
 //   S_0 = Q K_0^T | S_1 = Q K_1^T | O = P_0 V_0 | S_2 = Q K_2^T |
 //   O += P_1 V_1 | S_3 = Q K_3^T | ...
-// S_{j+2} overwrites the buffer holding P_j right after the MMA that reads
-// it, relying on one thread's tcgen05.mma operations executing in issue
-// order. A commit after every PV tells the softmax when O holds exactly the
-// blocks before its own (needed only for a rescale).
+// running on across tile boundaries (S of the next tile's first blocks is
+// computed while the softmax finishes the current tile). S_{n+2} overwrites
+// the buffer holding P_n right after the MMA that reads it, relying on one
+// thread's tcgen05.mma operations executing in issue order. A commit after
+// every PV tells the softmax when O holds exactly the blocks before its own
+// (needed only for a rescale); a commit after a tile's last PV releases its O
+// to the softmax warps, whose next P arrival in turn releases the columns.
 // TMEM: S / P buffer b at columns [128 b, 128 b + 128), O at [256, 384).
-// Causal CTAs stop at their diagonal block; heavy (late) query tiles launch
-// first. Every barrier wait is bounded; a role that gives up records an
-// error bit and the CTA leaves through the common exit after waiting
-// (bounded) for its copies and MMAs in flight.
+// Causal tiles stop at their diagonal block. Every barrier wait is bounded;
+// a role that gives up records an error bit and the CTA leaves through the
+// common exit after waiting (bounded) for its copies and MMAs in flight.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -43,26 +49,27 @@
 
 namespace tpk {
 
-constexpr int FA_BM = 128;                  // queries per tile (one tile per CTA)
+constexpr int FA_BM = 128;                  // queries per tile
 constexpr int FA_BN = 128;                  // keys per block
 constexpr int FA_D = 128;                   // head dim
 constexpr int FA_THREADS = 256;             // 8 warps: up to 255 registers per thread
 constexpr int FA_SUB = 128 * 128;           // one [128 rows][64 cols] bf16 box: 16 KB
 constexpr int FA_TILE = 2 * FA_SUB;         // a [128][128] bf16 tile: 32 KB
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + FA_TILE;      // 2 buffers
+constexpr int OFF_Q = 0;                    // 2 buffers (the next tile's Q loads early)
+constexpr int OFF_K = OFF_Q + 2 * FA_TILE;  // 2 buffers
 constexpr int OFF_V = OFF_K + 2 * FA_TILE;  // 2 buffers
 constexpr int OFF_BAR = OFF_V + 2 * FA_TILE;
-constexpr int FA_NUM_BARS = 16;
+constexpr int FA_NUM_BARS = 20;
 constexpr int FA_SMEM = 1024 + OFF_BAR + FA_NUM_BARS * 8 + 16;
 static_assert(FA_SMEM <= 232448, "shared memory budget");
 
-// barrier indices (K, V, S and P per buffer b)
-constexpr int B_Q = 0, B_KFULL = 1, B_VFULL = 3, B_KEMPTY = 5, B_VEMPTY = 7, B_SFULL = 9,
-              B_PFULL = 11, B_OUPD = 13, B_ODONE = 14;
+// barrier indices (Q, K, V, S and P per buffer b)
+constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = 6, B_VFULL = 8, B_VEMPTY = 10,
+              B_SFULL = 12, B_PFULL = 14, B_OUPD = 16, B_ODONE = 17, B_DRAIN = 18;
 
 struct AttnParams {
   int seq, batch, hps, causal, nq;
+  int n_units;  // (shard, sequence, local head) triples
   int q_w;    // query columns per shard (query heads per shard x 128)
   int kv_w;   // key (= value) columns per shard
   int group;  // local query heads per local kv head
@@ -72,6 +79,39 @@ struct AttnParams {
   long long lse_stride;  // per (shard, head): tokens per shard + 128
   unsigned* err;
 };
+
+// One query tile of the work list. Tiles are ordered heaviest first (for
+// causal attention, the latest query tiles see the most key blocks) and dealt
+// to the persistent CTAs in a snake: CTA c takes tile k G + c in even rounds k
+// and k G + G - 1 - c in odd ones (G CTAs), which evens out the causal work.
+struct AttnTile {
+  bool valid;
+  int head, g, q0, row_base, nb, kcol, vcol;
+};
+
+__device__ __forceinline__ AttnTile attn_tile(const AttnParams& p, int round) {
+  AttnTile t;
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const int w = round * G + ((round & 1) ? (G - 1 - c) : c);
+  t.valid = w < p.nq * p.n_units;
+  const int wi = t.valid ? w : 0;
+  const int qi = wi / p.n_units, y = wi % p.n_units;
+  const int qt = p.causal ? (p.nq - 1 - qi) : qi;
+  t.head = y % p.hps;
+  const int sidx = (y / p.hps) % p.batch;
+  t.g = y / (p.hps * p.batch);
+  t.q0 = qt * FA_BM;
+  t.row_base = sidx * p.seq;  // first token of the sequence within the shard
+  t.nb = (p.seq + FA_BN - 1) / FA_BN;
+  if (p.causal) {
+    const int last = (t.q0 + FA_BM - 1) / FA_BN + 1;
+    if (last < t.nb) t.nb = last;
+  }
+  const int kvh = t.head / p.group;  // the query head's local kv head
+  t.kcol = p.q_w + kvh * FA_D;
+  t.vcol = p.q_w + p.kv_w + kvh * FA_D;
+  return t;
+}
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
@@ -93,33 +133,21 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qt = p.causal ? (p.nq - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
-  const int y = blockIdx.y;
-  const int head = y % p.hps;
-  const int sidx = (y / p.hps) % p.batch;
-  const int g = y / (p.hps * p.batch);
-  const int q0 = qt * FA_BM;
-  const int row_base = sidx * p.seq;  // first token of this sequence within the shard
-  int nb = (p.seq + FA_BN - 1) / FA_BN;
-  if (p.causal) {
-    const int last = (q0 + FA_BM - 1) / FA_BN + 1;
-    if (last < nb) nb = last;
-  }
-  const int kvh = head / p.group;  // this query head's local kv head
-  const int kcol = p.q_w + kvh * FA_D, vcol = p.q_w + p.kv_w + kvh * FA_D;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(B_Q), 1);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(B_QFULL + b), 1);
+      mbar_init(bar(B_QEMPTY + b), 1);
       mbar_init(bar(B_KFULL + b), 1);
-      mbar_init(bar(B_VFULL + b), 1);
       mbar_init(bar(B_KEMPTY + b), 1);
+      mbar_init(bar(B_VFULL + b), 1);
       mbar_init(bar(B_VEMPTY + b), 1);
       mbar_init(bar(B_SFULL + b), 1);
       mbar_init(bar(B_PFULL + b), 4);  // one arrival per softmax warp
     }
     mbar_init(bar(B_OUPD), 1);
     mbar_init(bar(B_ODONE), 1);
+    mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -132,31 +160,45 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 
   if (warp == 4 || warp == 6) {
     // ------------------------------------------------------------ TMA (Q + K | V)
+    // Blocks are counted over the CTA's whole work list, so the rings run on
+    // across tile boundaries and the next tile's Q and first K / V blocks
+    // load while the current tile finishes.
     if (lane == 0) {
       const bool is_k = warp == 4;
-      const int col = is_k ? kcol : vcol;
       const int full = is_k ? B_KFULL : B_VFULL, empty = is_k ? B_KEMPTY : B_VEMPTY;
       const uint32_t ring = s0 + (is_k ? OFF_K : OFF_V);
       bool ok = true;
-      if (is_k) {
-        mbar_arrive_expect_tx(bar(B_Q), FA_TILE);
-        const int qrow = row_base + q0;
-        tma_load_3d(s0 + OFF_Q, &tm, bar(B_Q), head * FA_D, qrow, g);
-        tma_load_3d(s0 + OFF_Q + FA_SUB, &tm, bar(B_Q), head * FA_D + 64, qrow, g);
-      }
-      int issued = 0;
-      for (int j = 0; j < nb; ++j) {
-        const int b = j & 1;
-        if (!mbar_wait(bar(empty + b), ((j >> 1) & 1) ^ 1u, abort_flag)) {
-          ok = false;
-          break;
+      int nblk = 0, ntile = 0;  // blocks and tiles issued
+      for (int round = 0; ok; ++round) {
+        const AttnTile t = attn_tile(p, round);
+        if (!t.valid) break;
+        if (is_k) {
+          const int qb = ntile & 1;
+          if (!mbar_wait(bar(B_QEMPTY + qb), ((ntile >> 1) & 1) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(B_QFULL + qb), FA_TILE);
+          const uint32_t qd = s0 + OFF_Q + qb * FA_TILE;
+          tma_load_3d(qd, &tm, bar(B_QFULL + qb), t.head * FA_D, t.row_base + t.q0, t.g);
+          tma_load_3d(qd + FA_SUB, &tm, bar(B_QFULL + qb), t.head * FA_D + 64, t.row_base + t.q0,
+                      t.g);
         }
-        const uint32_t d = ring + b * FA_TILE;
-        const int krow = row_base + j * FA_BN;
-        mbar_arrive_expect_tx(bar(full + b), FA_TILE);
-        tma_load_3d(d, &tm, bar(full + b), col, krow, g);
-        tma_load_3d(d + FA_SUB, &tm, bar(full + b), col + 64, krow, g);
-        ++issued;
+        ++ntile;
+        const int col = is_k ? t.kcol : t.vcol;
+        for (int j = 0; j < t.nb; ++j) {
+          const int b = nblk & 1;
+          if (!mbar_wait(bar(empty + b), ((nblk >> 1) & 1) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t d = ring + b * FA_TILE;
+          const int krow = t.row_base + j * FA_BN;
+          mbar_arrive_expect_tx(bar(full + b), FA_TILE);
+          tma_load_3d(d, &tm, bar(full + b), col, krow, t.g);
+          tma_load_3d(d + FA_SUB, &tm, bar(full + b), col + 64, krow, t.g);
+          ++nblk;
+        }
       }
       if (!ok) {
         atomicOr(p.err, ERR_WAIT_ATTN);
@@ -164,27 +206,48 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       }
       // every load issued must land before the CTA exits
       int never = 0;
-      if (is_k && !mbar_wait(bar(B_Q), 0, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
-      for (int jj = (issued >= 2 ? issued - 2 : 0); jj < issued; ++jj)
+      if (is_k)
+        for (int i = (ntile >= 2 ? ntile - 2 : 0); i < ntile; ++i)
+          if (!mbar_wait(bar(B_QFULL + (i & 1)), (i >> 1) & 1, &never))
+            atomicOr(p.err, ERR_WAIT_DRAIN);
+      for (int jj = (nblk >= 2 ? nblk - 2 : 0); jj < nblk; ++jj)
         if (!mbar_wait(bar(full + (jj & 1)), (jj >> 1) & 1, &never))
           atomicOr(p.err, ERR_WAIT_DRAIN);
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA
+    // Two cursors walk the work list: the QK^T cursor runs two blocks ahead
+    // of the PV cursor (S is double-buffered), across tile boundaries.
     if (lane == 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16_f32(FA_BM, FA_BN);
       constexpr uint32_t idesc_o = umma_idesc_bf16_f32_bmn(FA_BM, FA_D);
       // descriptors built once; each MMA moves them by a constant offset
-      const uint64_t dq = umma_desc_sw128(s0 + OFF_Q);
+      const uint64_t dq0 = umma_desc_sw128(s0 + OFF_Q), dq1 = umma_desc_sw128(s0 + OFF_Q + FA_TILE);
       const uint64_t dk0 = umma_desc_sw128(s0 + OFF_K), dk1 = umma_desc_sw128(s0 + OFF_K + FA_TILE);
       const uint64_t dv0 = umma_desc_sw128_mn(s0 + OFF_V, FA_SUB);
       const uint64_t dv1 = umma_desc_sw128_mn(s0 + OFF_V + FA_TILE, FA_SUB);
-      // S_j = Q K_j^T into buffer j & 1
-      auto qk = [&](int j) -> bool {
-        const int b = j & 1;
-        if (!mbar_wait(bar(B_KFULL + b), (j >> 1) & 1, abort_flag)) return false;
+      struct Cursor {
+        AttnTile t;
+        int round, tile, j, blk;  // work-list round, local tile, block within it, global block
+      };
+      Cursor cq{attn_tile(p, 0), 0, 0, 0, 0};
+      Cursor cp = cq;
+      auto advance = [&](Cursor& c) {
+        ++c.blk;
+        if (++c.j == c.t.nb) {
+          c.j = 0;
+          ++c.tile;
+          c.t = attn_tile(p, ++c.round);
+        }
+      };
+      bool ok = true;
+      // S_blk = Q K_blk^T into buffer blk & 1
+      auto qk = [&]() -> bool {
+        const int qb = cq.tile & 1, b = cq.blk & 1;
+        if (cq.j == 0 && !mbar_wait(bar(B_QFULL + qb), (cq.tile >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar(B_KFULL + b), (cq.blk >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint64_t dk = b ? dk1 : dk0;
+        const uint64_t dq = qb ? dq1 : dq0, dk = b ? dk1 : dk0;
 #pragma unroll
         for (int kk = 0; kk < FA_D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * FA_SUB + (kk & 3) * 32;
@@ -193,14 +256,14 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
         umma_commit(bar(B_KEMPTY + b));
         umma_commit(bar(B_SFULL + b));
+        if (cq.j == cq.t.nb - 1) umma_commit(bar(B_QEMPTY + qb));  // the tile's last QK^T
+        advance(cq);
         return true;
       };
-      bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
-      if (ok) ok = qk(0);
-      if (ok && nb > 1) ok = qk(1);
-      for (int j = 0; ok && j < nb; ++j) {
-        const int b = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
+      for (int n = 0; ok && n < 2 && cq.t.valid; ++n) ok = qk();
+      while (ok && cp.t.valid) {
+        const int b = cp.blk & 1;
+        const uint32_t ph = (cp.blk >> 1) & 1;
         if (!mbar_wait(bar(B_VFULL + b), ph, abort_flag) ||
             !mbar_wait(bar(B_PFULL + b), ph, abort_flag)) {
           ok = false;
@@ -209,113 +272,124 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         tc_fence_after();
         const uint64_t dv = b ? dv1 : dv0;
 #pragma unroll
-        for (int kk = 0; kk < FA_BN / 16; ++kk)             // O (+)= P_j V_j
+        for (int kk = 0; kk < FA_BN / 16; ++kk)             // O (+)= P V
           umma_bf16_tmem_a(tmem + 2 * FA_BN, tmem + b * FA_BN + kk * 8,
-                           desc_advance(dv, kk * 2048), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                           desc_advance(dv, kk * 2048), idesc_o, (cp.j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(B_VEMPTY + b));
         umma_commit(bar(B_OUPD));
-        if (j + 2 < nb) ok = qk(j + 2);                    // reuses the buffer P_j was in
+        if (cp.j == cp.t.nb - 1) umma_commit(bar(B_ODONE));  // the tile's O is complete
+        advance(cp);
+        if (cq.t.valid) ok = qk();                           // reuses the buffer P was in
       }
       if (!ok) {
         atomicOr(p.err, ERR_WAIT_ATTN);
         *abort_flag = 1;
       }
-      // o_done doubles as the drain of every MMA this thread issued
-      umma_commit(bar(B_ODONE));
+      // drain every MMA this thread issued
+      umma_commit(bar(B_DRAIN));
       int never = 0;
-      if (!mbar_wait(bar(B_ODONE), 0, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
+      if (!mbar_wait(bar(B_DRAIN), 0, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ softmax
     const int r = warp * 32 + lane;  // row within the tile (= TMEM lane)
-    const int t = q0 + r;            // query position within the sequence
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t o_cols = tmem + lane_addr + 2 * FA_BN;
     const float sl2 = p.scale_log2;
-    float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nb; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(bar(B_SFULL + b), (j >> 1) & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t s_cols = tmem + lane_addr + b * FA_BN;
-      const int k0 = j * FA_BN;
-      uint32_t v[FA_BN];
-#pragma unroll
-      for (int c = 0; c < FA_BN / 32; ++c) tmem_ld_32x32b_x32(s_cols + c * 32, &v[c * 32]);
-      tmem_ld_wait();
-      if (k0 + FA_BN > p.seq || (p.causal && k0 + FA_BN - 1 > q0)) {
-        // keys k0 + e with e >= lim are past the sequence or (causal) after t
-        const int lim = min(p.seq, p.causal ? t + 1 : p.seq) - k0;
-#pragma unroll
-        for (int e = 0; e < FA_BN; ++e) v[e] = e < lim ? v[e] : 0xFF800000u;  // -inf
-      }
-      float m8[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) m8[u] = fmaxf(__uint_as_float(v[u]), __uint_as_float(v[u + 8]));
-#pragma unroll
-      for (int e = 16; e < FA_BN; e += 16) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          m8[u] = fmax3(m8[u], __uint_as_float(v[e + u]), __uint_as_float(v[e + 8 + u]));
-      }
-      const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-      // lazy max: move it (and rescale) only when exp2 would exceed 2^8
-      const bool need = (mx != -INFINITY) && ((mx - m_used) * sl2 > 8.f);
-      float alpha = 1.f;
-      if (need) {
-        alpha = exp2f((m_used - mx) * sl2);  // 0 when m_used is still -inf
-        l *= alpha;
-        m_used = mx;
-      }
-      if (__any_sync(0xffffffffu, need && j > 0)) {
-        // O must hold exactly the blocks before j: wait for PV_{j-1}
-        if (!mbar_wait(bar(B_OUPD), (j - 1) & 1, abort_flag)) {
+    int blk = 0;  // global block count of this CTA
+    for (int round = 0, tile = 0; ok; ++round, ++tile) {
+      const AttnTile tl = attn_tile(p, round);
+      if (!tl.valid) break;
+      const int q0 = tl.q0;
+      const int t = q0 + r;  // query position within the sequence
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < tl.nb; ++j, ++blk) {
+        const int b = blk & 1;
+        if (!mbar_wait(bar(B_SFULL + b), (blk >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t s_cols = tmem + lane_addr + b * FA_BN;
+        const int k0 = j * FA_BN;
+        uint32_t v[FA_BN];
+#pragma unroll
+        for (int c = 0; c < FA_BN / 32; ++c) tmem_ld_32x32b_x32(s_cols + c * 32, &v[c * 32]);
+        tmem_ld_wait();
+        if (k0 + FA_BN > p.seq || (p.causal && k0 + FA_BN - 1 > q0)) {
+          // keys k0 + e with e >= lim are past the sequence or (causal) after t
+          const int lim = min(p.seq, p.causal ? t + 1 : p.seq) - k0;
+#pragma unroll
+          for (int e = 0; e < FA_BN; ++e) v[e] = e < lim ? v[e] : 0xFF800000u;  // -inf
+        }
+        float m8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m8[u] = fmaxf(__uint_as_float(v[u]), __uint_as_float(v[u + 8]));
+#pragma unroll
+        for (int e = 16; e < FA_BN; e += 16) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            m8[u] = fmax3(m8[u], __uint_as_float(v[e + u]), __uint_as_float(v[e + 8 + u]));
+        }
+        const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+        // lazy max: move it (and rescale) only when exp2 would exceed 2^8
+        const bool need = (mx != -INFINITY) && ((mx - m_used) * sl2 > 8.f);
+        float alpha = 1.f;
+        if (need) {
+          alpha = exp2f((m_used - mx) * sl2);  // 0 when m_used is still -inf
+          l *= alpha;
+          m_used = mx;
+        }
+        if (__any_sync(0xffffffffu, need && j > 0)) {
+          // O must hold exactly the tile's blocks before j: wait for the previous PV
+          if (!mbar_wait(bar(B_OUPD), (blk - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < FA_D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(o_cols + c * 32, o);
-          tmem_ld_wait();
+          for (int c = 0; c < FA_D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(o_cols + c * 32, o);
+            tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st_32x32b_x32(o_cols + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st_32x32b_x32(o_cols + c * 32, o);
+          }
         }
-      }
-      const float base = (m_used == -INFINITY) ? 0.f : m_used * sl2;
-      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float base = (m_used == -INFINITY) ? 0.f : m_used * sl2;
+        float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < FA_BN / 32; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < FA_BN / 32; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float a = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e]), sl2, -base));
-          const float bb = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e + 1]), sl2, -base));
-          s8[(e >> 1) & 7] += a + bb;
-          pk[e >> 1] = pack_bf16x2(a, bb);
+          for (int e = 0; e < 32; e += 2) {
+            const float a = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e]), sl2, -base));
+            const float bb = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e + 1]), sl2, -base));
+            s8[(e >> 1) & 7] += a + bb;
+            pk[e >> 1] = pack_bf16x2(a, bb);
+          }
+          tmem_st_32x32b_x16(s_cols + c * 16, pk);
         }
-        tmem_st_32x32b_x16(s_cols + c * 16, pk);
+        l += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PFULL + b));
       }
-      l += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_PFULL + b));
-    }
-    if (!ok) {
-      if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
-      *abort_flag = 1;
-    } else if (mbar_wait(bar(B_ODONE), 0, abort_flag)) {
+      if (!ok) break;
+      // the tile's O: normalise, store, and release the columns (the next
+      // tile's first PV overwrites them only after this warp's next P arrive)
+      if (!mbar_wait(bar(B_ODONE), tile & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float base_final = (m_used == -INFINITY) ? 0.f : m_used * sl2;
-      uint16_t* orow = O + (static_cast<int64_t>(g) * p.M + row_base + t) * p.q_w + head * FA_D;
+      uint16_t* orow =
+          O + (static_cast<int64_t>(tl.g) * p.M + tl.row_base + t) * p.q_w + tl.head * FA_D;
 #pragma unroll 1
       for (int c = 0; c < FA_D / 32; ++c) {
         uint32_t o[32];
@@ -335,9 +409,10 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       }
       // P = exp2(s sl2 - base) / l = exp2(s sl2 - (base + log2 l))
       if (p.lse != nullptr && t < p.seq)
-        p.lse[(static_cast<int64_t>(g) * p.hps + head) * p.lse_stride + row_base + t] =
+        p.lse[(static_cast<int64_t>(tl.g) * p.hps + tl.head) * p.lse_stride + tl.row_base + t] =
             base_final + log2f(l);
-    } else {
+    }
+    if (!ok) {
       if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
       *abort_flag = 1;
     }
@@ -400,8 +475,20 @@ int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, i
   p.lse = lse;
   p.lse_stride = M + 128;
   p.err = err;
+  p.n_units = static_cast<int>(n_shards * batch * hps);
   cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM);
-  const dim3 grid(p.nq, static_cast<unsigned>(n_shards * batch * hps));
+  // persistent: one CTA per SM (shared memory and TMEM admit one), each
+  // walking its share of the query tiles
+  static int num_sms = 0;
+  if (num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        num_sms <= 0)
+      return 2;
+  }
+  const int64_t tiles = static_cast<int64_t>(p.nq) * p.n_units;
+  const dim3 grid(static_cast<unsigned>(tiles < num_sms ? tiles : num_sms));
   attention_tc_kernel<<<grid, FA_THREADS, FA_SMEM, s>>>(tm, static_cast<uint16_t*>(O), p);
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
