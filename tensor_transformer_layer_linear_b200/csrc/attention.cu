@@ -15,8 +15,9 @@
 //              over the S columns. The running max moves lazily: O and the
 //              sum are rescaled only when the max grows by more than 2^8, so
 //              P stays <= 256 and O / l is unchanged (the same max scales
-//              numerator and denominator). After a tile's last block they
-//              normalise O, store it and start on the next tile.
+//              numerator and denominator). A tile's O is normalised and
+//              stored once the next tile's first P is formed, so the wait for
+//              the tile's last PV overlaps that work.
 //   warp 4     TMA: each tile's Q into a 2-deep ring (the next tile's Q loads
 //              while the current one runs), then 128-key K blocks into a
 //              2-deep ring straight out of the QKV projection's
@@ -297,8 +298,47 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     const uint32_t o_cols = tmem + lane_addr + 2 * FA_BN;
     const float sl2 = p.scale_log2;
     bool ok = true;
+    // A tile's O: normalise and store it. It runs after the next tile's first
+    // P is formed (its wait for the last PV overlaps that work) and before
+    // that P's arrival, which is what lets the next tile's first PV
+    // overwrite the O columns.
+    auto epilogue = [&](const AttnTile& tl, int tile, float m_used, float l) -> bool {
+      if (!mbar_wait(bar(B_ODONE), tile & 1, abort_flag)) return false;
+      tc_fence_after();
+      const int t = tl.q0 + r;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float base_final = (m_used == -INFINITY) ? 0.f : m_used * sl2;
+      uint16_t* orow =
+          O + (static_cast<int64_t>(tl.g) * p.M + tl.row_base + t) * p.q_w + tl.head * FA_D;
+#pragma unroll 1
+      for (int c = 0; c < FA_D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(o_cols + c * 32, o);
+        tmem_ld_wait();
+        if (t < p.seq) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + 8 * e) = w;
+          }
+        }
+      }
+      // P = exp2(s sl2 - base) / l = exp2(s sl2 - (base + log2 l))
+      if (p.lse != nullptr && t < p.seq)
+        p.lse[(static_cast<int64_t>(tl.g) * p.hps + tl.head) * p.lse_stride + tl.row_base + t] =
+            base_final + log2f(l);
+      return true;
+    };
+    AttnTile prev{};
+    float prev_m = -INFINITY, prev_l = 0.f;
+    bool pending = false;  // prev's O still to be stored
     int blk = 0;  // global block count of this CTA
-    for (int round = 0, tile = 0; ok; ++round, ++tile) {
+    int tile = 0;
+    for (int round = 0; ok; ++round, ++tile) {
       const AttnTile tl = attn_tile(p, round);
       if (!tl.valid) break;
       const int q0 = tl.q0;
@@ -373,45 +413,25 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
           tmem_st_32x32b_x16(s_cols + c * 16, pk);
         }
         l += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+        if (j == 0 && pending) {
+          if (!epilogue(prev, tile - 1, prev_m, prev_l)) {
+            ok = false;
+            break;
+          }
+          pending = false;
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_PFULL + b));
       }
       if (!ok) break;
-      // the tile's O: normalise, store, and release the columns (the next
-      // tile's first PV overwrites them only after this warp's next P arrive)
-      if (!mbar_wait(bar(B_ODONE), tile & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float base_final = (m_used == -INFINITY) ? 0.f : m_used * sl2;
-      uint16_t* orow =
-          O + (static_cast<int64_t>(tl.g) * p.M + tl.row_base + t) * p.q_w + tl.head * FA_D;
-#pragma unroll 1
-      for (int c = 0; c < FA_D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld_32x32b_x32(o_cols + c * 32, o);
-        tmem_ld_wait();
-        if (t < p.seq) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + 8 * e) = w;
-          }
-        }
-      }
-      // P = exp2(s sl2 - base) / l = exp2(s sl2 - (base + log2 l))
-      if (p.lse != nullptr && t < p.seq)
-        p.lse[(static_cast<int64_t>(tl.g) * p.hps + tl.head) * p.lse_stride + tl.row_base + t] =
-            base_final + log2f(l);
+      prev = tl;
+      prev_m = m_used;
+      prev_l = l;
+      pending = true;
     }
+    if (ok && pending && !epilogue(prev, tile - 1, prev_m, prev_l)) ok = false;
     if (!ok) {
       if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
       *abort_flag = 1;
