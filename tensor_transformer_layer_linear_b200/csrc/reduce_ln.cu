@@ -136,6 +136,20 @@ __global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
   const int nch = h >> 3;
   float v[CH][8];
   float s = 0.f;
+  // gamma and beta of this thread's chunks, in flight with the row's loads
+  // (not one L2 round trip per chunk after the statistics); wide rows load
+  // them per chunk instead, to stay within the register budget
+  constexpr bool kPre = CH <= 4;
+  uint4 gq[kPre ? CH : 1], bq[kPre ? CH : 1];
+#pragma unroll
+  for (int c = 0; c < (kPre ? CH : 0); ++c) {
+    const int ch = threadIdx.x + c * kRowThreads;
+    gq[c] = bq[c] = make_uint4(0u, 0u, 0u, 0u);
+    if (Yln != nullptr && ch < nch) {
+      gq[c] = __ldg(reinterpret_cast<const uint4*>(gamma + (ch << 3)));
+      bq[c] = __ldg(reinterpret_cast<const uint4*>(beta + (ch << 3)));
+    }
+  }
 #pragma unroll
   for (int c = 0; c < CH; ++c) {
     const int ch = threadIdx.x + c * kRowThreads;
@@ -181,8 +195,8 @@ __global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
   for (int c = 0; c < CH; ++c) {
     const int ch = threadIdx.x + c * kRowThreads;
     if (ch < nch) {
-      const uint4 g = __ldg(reinterpret_cast<const uint4*>(gamma + (ch << 3)));
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(beta + (ch << 3)));
+      const uint4 g = kPre ? gq[kPre ? c : 0] : __ldg(reinterpret_cast<const uint4*>(gamma + (ch << 3)));
+      const uint4 b = kPre ? bq[kPre ? c : 0] : __ldg(reinterpret_cast<const uint4*>(beta + (ch << 3)));
       float gv[8] = {bf16_lo(g.x), bf16_hi(g.x), bf16_lo(g.y), bf16_hi(g.y),
                      bf16_lo(g.z), bf16_hi(g.z), bf16_lo(g.w), bf16_hi(g.w)};
       float bv[8] = {bf16_lo(b.x), bf16_hi(b.x), bf16_lo(b.y), bf16_hi(b.y),
@@ -201,19 +215,29 @@ __global__ void __launch_bounds__(kRowThreads) rows_sum_ln_kernel(
 // once. CHW = 8-element chunks per lane (h <= CHW * 256); lane l holds chunks
 // l, l + 32, ... so each step of the warp reads 512 contiguous bytes. The
 // row value is bias + residual rounded to bf16 (written to Y_sum when given);
-// statistics are taken over the rounded values, population variance.
+// statistics are taken over the rounded values, population variance. gamma
+// and beta are staged in shared memory once per CTA (read per chunk from
+// global memory they cost one L2 round trip per chunk after the statistics).
 template <int CHW>
 __global__ void __launch_bounds__(256) layernorm_rows_warp_kernel(
     int64_t rows, int h, const uint16_t* __restrict__ bias, const uint16_t* __restrict__ res,
     const uint16_t* __restrict__ gamma, const uint16_t* __restrict__ beta, float eps,
     uint16_t* __restrict__ Ysum, uint16_t* __restrict__ Yln, SeqShard sp, int ln_natural) {
+  extern __shared__ uint4 gb_s[];  // [2][h / 8]: gamma, then beta
   const int lane = threadIdx.x & 31;
+  const int nch = h >> 3;
+  if (Yln != nullptr) {
+    for (int i = threadIdx.x; i < nch; i += blockDim.x) {
+      gb_s[i] = __ldg(reinterpret_cast<const uint4*>(gamma) + i);
+      gb_s[nch + i] = __ldg(reinterpret_cast<const uint4*>(beta) + i);
+    }
+  }
+  __syncthreads();
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int64_t row_off = row * h;
   const int64_t sh_off = seq_shard_row(sp, row) * h;  // same row, sharded layout
   const int64_t ln_off = ln_natural ? row_off : sh_off;
-  const int nch = h >> 3;
   uint4 x[CHW];
 #pragma unroll
   for (int c = 0; c < CHW; ++c) {
@@ -266,8 +290,8 @@ __global__ void __launch_bounds__(256) layernorm_rows_warp_kernel(
   for (int c = 0; c < CHW; ++c) {
     const int ch = lane + 32 * c;
     if (ch < nch) {
-      const uint4 g = __ldg(reinterpret_cast<const uint4*>(gamma + (ch << 3)));
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(beta + (ch << 3)));
+      const uint4 g = gb_s[ch];
+      const uint4 b = gb_s[nch + ch];
       const float v[8] = {bf16_lo(x[c].x), bf16_hi(x[c].x), bf16_lo(x[c].y), bf16_hi(x[c].y),
                           bf16_lo(x[c].z), bf16_hi(x[c].z), bf16_lo(x[c].w), bf16_hi(x[c].w)};
       const float gv[8] = {bf16_lo(g.x), bf16_hi(g.x), bf16_lo(g.y), bf16_hi(g.y),
@@ -287,7 +311,8 @@ static void launch_ln_warp(int64_t rows, int64_t h, const void* bias, const void
                            const void* gamma, const void* beta, float eps, void* Y_sum,
                            void* Y_ln, cudaStream_t s, SeqShard sp, int ln_nat) {
   const dim3 grid(static_cast<unsigned>((rows + 7) / 8));
-  layernorm_rows_warp_kernel<CHW><<<grid, 256, 0, s>>>(
+  const size_t smem = Y_ln != nullptr ? static_cast<size_t>(h / 8) * 2 * sizeof(uint4) : 0;
+  layernorm_rows_warp_kernel<CHW><<<grid, 256, smem, s>>>(
       rows, static_cast<int>(h), static_cast<const uint16_t*>(bias),
       static_cast<const uint16_t*>(residual), static_cast<const uint16_t*>(gamma),
       static_cast<const uint16_t*>(beta), eps, static_cast<uint16_t*>(Y_sum),
