@@ -223,6 +223,38 @@ def test_attention(tp, n, causal):
         assert_parity(got[i], ref, f"shard {i}")
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_attention_more_tiles_than_sms(tp, causal):
+    """512 query tiles (2 shards x 2 sequences x 16 heads x 8 tiles of a
+    1000-token sequence, the last ragged) over the persistent CTAs: every CTA
+    walks several tiles, so the Q ring, the block numbering across tiles and
+    the deferred O store of each tile are all exercised. Every output and, for
+    two heads per shard, the log-sum-exp are checked."""
+    rng = np.random.default_rng(870 + int(causal))
+    n, batch, seq, n_heads, d = 2, 2, 1000, 32, 128
+    h = n_heads * d
+    hs, hps = h // n, n_heads // n
+    M = batch * seq
+    QKV = _rand_bits(rng, (n, M, 3 * hs))
+    O_ = torch.empty((n, M, hs), dtype=torch.int16, device="cuda")
+    lse = torch.empty(n * hps * (M + 128), dtype=torch.float32, device="cuda")
+    tp.tp_attention_lse(to_dev(QKV), batch, seq, h, n_heads, causal, n, O_, lse)
+    got = from_dev_bf16(O_)
+    lse_h = lse.cpu().numpy().reshape(n * hps, M + 128)
+    q = f64(QKV)
+    for i in range(n):
+        Q, K, V = q[i][:, :hs], q[i][:, hs:2 * hs], q[i][:, 2 * hs:]
+        ref = O.attention_heads(Q, K, V, batch, seq, hps, causal)
+        assert_parity(got[i], ref, f"shard {i}")
+        for kk in (0, hps - 1):
+            c = slice(kk * d, (kk + 1) * d)
+            for s in range(batch):
+                r = slice(s * seq, (s + 1) * seq)
+                np.testing.assert_allclose(lse_h[i * hps + kk, r] * np.log(2.0),
+                                           O.attention_logsumexp(Q[r, c], K[r, c], causal),
+                                           rtol=0, atol=2e-3)
+
+
 def test_attention_first_query_sees_itself(tp):
     """Causal: the first query of every sequence returns its own V row."""
     rng = np.random.default_rng(850)
