@@ -54,6 +54,8 @@ NCU_TRAFFIC = {
     (DEFAULT_WORKLOAD, "gemm_column_parallel"): 280.2e6,
     # W_O 540.5 MB and MLP-down 765.1 MB -> mean per launch
     (DEFAULT_WORKLOAD, "gemm_row_parallel"): 652.8e6,
+    # persistent attention: 134.5 MB read + 13.6 MB written
+    (DEFAULT_WORKLOAD, "attention"): 148.1e6,
 }
 
 
