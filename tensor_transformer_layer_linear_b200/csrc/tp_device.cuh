@@ -409,16 +409,6 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
 }
 
 
-// Warpgroup register reallocation (all four warps of a warpgroup execute it).
-template <int N>
-__device__ __forceinline__ void setmaxnreg_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void setmaxnreg_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // Row m = b S + s of the token-ordered [batch][S] rows, stored in the
 // sequence-sharded layout [N][batch][S/N]: shard s / (S/N) keeps positions
 // [i S/N, (i+1) S/N) of every sequence ("Sequence Parallelism"). sp.n == 0
