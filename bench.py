@@ -440,6 +440,23 @@ class Model:
                               X if cfg.get("residual") else None, self.ws, self.ws_bytes, Y)
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest x over all ranks, returned on every rank (x itself
+    without a process group): a step time is the slowest rank's."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
+    """Weak scaling: every rank runs its own replica of the workload, so the
+    job's throughput is all ranks' work over the slowest rank's time."""
+    return flops_per_rank * world / (ms * 1e-3) / 1e12
+
+
 def run_ours(args, cfg) -> None:
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -491,10 +508,7 @@ def run_ours(args, cfg) -> None:
     st = tp.tp_get_last_error()
     if st != tp.TP_OK:
         raise RuntimeError(f"device error during the timed region: {tp.tp_status_string(st)}")
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, "cuda")
 
     # end-to-end through the public API with host buffers: every step copies
     # its own input (X and, for a backward step, dY) from pinned host memory
@@ -552,10 +566,7 @@ def run_ours(args, cfg) -> None:
     if bwd:
         model.dY = dY_keep
     e2e_ms = e0.elapsed_time(e1) / args.steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
 
     # per-kernel figures from the trace of the timed region
     per = {}
@@ -596,8 +607,8 @@ def run_ours(args, cfg) -> None:
             step_breakdown.append([recs[pos][0], round(sum(times) / len(times), 5)])
     reduce_fig = kernels.get("reduce_partials") or kernels.get("reduce_partials_layernorm_backward")
 
-    value = w["total_flops"] * world / (ms * 1e-3) / 1e12
-    e2e_value = w["total_flops"] * world / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_tflops(w["total_flops"], world, ms)
+    e2e_value = whole_job_tflops(w["total_flops"], world, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
