@@ -565,6 +565,15 @@ size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn,
  * call, TP_ERR_CUDA if the stream reports a CUDA error, else TP_OK. */
 tp_status tp_get_last_error(void* stream);
 
+/* tp_selftest_wait_timeout - a self-test of the failure path, with no
+ * counterpart on the pages: launches, on `stream`, one thread that waits for
+ * at most limit_us microseconds (1 .. 1000000) on an mbarrier that nothing
+ * arrives on, then gives up the way every bounded wait in the library does
+ * (a bit in the device's error word). The next tp_get_last_error returns
+ * TP_ERR_TIMEOUT and clears the word; the context stays usable. Returns
+ * TP_ERR_SHAPE for a limit out of range, TP_ERR_CUDA if the launch fails. */
+tp_status tp_selftest_wait_timeout(int64_t limit_us, void* stream);
+
 /* Static string for a status code. */
 const char* tp_status_string(int status);
 

@@ -193,6 +193,17 @@ tp_status tp_get_last_error(void* stream) {
   return TP_OK;
 }
 
+tp_status tp_selftest_wait_timeout(int64_t limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return TP_ERR_SHAPE;
+  DevInfo d;
+  tp_status st = device_info(&d);
+  if (st != TP_OK) return st;
+  return tpk::launch_selftest_wait(d.err, static_cast<uint64_t>(limit_us) * 1000ull,
+                                   as_stream(stream)) == 0
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
 tp_status tp_shard_index_map(int kind, int64_t h_in, int64_t h_out, int n_shards,
                              int64_t head_dim, int32_t* host_owner, int64_t* host_local) {
   if (host_owner == nullptr || host_local == nullptr) return TP_ERR_NULL;

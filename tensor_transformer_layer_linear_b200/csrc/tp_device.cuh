@@ -17,6 +17,7 @@ enum : unsigned {
   ERR_WAIT_EPILOGUE = 1u << 2,
   ERR_WAIT_DRAIN = 1u << 3,
   ERR_WAIT_ATTN = 1u << 4,
+  ERR_WAIT_SELFTEST = 1u << 5,
 };
 
 // Every wait on a barrier gives up after this many nanoseconds of
@@ -71,9 +72,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Returns false if
-// the wait ran past kWaitLimitNs or *abort became non-zero (another role of
-// the CTA gave up), so that the caller can leave its loop.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+// the wait ran past limit_ns of %globaltimer or *abort became non-zero
+// (another role of the CTA gave up), so that the caller can leave its loop.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, volatile int* abort,
+                                              uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
@@ -81,8 +83,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -126,4 +126,8 @@ int launch_rows_sum_ln_bwd(const float* P, int n_shards, int64_t rows, int64_t h
                            cudaStream_t s, int num_sms, int sp_n = 0, int sp_batch = 0,
                            int sp_seq = 0);
 
+// One thread waits, for at most limit_ns, on an mbarrier nothing arrives on,
+// then ORs ERR_WAIT_SELFTEST into *err (the bounded-wait failure path).
+int launch_selftest_wait(unsigned* err, uint64_t limit_ns, cudaStream_t s);
+
 }  // namespace tpk

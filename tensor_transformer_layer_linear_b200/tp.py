@@ -100,6 +100,7 @@ _SIGS = {
                                     ctypes.POINTER(tp_layer_grads), _vp]),
     "tp_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "tp_get_last_error": (_i32, [_vp]),
+    "tp_selftest_wait_timeout": (_i32, [_i64, _vp]),
     "tp_status_string": (ctypes.c_char_p, [_i32]),
     "tp_trace_begin": (_i32, [_i32]),
     "tp_trace_end": (_i32, []),
@@ -388,6 +389,10 @@ def tp_layer_backward_sp(X_shards, batch, seq, h, n_heads, ffn, n_shards,
 
 def tp_get_last_error(stream=None) -> int:
     return int(lib.tp_get_last_error(_s(stream)))
+
+
+def tp_selftest_wait_timeout(limit_us, stream=None):
+    _check(lib.tp_selftest_wait_timeout(limit_us, _s(stream)), "tp_selftest_wait_timeout")
 
 
 def tp_trace_begin(max_records: int) -> None:
