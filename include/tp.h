@@ -521,8 +521,13 @@ tp_status tp_layer_forward_sp(const uint16_t* X_shards, int64_t batch,
                               void* stream);
 
 /* Size in bytes of the library-owned scratch array used by
- * tp_mlp_forward_noalloc (32 MiB, reserved on every GPU that loads the
- * library, until the process exits). */
+ * tp_mlp_forward_noalloc (32 MiB per GPU). The array belongs to the CUDA
+ * module of the file that defines it; the CUDA runtime reserves it on a GPU
+ * when it loads that module there. With lazy module loading (the CUDA 12
+ * default, CUDA_MODULE_LOADING=LAZY) that is the first
+ * tp_mlp_forward_noalloc call on that GPU; with eager loading it is the
+ * first CUDA call of the process that creates the GPU's context. It stays
+ * reserved until the process exits. */
 #define TP_NOALLOC_WS_BYTES (32u * 1024u * 1024u)
 
 /* tp_mlp_forward_noalloc - tp_mlp_forward for callers that cannot allocate
@@ -539,8 +544,16 @@ tp_status tp_layer_forward_sp(const uint16_t* X_shards, int64_t batch,
  *   (unordered streams or host threads) race on it: the caller must order
  *   them.
  * - The first call on a device looks up and caches the array's device
- *   address; make it before any stream capture begins.
- * - Calls no cudaMalloc, cudaFree or other allocating routine. */
+ *   address (cudaGetSymbolAddress, with that device current). Under lazy
+ *   module loading that lookup is also what loads the module and reserves
+ *   the 32 MiB, so a caller whose memory pool later takes all free device
+ *   memory must make its first call BEFORE the pool reserves it, and before
+ *   any stream capture begins. If the GPU has no room left for the array at
+ *   that point the call returns TP_ERR_WORKSPACE (nothing is launched).
+ * - The cached address is that of the device's primary context: after
+ *   cudaDeviceReset on a device, call nothing of this library on it again in
+ *   the same process.
+ * - Calls no cudaMalloc, cudaFree or other allocating routine itself. */
 tp_status tp_mlp_forward_noalloc(const uint16_t* X, int64_t B, int64_t h,
                                  int64_t ffn, int n_shards,
                                  const uint16_t* A_shards,

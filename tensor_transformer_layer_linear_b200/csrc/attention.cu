@@ -464,7 +464,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 attn_map_encoder() {
 
 int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, int64_t kv_local,
                      int n_shards, int causal, void* O, cudaStream_t s, unsigned* err,
-                     float* lse) {
+                     int num_sms, float* lse) {
   const int hps = static_cast<int>(n_q / n_shards);
   const int64_t q_w = hps * FA_D, kv_w = kv_local * FA_D;
   const int64_t ld = q_w + 2 * kv_w;  // QKV row width per shard
@@ -499,14 +499,7 @@ int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, i
   cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM);
   // persistent: one CTA per SM (shared memory and TMEM admit one), each
   // walking its share of the query tiles
-  static int num_sms = 0;
-  if (num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        num_sms <= 0)
-      return 2;
-  }
+  if (num_sms <= 0) return 2;
   const int64_t tiles = static_cast<int64_t>(p.nq) * p.n_units;
   const dim3 grid(static_cast<unsigned>(tiles < num_sms ? tiles : num_sms));
   attention_tc_kernel<<<grid, FA_THREADS, FA_SMEM, s>>>(tm, static_cast<uint16_t*>(O), p);

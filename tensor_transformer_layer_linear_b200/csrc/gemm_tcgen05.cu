@@ -30,6 +30,7 @@
 // TMEM and returns through the same exit path.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "tp_device.cuh"
@@ -41,6 +42,7 @@ constexpr int BM = 128;            // accumulator rows per CTA (TMEM lanes)
 constexpr int BK = 64;             // 64 bf16 = 128 bytes = one swizzle row
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, each half the columns
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kMaxGemmDevices = 64;  // device ordinals with a cached residency count
 
 template <int BN, int CTAS>
 struct GemmCfg {
@@ -612,7 +614,14 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
   cfg.numAttrs = 1;
   // Persistent grid: as many CTAs (pairs) as can be resident at once; pairs
   // need two free SMs of one GPC, which the occupancy query accounts for.
-  static int resident_units = 0;
+  // The count is cached per device ordinal (atomically: concurrent first
+  // calls compute the same value).
+  static std::atomic<int> resident_cache[kMaxGemmDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 2;
+  int resident_units = (dev >= 0 && dev < kMaxGemmDevices)
+                           ? resident_cache[dev].load(std::memory_order_relaxed)
+                           : 0;
   if (resident_units == 0) {
     int n = num_sms / CTAS;
     if (CTAS > 1) {
@@ -623,7 +632,9 @@ static int launch_gemm_t(const GemmProblem& pr, cudaStream_t s, unsigned* err, i
         n = clusters;
       cudaGetLastError();
     }
-    resident_units = n;
+    resident_units = n > 0 ? n : 1;
+    if (dev >= 0 && dev < kMaxGemmDevices)
+      resident_cache[dev].store(resident_units, std::memory_order_relaxed);
   }
   const int units = p.num_tiles < resident_units ? p.num_tiles : resident_units;
   cfg.gridDim = dim3(static_cast<unsigned>(units * CTAS));

@@ -419,7 +419,7 @@ tp_status tp_attention(const uint16_t* QKV_shards, int64_t batch, int64_t seq, i
   TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
   const int rc = tpk::launch_attention(QKV_shards, batch, seq, n_heads, n_heads / n_shards,
                                        n_shards, causal ? 1 : 0, O_shards, as_stream(stream),
-                                       d.err);
+                                       d.err, d.num_sms);
   return rc == 0 ? TP_OK : (rc == 3 ? TP_ERR_UNSUPPORTED : TP_ERR_CUDA);
 }
 
@@ -444,6 +444,18 @@ static size_t ln_bwd_bytes(size_t H) { return round256(2 * static_cast<size_t>(k
 
 size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int n_shards) {
   if (tokens <= 0 || h <= 0 || n_shards <= 0) return 0;
+  // Every product below is at most a few terms of N*M*H*4, M*3H*2,
+  // M*F*2, 256*(F+4H)*4 or (H/128)*(M+128)*4; when each factor is below
+  // 2^31 and those largest products fit in 2^60 (checked here), no sum of
+  // them can wrap a 64-bit size_t.
+  if (tokens > kIntMax || h > kIntMax || ffn > kIntMax || ffn < 0) return 0;
+  {
+    const unsigned __int128 M = static_cast<uint64_t>(tokens), H = static_cast<uint64_t>(h);
+    const unsigned __int128 F = static_cast<uint64_t>(ffn), N = static_cast<uint64_t>(n_shards);
+    const unsigned __int128 lim = static_cast<unsigned __int128>(1) << 60;
+    if (N * M * H * 4 >= lim || M * (F + 3 * H) * 2 >= lim || (M + 128) * H * 4 >= lim)
+      return 0;
+  }
   const size_t M = static_cast<size_t>(tokens), H = static_cast<size_t>(h);
   const size_t N = static_cast<size_t>(n_shards);
   const size_t partials = round256(N * M * H * 4);
@@ -754,7 +766,7 @@ tp_status tp_attention_gqa(const uint16_t* QKV_shards, int64_t batch, int64_t se
   TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
   const int rc = tpk::launch_attention(QKV_shards, batch, seq, n_q, gqa_kv_local(n_kv, n_shards),
                                        n_shards, causal ? 1 : 0, O_shards, as_stream(stream),
-                                       d.err);
+                                       d.err, d.num_sms);
   return rc == 0 ? TP_OK : (rc == 3 ? TP_ERR_UNSUPPORTED : TP_ERR_CUDA);
 }
 
@@ -912,7 +924,7 @@ tp_status tp_attention_lse(const uint16_t* QKV_shards, int64_t batch, int64_t se
   TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
   const int rc = tpk::launch_attention(QKV_shards, batch, seq, n_heads, n_heads / n_shards,
                                        n_shards, causal ? 1 : 0, O_shards, as_stream(stream),
-                                       d.err, lse);
+                                       d.err, d.num_sms, lse);
   return rc == 0 ? TP_OK : (rc == 3 ? TP_ERR_UNSUPPORTED : TP_ERR_CUDA);
 }
 
@@ -1250,7 +1262,7 @@ tp_status tp_attention_gqa_lse(const uint16_t* QKV_shards, int64_t batch, int64_
   TraceScope ts(tpk::KID_ATTENTION, as_stream(stream));
   const int rc = tpk::launch_attention(QKV_shards, batch, seq, n_q, gqa_kv_local(n_kv, n_shards),
                                        n_shards, causal ? 1 : 0, O_shards, as_stream(stream),
-                                       d.err, lse);
+                                       d.err, d.num_sms, lse);
   return rc == 0 ? TP_OK : (rc == 3 ? TP_ERR_UNSUPPORTED : TP_ERR_CUDA);
 }
 

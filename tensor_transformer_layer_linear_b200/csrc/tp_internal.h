@@ -87,9 +87,10 @@ int launch_rows_sum_ln(const float* P, int n_shards, int64_t rows, int64_t h, co
 // register split needs (it is then not launched). With lse != nullptr the
 // base-2 log-sum-exp of every query's scaled scores is written to
 // lse[(shard * (n_q/N) + k) * (M + 128) + token], M = batch * seq.
+// num_sms: the current device's SM count (the persistent grid's size).
 int launch_attention(const void* QKV, int64_t batch, int64_t seq, int64_t n_q, int64_t kv_local,
                      int n_shards, int causal, void* O, cudaStream_t s, unsigned* err,
-                     float* lse = nullptr);
+                     int num_sms, float* lse = nullptr);
 
 // Attention backward of every shard's heads (head_dim 128; n_q/N query heads
 // and kv_local key/value heads per shard, laid out like the forward's QKV):

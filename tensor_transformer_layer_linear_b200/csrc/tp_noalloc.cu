@@ -11,8 +11,12 @@
 // partials) live in g_tp_noalloc_ws below.
 //
 // Properties a caller must know:
-//   * The array is TP_NOALLOC_WS_BYTES (include/tp.h) per GPU, reserved on
-//     every GPU that loads the library, for the life of the process.
+//   * The array is TP_NOALLOC_WS_BYTES (include/tp.h) per GPU. It belongs
+//     to this file's CUDA module, and the runtime reserves it when it loads
+//     the module on a GPU: under lazy module loading (the CUDA 12 default)
+//     that is the first call here on that GPU, whose cudaGetSymbolAddress
+//     triggers the load; under eager loading, context creation. It stays
+//     reserved until the process exits.
 //   * A problem whose scratch exceeds it is rejected with TP_ERR_WORKSPACE
 //     before anything is launched.
 //   * Every call on a device shares the same array and it keeps the last
@@ -22,7 +26,10 @@
 //     between them) race on the array and corrupt each other's results.
 //   * The first call on a device looks up the array's device address
 //     (cudaGetSymbolAddress, with that device current) and caches it; make
-//     that first call before any stream capture begins.
+//     that first call before any stream capture begins, and before a memory
+//     pool of the caller's takes the free device memory (the lazy module
+//     load needs room for the array; without it the call returns
+//     TP_ERR_WORKSPACE). After cudaDeviceReset the cached address is stale.
 //   * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
 #include <cuda_runtime.h>
 
@@ -58,8 +65,12 @@ extern "C" tp_status tp_mlp_forward_noalloc(const uint16_t* X, int64_t B, int64_
     std::lock_guard<std::mutex> lk(g_mu);
     if (g_ws_ptr[dev] == nullptr) {
       void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_tp_noalloc_ws) != cudaSuccess || p == nullptr)
-        return TP_ERR_CUDA;
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_tp_noalloc_ws);
+      if (e == cudaErrorMemoryAllocation) {
+        cudaGetLastError();  // not sticky: clear it and report the missing room
+        return TP_ERR_WORKSPACE;
+      }
+      if (e != cudaSuccess || p == nullptr) return TP_ERR_CUDA;
       g_ws_ptr[dev] = p;
     }
     ws = g_ws_ptr[dev];

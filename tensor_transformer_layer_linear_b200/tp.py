@@ -246,10 +246,17 @@ def tp_attn_forward(X, batch, seq, h, n_heads, causal, n_shards, Wqkv_shards, bq
 
 
 def make_layer_weights(**tensors) -> tp_layer_weights:
-    """Build the tp_layer_weights struct from tensors named like its fields."""
+    """Build the tp_layer_weights struct from tensors named like its fields.
+
+    The struct holds raw device addresses, so it also keeps a reference to
+    every tensor it was built from: the memory stays allocated for as long as
+    the struct lives, even when the caller passed temporaries (otherwise
+    torch's caching allocator could hand those bytes to the next tensor, e.g.
+    the workspace, and the layer would read its own scratch as weights)."""
     w = tp_layer_weights()
     for name, _ in tp_layer_weights._fields_:
         setattr(w, name, _p(tensors.get(name)))
+    w._tensors = dict(tensors)
     return w
 
 
@@ -339,10 +346,12 @@ def tp_reduce_partials_layernorm_backward(partials, n_shards, B, h, x, gamma, re
 
 
 def make_layer_grads(**tensors) -> tp_layer_grads:
-    """Build the tp_layer_grads struct from fp32 tensors named like its fields."""
+    """Build the tp_layer_grads struct from fp32 tensors named like its fields
+    (the struct keeps a reference to each, as make_layer_weights does)."""
     g = tp_layer_grads()
     for name, _ in tp_layer_grads._fields_:
         setattr(g, name, _p(tensors.get(name)))
+    g._tensors = dict(tensors)
     return g
 
 

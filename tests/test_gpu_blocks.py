@@ -172,12 +172,47 @@ def test_workload_attn_4x2048_n8(tp):
     assert_parity(Y[rows], attn_ref(inp, cfg, rows))
 
 
-def test_workload_layer_2x2048_n8(tp):
+@pytest.fixture(scope="module")
+def layer_workload():
     cfg = synth.config("layer_2x2048_h4096_32x128_f16384_n8")
     inp = synth.make_inputs(cfg)
     rows = synth.sample_rows(cfg["batch"], cfg["seq"])
-    Y = from_dev_bf16(run_layer(tp, inp, cfg, cfg["n_shards"]))
-    assert_parity(Y[rows], layer_ref(inp, cfg, rows))
+    return cfg, inp, rows, layer_ref(inp, cfg, rows), {}
+
+
+@pytest.mark.parametrize("n", [8, 16])
+def test_workload_layer_2x2048(tp, layer_workload, n):
+    """The full layer workload at its own shard count (8) and at 16 (two of
+    the 32 heads per shard), on sampled rows; the two outputs agree on every
+    element."""
+    cfg, inp, rows, ref, outs = layer_workload
+    Y = from_dev_bf16(run_layer(tp, inp, cfg, n))
+    torch.cuda.empty_cache()
+    assert_parity(Y[rows], ref, f"N={n}")
+    outs[n] = Y
+    if n != 8 and 8 in outs:
+        assert_parity(Y, outs[8], f"N={n} vs N=8")
+
+
+@pytest.fixture(scope="module")
+def layer_sweep():
+    cfg = dict(kind="layer", batch=2, seq=192, h=2048, n_heads=16, ffn=8192, x_std=1.0,
+               w_std=0.02, b_std=0.01, ln_eps=1e-5)
+    inp = synth.make_inputs(cfg, seed=4)
+    return cfg, inp, layer_ref(inp, cfg), {}
+
+
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16])
+def test_layer_shard_sweep_all_elements(tp, layer_sweep, n):
+    """A 16-head layer (h 2048, F 8192, 2 x 192 tokens: a ragged last query
+    tile) at every shard count the heads allow up to 16, every element
+    against the unsharded oracle and against the N = 1 output."""
+    cfg, inp, ref, outs = layer_sweep
+    Y = from_dev_bf16(run_layer(tp, inp, cfg, n))
+    assert_parity(Y, ref, f"N={n}")
+    outs[n] = Y
+    if n != 1 and 1 in outs:
+        assert_parity(Y, outs[1], f"N={n} vs N=1")
 
 
 @pytest.fixture(scope="module")
