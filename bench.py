@@ -56,6 +56,10 @@ NCU_TRAFFIC = {
     (DEFAULT_WORKLOAD, "gemm_row_parallel"): 652.8e6,
     # persistent attention: 134.5 MB read + 13.6 MB written
     (DEFAULT_WORKLOAD, "attention"): 148.1e6,
+    # the reductions and LN1 (profiles/reduce_partials_ncu.md): read + write per launch
+    (DEFAULT_WORKLOAD, "reduce_partials"): 574.3e6,
+    (DEFAULT_WORKLOAD, "reduce_partials_layernorm"): 592.3e6,
+    (DEFAULT_WORKLOAD, "layernorm"): 33.9e6,
 }
 
 
@@ -74,66 +78,76 @@ def peaks() -> dict:
 # --------------------------------------------------------------------------
 
 def work(cfg: dict) -> dict:
-    """Per-step algorithmic FLOPs per kernel kind and bytes per reduction kind."""
+    """Per-step algorithmic work by kernel name (as the launch trace names
+    the kernels): FLOPs of the contractions, bytes of the HBM-bound kernels
+    (per-step totals), and the bytes of one launch of each HBM-bound kernel."""
     M = cfg["batch"] * cfg["seq"]
     h = cfg["h"]
     n = cfg["n_shards"]
     kind = cfg["kind"]
     fl = {"gemm_column_parallel": 0.0, "gemm_row_parallel": 0.0, "attention": 0.0}
-    by = {}
-    if kind in ("attn", "layer"):
-        fl["gemm_column_parallel"] += 2.0 * M * h * 3 * h
-        d = h // cfg["n_heads"]
-        fl["attention"] += 4.0 * cfg["seq"] ** 2 * d * cfg["n_heads"] * cfg["batch"] / (
-            2 if cfg.get("causal", True) else 1)
-        fl["gemm_row_parallel"] += 2.0 * M * h * h
-    if kind in ("mlp", "layer"):
-        F = cfg["ffn"]
-        fl["gemm_column_parallel"] += 2.0 * M * h * F
-        fl["gemm_row_parallel"] += 2.0 * M * F * h
-    if kind == "attn_gqa":
-        d = h // cfg["n_heads"]
-        fl["gemm_column_parallel"] += 2.0 * M * h * (cfg["n_heads"] + 2 * cfg["n_kv_heads"]) * d
-        fl["attention"] += 4.0 * cfg["seq"] ** 2 * d * cfg["n_heads"] * cfg["batch"] / (
-            2 if cfg.get("causal", True) else 1)
-        fl["gemm_row_parallel"] += 2.0 * M * h * h
+    by, launch = {}, {}
+    partial_read = n * M * h * 4
+    act = M * h * 2
+
+    def hbm(name, nbytes):
+        by[name] = by.get(name, 0) + nbytes
+        launch[name] = nbytes
+
+    def row_block(K, res, ln_after=False):
+        """A block's output projection (K = its per-shard inner size) and its
+        one reduction of the N partials (+ bias, + residual when res, + LN
+        when ln_after)."""
+        fl["gemm_row_parallel"] += 2.0 * M * (K * n) * h
+        if ln_after:
+            hbm("reduce_partials_layernorm", partial_read + act + 3 * h * 2 + 2 * act)
+        else:
+            hbm("reduce_partials", partial_read + (act if res else 0) + h * 2 + act)
+
     if cfg.get("backward"):
         # algorithmic backward work (recomputed forward products are extra):
         # MLP dH, dX, dA, dB; attention block dO, dX, dW_QKV, dW_O and the
         # head gradients dV, dP, dK, dQ (twice the forward attention)
         F = cfg.get("ffn", 0)
         gb, ab = 0.0, 0.0
+        att = 0.0
+        if kind in ("attn", "layer", "attn_gqa"):
+            d = h // cfg["n_heads"]
+            att = 4.0 * cfg["seq"] ** 2 * d * cfg["n_heads"] * cfg["batch"] / (
+                2 if cfg.get("causal", True) else 1)
         if kind in ("mlp", "layer"):
             gb += 8.0 * M * h * F
         if kind in ("attn", "layer"):
             gb += 16.0 * M * h * h
-            ab = 2.0 * fl["attention"]
+            ab = 2.0 * att
         if kind == "attn_gqa":
             qkv = (cfg["n_heads"] + 2 * cfg["n_kv_heads"]) * (h // cfg["n_heads"])
             gb += 4.0 * M * h * h + 4.0 * M * qkv * h   # dO, dW_O; dX, dW_QKV
-            ab = 2.0 * fl["attention"]
-        fl = {"gemm_backward": gb, "attention_backward": ab, "gemm_column_parallel": 0.0,
-              "gemm_row_parallel": 0.0, "attention": 0.0}
+            ab = 2.0 * att
+        fl = {"gemm_backward": gb, "attention_backward": ab}
         if kind == "layer":
-            by["reduce_partials_layernorm_backward"] = n * M * h * 4 + 3 * M * h * 2 + h * 2
+            hbm("reduce_partials_layernorm_backward", n * M * h * 4 + 3 * M * h * 2 + h * 2)
         else:
-            res = M * h * 2 if cfg.get("residual") else 0
-            by["reduce_partials"] = n * M * h * 4 + res + M * h * 2
-        return dict(flops=fl, bytes=by, total_flops=sum(fl.values()))
-    if kind == "swiglu":
-        F = cfg["ffn"]
-        fl["gemm_column_parallel"] += 2.0 * M * h * 2 * F   # gate and up
-        fl["gemm_row_parallel"] += 2.0 * M * F * h
-    partial_read = n * M * h * 4
-    act = M * h * 2
+            hbm("reduce_partials", partial_read + (act if cfg.get("residual") else 0) + act)
+        return dict(flops=fl, bytes=by, launch_bytes=launch, total_flops=sum(fl.values()))
     if kind == "layer":
-        by["reduce_partials"] = partial_read + act + h * 2 + act          # + residual, bias, write
-        by["reduce_partials_layernorm"] = partial_read + act + 3 * h * 2 + 2 * act
-        by["layernorm"] = act + 2 * h * 2 + act
-    else:
-        res = act if cfg.get("residual") else 0
-        by["reduce_partials"] = partial_read + res + h * 2 + act
-    return dict(flops=fl, bytes=by, total_flops=sum(fl.values()))
+        hbm("layernorm", act + 2 * h * 2 + act)                      # LN1
+    if kind in ("attn", "layer"):
+        fl["gemm_column_parallel"] += 2.0 * M * h * 3 * h
+    if kind == "attn_gqa":
+        d = h // cfg["n_heads"]
+        fl["gemm_column_parallel"] += 2.0 * M * h * (cfg["n_heads"] + 2 * cfg["n_kv_heads"]) * d
+    if kind in ("attn", "layer", "attn_gqa"):
+        d = h // cfg["n_heads"]
+        fl["attention"] += 4.0 * cfg["seq"] ** 2 * d * cfg["n_heads"] * cfg["batch"] / (
+            2 if cfg.get("causal", True) else 1)
+        row_block(h // n, res=(kind == "layer" or cfg.get("residual")), ln_after=(kind == "layer"))
+    if kind in ("mlp", "layer", "swiglu"):
+        F = cfg["ffn"]
+        fl["gemm_column_parallel"] += 2.0 * M * h * F * (2 if kind == "swiglu" else 1)
+        row_block(F // n, res=(kind == "layer" or cfg.get("residual")))
+    fl = {k: v for k, v in fl.items() if v > 0}
+    return dict(flops=fl, bytes=by, launch_bytes=launch, total_flops=sum(fl.values()))
 
 
 # --------------------------------------------------------------------------
@@ -160,11 +174,11 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
-    def stop(self, t0: float = None, t1: float = None) -> dict:
-        """Median SM clock and the throttle reasons seen in samples taken
-        between host wall-clock times t0 and t1 (all samples if none are)."""
+    def stop(self) -> None:
+        """End sampling and parse what nvidia-smi printed."""
+        self.samples = []
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return
         self.proc.terminate()
         try:
             text, _ = self.proc.communicate(timeout=5)
@@ -184,7 +198,15 @@ class ClockSampler:
                                 [nm for nm, v in zip(names, f[6:10]) if v.lower() == "active"]))
             except ValueError:
                 continue
-        inside = [x for x in samples if t0 is not None and t0 <= x[0] <= t1]
+        self.samples = samples
+
+    def window(self, t0: float, t1: float) -> dict:
+        """Median SM clock and the throttle reasons seen in samples taken
+        between host wall-clock times t0 and t1 (all samples if none are)."""
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        samples = self.samples
+        inside = [x for x in samples if t0 <= x[0] <= t1]
         use = inside or samples
         sm = [x[1] for x in use]
         reasons = sorted({r for x in use for r in x[4]})
@@ -192,7 +214,74 @@ class ClockSampler:
                 "sm_max_mhz": max(x[2] for x in use) if use else None,
                 "power_w_max": max(x[3] for x in use) if use else None,
                 "reasons": reasons, "samples": len(use),
-                "window": "timed region" if inside else "whole run"}
+                "window": "timed region" if inside else "whole run", "source": "nvidia-smi"}
+
+
+class NvmlSampler:
+    """SM clock, power and clock-event reasons read through NVML (read-only
+    queries) by a host thread every few milliseconds, so that even a timed
+    region of a few tens of milliseconds holds several samples."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, device_index: int, period_s: float = 0.004):
+        import threading
+        import pynvml
+        import torch
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        gid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        self.h = pynvml.nvmlDeviceGetHandleByUUID(gid)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.bits = [(nm, getattr(pynvml, attr)) for nm, attr in self.REASONS
+                     if hasattr(pynvml, attr)]
+        self.samples = []
+        self.period = period_s
+        self.done = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv, h = self.nv, self.h
+        while not self.done.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                mw = float(nv.nvmlDeviceGetPowerUsage(h))
+                r = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                self.samples.append((time.time(), mhz, mw / 1000.0,
+                                     [nm for nm, b in self.bits if r & b]))
+            except Exception:
+                pass
+            self.done.wait(self.period)
+
+    def window(self, t0: float, t1: float) -> dict:
+        """Median SM clock and every reason seen between host times t0 and t1."""
+        use = [x for x in self.samples if t0 <= x[0] <= t1]
+        where = "timed region"
+        if not use:
+            use, where = self.samples, "whole run"
+        sm = [x[1] for x in use]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "power_w_max": max((x[2] for x in use), default=None),
+                "reasons": sorted({r for x in use for r in x[3]}), "samples": len(use),
+                "window": where, "source": "nvml"}
+
+    def stop(self) -> None:
+        self.done.set()
+        self.thread.join(timeout=2)
+
+
+def clock_sampler(device_index: int):
+    """NVML sampler when NVML answers, else the nvidia-smi one."""
+    try:
+        return NvmlSampler(device_index)
+    except Exception:
+        return ClockSampler(device_index)
 
 
 # --------------------------------------------------------------------------
@@ -457,6 +546,60 @@ def whole_job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
     return flops_per_rank * world / (ms * 1e-3) / 1e12
 
 
+def l2_cold_kernels(tp, torch, model, cfg, w, pk, reps: int = 20) -> dict:
+    """The HBM-bound kernels of the step timed one launch at a time with the
+    L2 emptied first (a read of a buffer twice the L2 size, which leaves the
+    L2 holding clean lines of that buffer only), so that every input byte
+    comes from HBM: median device time over `reps` launches (CUDA events on
+    the launching stream), algorithmic bytes / time against the measured
+    copy bandwidth. Inputs are the step's own shapes; the partials hold
+    arbitrary values."""
+    n, h, M = cfg["n_shards"], cfg["h"], model.M
+    stream = torch.cuda.current_stream()
+    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    P = torch.randn((n, M, h), dtype=torch.float32, device="cuda")
+    Y = torch.empty((M, h), dtype=torch.int16, device="cuda")
+    Y2 = torch.empty((M, h), dtype=torch.int16, device="cuda")
+    res = model.X if (cfg["kind"] == "layer" or cfg.get("residual")) else None
+    bias = model.b2 if hasattr(model, "b2") else getattr(model, "bo", None)
+    runs = {"reduce_partials": lambda: tp.tp_reduce_partials(P, n, M, h, bias, res, Y)}
+    if cfg["kind"] == "layer":
+        g = model.w._tensors
+        eps = cfg.get("ln_eps", 1e-5)
+        runs["reduce_partials_layernorm"] = lambda: tp.tp_reduce_partials_layernorm(
+            P, n, M, h, model.bo, model.X, g["ln2_gamma"], g["ln2_beta"], eps, Y, Y2)
+        runs["layernorm"] = lambda: tp.tp_layernorm(model.X, M, h, g["ln1_gamma"],
+                                                    g["ln1_beta"], eps, Y)
+    out = {}
+    # one launch's bytes of each kernel (whether or not the step itself runs it)
+    act = M * h * 2
+    one = {"reduce_partials": n * M * h * 4 + (act if res is not None else 0) + h * 2 + act,
+           "reduce_partials_layernorm": n * M * h * 4 + act + 3 * h * 2 + 2 * act,
+           "layernorm": act + 2 * h * 2 + act}
+    for name, fn in runs.items():
+        fn()
+        times = []
+        for _ in range(reps):
+            flush.sum()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        t = statistics.median(times)
+        gbs = one[name] / (t * 1e-3) / 1e9
+        out[name] = {"ms": t, "achieved": gbs, "unit": "GB/s", "peak": pk["hbm"],
+                     "frac": gbs / pk["hbm"], "bytes": one[name], "reps": reps,
+                     "flush": "read of a 2 x L2 buffer before each launch"}
+    del flush, P
+    torch.cuda.empty_cache()
+    if tp.tp_get_last_error() != tp.TP_OK:
+        raise RuntimeError("device error in the L2-cold kernel timings")
+    return out
+
+
 def run_ours(args, cfg) -> None:
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -487,28 +630,50 @@ def run_ours(args, cfg) -> None:
     assert tp.tp_get_last_error() == tp.TP_OK
     barrier()
 
-    # device-timed region (inputs resident in HBM)
+    # device-timed region (inputs resident in HBM); an event after every step
+    # gives the per-step times whose median is reported beside the mean
     stream = torch.cuda.current_stream()
-    sampler = ClockSampler(local)
+    sampler = clock_sampler(local)
     time.sleep(0.3)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     tp.tp_trace_begin(64 * args.steps)
     barrier()
     t_wall0 = time.time()
-    ev0.record(stream)
-    for _ in range(args.steps):
+    step_ev[0].record(stream)
+    for i in range(args.steps):
         model.step()
-    ev1.record(stream)
+        step_ev[i + 1].record(stream)
     barrier()
     t_wall1 = time.time()
     recs, launches = tp.tp_trace_end()
-    clocks = sampler.stop(t_wall0, t_wall1)
-    ms = ev0.elapsed_time(ev1) / args.steps
+    ms = step_ev[0].elapsed_time(step_ev[-1]) / args.steps
+    median_ms = statistics.median(step_ev[i].elapsed_time(step_ev[i + 1])
+                                  for i in range(args.steps))
     st = tp.tp_get_last_error()
     if st != tp.TP_OK:
         raise RuntimeError(f"device error during the timed region: {tp.tp_status_string(st)}")
     ms = max_over_ranks(ms, dist, "cuda")
+    median_ms = max_over_ranks(median_ms, dist, "cuda")
+
+    # sustained window: the same step back to back for about --sustained-s
+    # seconds, long enough for the 1 kW power cap to settle the clocks
+    sustained = None
+    if args.sustained_s > 0:
+        n_sus = max(50, int(args.sustained_s * 1e3 / ms))
+        sa = torch.cuda.Event(enable_timing=True)
+        sb = torch.cuda.Event(enable_timing=True)
+        barrier()
+        t_s0 = time.time()
+        sa.record(stream)
+        for _ in range(n_sus):
+            model.step()
+        sb.record(stream)
+        barrier()
+        t_s1 = time.time()
+        ms_s = max_over_ranks(sa.elapsed_time(sb) / n_sus, dist, "cuda")
+        sustained = {"steps": n_sus, "ms_per_step": ms_s, "window": (t_s0, t_s1)}
+    if tp.tp_get_last_error() != tp.TP_OK:
+        raise RuntimeError("device error during the sustained window")
 
     # end-to-end through the public API with host buffers: every step copies
     # its own input (X and, for a backward step, dY) from pinned host memory
@@ -567,6 +732,18 @@ def run_ours(args, cfg) -> None:
         model.dY = dY_keep
     e2e_ms = e0.elapsed_time(e1) / args.steps
     e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
+
+    l2_cold = l2_cold_kernels(tp, torch, model, cfg, w, pk) if not bwd else None
+    sampler.stop()
+    clocks = sampler.window(t_wall0, t_wall1)
+    clocks["kcycles_per_step"] = (ms * clocks["sm_mhz"]) if clocks.get("sm_mhz") else None
+    if sustained is not None:
+        t_s0, t_s1 = sustained.pop("window")
+        c = sampler.window(t_s0, t_s1)
+        sustained.update(
+            value=whole_job_tflops(w["total_flops"], world, sustained["ms_per_step"]),
+            unit="TFLOP/s", clocks=c,
+            kcycles_per_step=(sustained["ms_per_step"] * c["sm_mhz"]) if c.get("sm_mhz") else None)
 
     # per-kernel figures from the trace of the timed region
     per = {}
@@ -641,6 +818,9 @@ def run_ours(args, cfg) -> None:
                 "d2h_bytes_per_step": M * h * 2, "ms_per_step": e2e_ms,
                 "copies": "own streams, double-buffered, overlapping the neighbouring steps"},
         "clocks": clocks,
+        "median_ms_per_step": median_ms,
+        "sustained": sustained,
+        "partial_reduce_l2_cold": l2_cold,
         "gpu_launches": launches,
         "gflop_per_step": w["total_flops"] / 1e9,
         "step_breakdown_ms": step_breakdown,
@@ -683,7 +863,7 @@ def run_sweep(args, cfg) -> None:
         for name, kms in recs:
             kern[name] = kern.get(name, 0.0) + kms / args.steps
         w = work(c)
-        red_bytes = w["bytes"]["reduce_partials"]
+        red_bytes = w["bytes"].get("reduce_partials", 0)
         res[n] = {"ms_per_step": ms, "tflops": w["total_flops"] / ms / 1e9,
                   "frac_of_bf16_peak": w["total_flops"] / ms / 1e9 / pk["bf16"],
                   "kernel_ms": {k: round(v, 4) for k, v in kern.items()},
@@ -705,7 +885,9 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--sustained-s", type=float, default=3.0,
+                    help="seconds of back-to-back steps timed after the main region (0: skip)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.CONFIGS))
     ap.add_argument("--shards", type=int, default=0, help="override the shard count N")

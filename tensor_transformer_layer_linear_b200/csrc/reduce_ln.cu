@@ -226,6 +226,20 @@ __global__ void __launch_bounds__(256) layernorm_rows_warp_kernel(
   extern __shared__ uint4 gb_s[];  // [2][h / 8]: gamma, then beta
   const int lane = threadIdx.x & 31;
   const int nch = h >> 3;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const bool active = row < rows;
+  const int64_t row_off = row * h;
+  const int64_t sh_off = active ? seq_shard_row(sp, row) * h : 0;  // same row, sharded layout
+  const int64_t ln_off = ln_natural ? row_off : sh_off;
+  // the row's loads go out first; gamma and beta are staged while they fly
+  uint4 x[CHW];
+#pragma unroll
+  for (int c = 0; c < CHW; ++c) {
+    const int ch = lane + 32 * c;
+    x[c] = make_uint4(0u, 0u, 0u, 0u);
+    if (active && res != nullptr && ch < nch)
+      x[c] = __ldg(reinterpret_cast<const uint4*>(res + sh_off + (ch << 3)));
+  }
   if (Yln != nullptr) {
     for (int i = threadIdx.x; i < nch; i += blockDim.x) {
       gb_s[i] = __ldg(reinterpret_cast<const uint4*>(gamma) + i);
@@ -233,18 +247,7 @@ __global__ void __launch_bounds__(256) layernorm_rows_warp_kernel(
     }
   }
   __syncthreads();
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const int64_t row_off = row * h;
-  const int64_t sh_off = seq_shard_row(sp, row) * h;  // same row, sharded layout
-  const int64_t ln_off = ln_natural ? row_off : sh_off;
-  uint4 x[CHW];
-#pragma unroll
-  for (int c = 0; c < CHW; ++c) {
-    const int ch = lane + 32 * c;
-    x[c] = make_uint4(0u, 0u, 0u, 0u);
-    if (res != nullptr && ch < nch) x[c] = __ldg(reinterpret_cast<const uint4*>(res + sh_off + (ch << 3)));
-  }
+  if (!active) return;
   float s = 0.f;
 #pragma unroll
   for (int c = 0; c < CHW; ++c) {

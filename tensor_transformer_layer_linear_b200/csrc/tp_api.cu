@@ -493,6 +493,17 @@ size_t tp_workspace_bytes(int kind, int64_t tokens, int64_t h, int64_t ffn, int 
   return 0;
 }
 
+// A block's output projection and its one reduction: the row-parallel GEMM
+// into the N fp32 partials, then their sum with the bias and the residual.
+static tp_status row_block_output(const uint16_t* X_shards, int64_t M, int64_t h_in,
+                                  const uint16_t* W_shards, int64_t h_out, int n_shards,
+                                  const uint16_t* bias, const uint16_t* residual, float* part,
+                                  uint16_t* Y, void* stream) {
+  tp_status st = tp_row_linear(X_shards, M, h_in, W_shards, h_out, n_shards, part, stream);
+  if (st != TP_OK) return st;
+  return tp_reduce_partials(part, n_shards, M, h_out, bias, residual, Y, stream);
+}
+
 tp_status tp_mlp_forward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, int n_shards,
                          const uint16_t* A_shards, const uint16_t* b1_shards,
                          const uint16_t* B_shards, const uint16_t* b2, const uint16_t* residual,
@@ -510,9 +521,7 @@ tp_status tp_mlp_forward(const uint16_t* X, int64_t B, int64_t h, int64_t ffn, i
   tp_status st = tp_column_linear(X, B, h, A_shards, b1_shards, ffn, n_shards, TP_ACT_GELU_ERF,
                                   act, stream);
   if (st != TP_OK) return st;
-  st = tp_row_linear(act, B, ffn, B_shards, h, n_shards, part, stream);
-  if (st != TP_OK) return st;
-  return tp_reduce_partials(part, n_shards, B, h, b2, residual, Y, stream);
+  return row_block_output(act, B, ffn, B_shards, h, n_shards, b2, residual, part, Y, stream);
 }
 
 tp_status tp_mlp_forward_swiglu(const uint16_t* X, int64_t B, int64_t h, int64_t ffn,
@@ -533,9 +542,7 @@ tp_status tp_mlp_forward_swiglu(const uint16_t* X, int64_t B, int64_t h, int64_t
   tp_status st = tp_column_linear(X, B, h, GU_shards, nullptr, 2 * ffn, n_shards, TP_ACT_SWIGLU,
                                   act, stream);
   if (st != TP_OK) return st;
-  st = tp_row_linear(act, B, ffn, B_shards, h, n_shards, part, stream);
-  if (st != TP_OK) return st;
-  return tp_reduce_partials(part, n_shards, B, h, b2, residual, Y, stream);
+  return row_block_output(act, B, ffn, B_shards, h, n_shards, b2, residual, part, Y, stream);
 }
 
 tp_status tp_attn_forward(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
@@ -564,9 +571,7 @@ tp_status tp_attn_forward(const uint16_t* X, int64_t batch, int64_t seq, int64_t
   if (st != TP_OK) return st;
   st = tp_attention(qkv, batch, seq, h, n_heads, causal, n_shards, o, stream);
   if (st != TP_OK) return st;
-  st = tp_row_linear(o, M, h, Wo_shards, h, n_shards, part, stream);
-  if (st != TP_OK) return st;
-  return tp_reduce_partials(part, n_shards, M, h, bo, residual, Y, stream);
+  return row_block_output(o, M, h, Wo_shards, h, n_shards, bo, residual, part, Y, stream);
 }
 
 tp_status tp_layer_forward(const uint16_t* X, int64_t batch, int64_t seq, int64_t h,
@@ -612,9 +617,7 @@ tp_status tp_layer_forward(const uint16_t* X, int64_t batch, int64_t seq, int64_
   st = tp_column_linear(x2, M, h, w->A_shards, w->b1_shards, ffn, n_shards, TP_ACT_GELU_ERF, a,
                         stream);
   if (st != TP_OK) return st;
-  st = tp_row_linear(a, M, ffn, w->B_shards, h, n_shards, part, stream);
-  if (st != TP_OK) return st;
-  return tp_reduce_partials(part, n_shards, M, h, w->b2, h1, Y, stream);
+  return row_block_output(a, M, ffn, w->B_shards, h, n_shards, w->b2, h1, part, Y, stream);
 }
 
 
@@ -799,9 +802,7 @@ tp_status tp_attn_forward_gqa(const uint16_t* X, int64_t batch, int64_t seq, int
   if (st != TP_OK) return st;
   st = tp_attention_gqa(qkv, batch, seq, n_q, n_kv, 128, causal, n_shards, o, stream);
   if (st != TP_OK) return st;
-  st = tp_row_linear(o, M, h, Wo_shards, h, n_shards, part, stream);
-  if (st != TP_OK) return st;
-  return tp_reduce_partials(part, n_shards, M, h, bo, residual, Y, stream);
+  return row_block_output(o, M, h, Wo_shards, h, n_shards, bo, residual, part, Y, stream);
 }
 
 // One GEMM of a backward pass over all shards (see tpk::GemmProblem).

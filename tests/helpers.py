@@ -1,4 +1,10 @@
-"""Shared test helpers: bf16 bit arrays <-> torch tensors, the parity gate."""
+"""Shared test helpers: bf16 bit arrays <-> torch tensors, the parity gate.
+
+With TP_PARITY_LOG set to a file path, every parity check appends its
+observed errors to that file as one JSON line."""
+import json
+import os
+
 import numpy as np
 
 from tensor_transformer_layer_linear_b200 import synth
@@ -41,6 +47,13 @@ def assert_parity(gpu: np.ndarray, ref: np.ndarray, what: str = "",
     scale = np.max(np.abs(ref))
     fro = np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-300)
     stats = dict(max_abs=float(err.max()), max_ref=float(scale), fro_rel=float(fro))
+    log = os.environ.get("TP_PARITY_LOG")
+    if log:   # observed errors, one JSON line per check (for the tolerance notes)
+        with open(log, "a") as f:
+            f.write(json.dumps(dict(test=os.environ.get("PYTEST_CURRENT_TEST", ""), what=what,
+                                    max_rel_gate=max_rel, fro_gate=fro_rel,
+                                    max_rel=stats["max_abs"] / max(stats["max_ref"], 1e-300),
+                                    **stats)) + "\n")
     assert err.max() <= max_rel * scale, f"{what}: max error {stats}"
     assert fro <= fro_rel, f"{what}: Frobenius error {stats}"
     return stats

@@ -63,6 +63,11 @@ def test_layer_work_is_the_pages_flop_count():
     assert w["flops"]["gemm_column_parallel"] == qkv + up
     assert w["flops"]["gemm_row_parallel"] == wo + down
     assert w["flops"]["attention"] == attn
+    # the two reductions (the first fused with LN2) read the N fp32 partials
+    n = 8
+    assert w["bytes"]["reduce_partials"] == n * M * h * 4 + 2 * M * h * 2 + h * 2
+    assert w["bytes"]["reduce_partials_layernorm"] == n * M * h * 4 + 3 * M * h * 2 + 3 * h * 2
+    assert w["bytes"]["layernorm"] == 2 * M * h * 2 + 2 * h * 2            # LN1
     assert w["total_flops"] == qkv + up + wo + down + attn
     assert w["total_flops"] / 1e9 == pytest.approx(1717.99, abs=0.01)
 

@@ -90,3 +90,44 @@ def test_mlp_backward_workload(tp):
     got = _run_backward(tp, inp["X"], inp["A"], inp["b1"], inp["B"], dY, n)
     ref = O.mlp_backward(f64(inp["X"]), f64(inp["A"]), f64(inp["b1"]), f64(inp["B"]), f64(dY))
     _check(got, ref, n)
+
+
+def _bf16_ulp(v):
+    """Spacing of bf16 values at magnitude |v| (8 significand bits)."""
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+@pytest.mark.parametrize("n", [1, 2])
+def test_backward_gelu_epilogue_pointwise(tp, n):
+    """The backward recomputes H = GeLU(Z) and GeLU'(Z) in one GEMM epilogue
+    with the complementary error function of Abramowitz & Stegun eq. 7.1.26
+    (absolute error <= 1.5e-7 in erf, so <= 0.75e-7 in Phi). With A = I
+    (h = F), b1 = 0, dY = I (tokens = h) and B all ones, every product and sum
+    around that epilogue is exact: Z = X, dB_i^T[j][f] = H[j][f], and
+    dX[m][j] = bf16(1 * GeLU'(Z[m][j])) (no residual). So each of the 65536
+    grid values z is held to one bf16 rounding of GeLU(z) and of GeLU'(z),
+    beyond the approximation's bound plus fp32 evaluation slop
+    delta = 5e-7 (1 + |z|)."""
+    h = F = M = 256
+    grid = [0.0]
+    for e in range(-24, 4):                       # every bf16 value of 2^e <= |z| < 2^(e+1)
+        for m in range(128):
+            v = (1.0 + m / 128.0) * 2.0 ** e
+            if v <= 9.0:
+                grid += [v, -v]
+    rest = M * h - len(grid)
+    z = np.concatenate([np.asarray(grid), np.linspace(-9.0, 9.0, rest)]).astype(np.float32)
+    X = synth.f32_to_bf16_bits(z.reshape(M, h))
+    A = synth.f32_to_bf16_bits(np.eye(h, F, dtype=np.float32))
+    B = synth.f32_to_bf16_bits(np.ones((F, h), dtype=np.float32))
+    dY = synth.f32_to_bf16_bits(np.eye(M, h, dtype=np.float32))
+    b1 = np.zeros(F, dtype=np.uint16)
+    got = _run_backward(tp, X, A, b1, B, dY, n, residual=False)
+    zz = f64(X)
+    H = np.concatenate(list(got["dB"]), axis=1)   # [tokens][F]: H = GeLU(Z)
+    delta = 5e-7 * (1.0 + np.abs(zz))
+    for what, g, ref in (("GeLU", H, O.gelu(zz)), ("GeLU'", got["dX"], O.gelu_grad(zz))):
+        tol = _bf16_ulp(np.abs(ref) + delta) / 2 + delta
+        bad = np.abs(g - ref) > tol
+        assert not bad.any(), (what, zz[bad][:8], g[bad][:8], ref[bad][:8])

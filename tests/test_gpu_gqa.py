@@ -10,7 +10,7 @@ import pytest
 from oracle import tp_oracle as O
 from tensor_transformer_layer_linear_b200 import synth
 
-from helpers import BWD_FRO_REL, assert_parity, f64, from_dev_bf16, to_dev
+from helpers import BWD_FRO_REL, FRO_REL, assert_parity, f64, from_dev_bf16, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -184,12 +184,16 @@ def test_gqa_block_backward(tp, n_q, n_kv, n):
     ref = O.gqa_self_attention_backward_sharded(f64(inp["X"]), f64(inp["Wqkv"]), f64(inp["bqkv"]),
                                                 f64(inp["Wo"]), f64(inp["bo"]), f64(dY), batch,
                                                 seq, n_q, n_kv, n)
-    # backward gate: grouped key/value gradients add the group's rounding
-    assert_parity(from_dev_bf16(dX), ref["dX"], "dX", fro_rel=BWD_FRO_REL)
+    # With N > n_kv each duplicated key/value head's gradient is summed from
+    # bf16-stored per-replica shares: one more rounding in the longest chain,
+    # so those cases take the backward gate (measured 5.7e-3 at 8 query / 2
+    # key-value heads on 4 shards); without duplication the forward gate holds.
+    fro = BWD_FRO_REL if n > n_kv else FRO_REL
+    assert_parity(from_dev_bf16(dX), ref["dX"], "dX", fro_rel=fro)
     gW = dW.cpu().numpy().astype(np.float64)
     gb = db.cpu().numpy().astype(np.float64)
-    assert_parity(gW, ref["dWqkv_packed"], "dWqkv (per shard)", fro_rel=BWD_FRO_REL)
-    assert_parity(gb, ref["dbqkv_packed"], "dbqkv (per shard)", fro_rel=BWD_FRO_REL)
+    assert_parity(gW, ref["dWqkv_packed"], "dWqkv (per shard)", fro_rel=fro)
+    assert_parity(gb, ref["dbqkv_packed"], "dbqkv (per shard)", fro_rel=fro)
     assert_parity(dWo.cpu().numpy().astype(np.float64), O.packed_shards(ref["dWo"], O.SPLIT_ROW, n),
                   "dWo")
     assert_parity(dbo.cpu().numpy().astype(np.float64), ref["dbo"], "dbo")
@@ -197,4 +201,4 @@ def test_gqa_block_backward(tp, n_q, n_kv, n):
     logical = np.zeros_like(ref["dWqkv"])
     for i, c in enumerate(O.gqa_shard_columns(n_q, n_kv, d, n)):
         np.add.at(logical.T, c, gW[i])
-    assert_parity(logical, ref["dWqkv"], "dWqkv (replicas summed)", fro_rel=BWD_FRO_REL)
+    assert_parity(logical, ref["dWqkv"], "dWqkv (replicas summed)", fro_rel=fro)
