@@ -114,6 +114,31 @@ __device__ __forceinline__ AttnTile attn_tile(const AttnParams& p, int round) {
   return t;
 }
 
+// Packed two-wide fp32 FMA and add (sm_100: one instruction for two values):
+// the softmax forms S scale - m and accumulates the row sum a pair at a time,
+// half the FMA-pipe instructions of the scalar forms.
+__device__ __forceinline__ uint64_t pack_f32x2(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+  uint32_t a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(v));
+  lo = __uint_as_float(a);
+  hi = __uint_as_float(b);
+}
+__device__ __forceinline__ uint64_t ffma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -399,19 +424,26 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
           }
         }
         const float base = (m_used == -INFINITY) ? 0.f : m_used * sl2;
-        float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const uint64_t sl2x2 = pack_f32x2(__float_as_uint(sl2), __float_as_uint(sl2));
+        const uint64_t nbx2 = pack_f32x2(__float_as_uint(-base), __float_as_uint(-base));
+        uint64_t s4[4] = {0ull, 0ull, 0ull, 0ull};  // row-sum pairs (+0.0f, +0.0f)
 #pragma unroll
         for (int c = 0; c < FA_BN / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float a = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e]), sl2, -base));
-            const float bb = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e + 1]), sl2, -base));
-            s8[(e >> 1) & 7] += a + bb;
+            float xa, xb;
+            unpack_f32x2(ffma_f32x2(pack_f32x2(v[c * 32 + e], v[c * 32 + e + 1]), sl2x2, nbx2), xa, xb);
+            const float a = ex2_approx(xa);
+            const float bb = ex2_approx(xb);
+            s4[(e >> 1) & 3] = fadd_f32x2(s4[(e >> 1) & 3], pack_f32x2(__float_as_uint(a), __float_as_uint(bb)));
             pk[e >> 1] = pack_bf16x2(a, bb);
           }
           tmem_st_32x32b_x16(s_cols + c * 16, pk);
         }
+        float s8[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) unpack_f32x2(s4[u], s8[2 * u], s8[2 * u + 1]);
         l += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
         if (j == 0 && pending) {
           if (!epilogue(prev, tile - 1, prev_m, prev_l)) {
