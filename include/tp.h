@@ -34,6 +34,12 @@
  *     shard i is stored transposed (K-major), contiguous, one after another.
  *   - Arithmetic: bf16 inputs, fp32 accumulation, bf16 activations between
  *     the kernels, fp32 row-parallel partial sums.
+ *   - Per device, the library caches what it looks up once (the device's
+ *     error-word address, its SM count, the GEMM's resident CTA count, the
+ *     no-alloc array's address), keyed by device ordinal and guarded for
+ *     concurrent first calls. They belong to the device's primary context:
+ *     after cudaDeviceReset on a device, call nothing of this library on that
+ *     device again in the same process.
  */
 #ifndef TP_H
 #define TP_H
