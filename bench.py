@@ -126,7 +126,10 @@ def work(cfg: dict) -> dict:
             ab = 2.0 * att
         fl = {"gemm_backward": gb, "attention_backward": ab}
         if kind == "layer":
-            hbm("reduce_partials_layernorm_backward", n * M * h * 4 + 3 * M * h * 2 + h * 2)
+            # one LN-backward reduction per block (the MLP's through LN2, the
+            # attention block's through LN1), each of the same size
+            for _ in range(2):
+                hbm("reduce_partials_layernorm_backward", n * M * h * 4 + 3 * M * h * 2 + h * 2)
         else:
             hbm("reduce_partials", partial_read + (act if cfg.get("residual") else 0) + act)
         return dict(flops=fl, bytes=by, launch_bytes=launch, total_flops=sum(fl.values()))

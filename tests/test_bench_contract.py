@@ -80,3 +80,16 @@ def test_mlp_work_and_reduction_bytes():
     # the reduction reads N fp32 partials, the residual and the bias, writes Y
     expect = n * M * h * 4 + M * h * 2 + h * 2 + M * h * 2
     assert w["bytes"]["reduce_partials"] == expect
+
+
+def test_layer_backward_counts_both_ln_backward_reductions():
+    """The layer backward runs one LN-backward reduction per block (through
+    LN2 for the MLP, through LN1 for attention): the per-step bytes are two
+    launches' worth, each reading the N fp32 partials, the LN input and the
+    residual gradient and writing the input gradient."""
+    cfg = dict(synth.config("layer_2x2048_h4096_32x128_f16384_n8"), backward=True)
+    w = bench.work(cfg)
+    M, h, n = 2 * 2048, 4096, 8
+    one = n * M * h * 4 + 3 * M * h * 2 + h * 2
+    assert w["launch_bytes"]["reduce_partials_layernorm_backward"] == one
+    assert w["bytes"]["reduce_partials_layernorm_backward"] == 2 * one
