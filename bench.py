@@ -60,6 +60,8 @@ NCU_TRAFFIC = {
     (DEFAULT_WORKLOAD, "reduce_partials"): 574.0e6,
     (DEFAULT_WORKLOAD, "reduce_partials_layernorm"): 591.8e6,
     (DEFAULT_WORKLOAD, "layernorm"): 34.0e6,
+    # layer backward: the streamed LN-backward reduction (604.0 MB read + 13.8 MB written)
+    (DEFAULT_WORKLOAD, "reduce_partials_layernorm_backward"): 617.8e6,
 }
 
 

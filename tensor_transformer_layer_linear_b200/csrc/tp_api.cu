@@ -1096,7 +1096,7 @@ tp_status tp_reduce_partials_layernorm_backward(const float* partials, int n_sha
   TraceScope ts(tpk::KID_LAYERNORM_BWD, s);
   return tpk::launch_rows_sum_ln_bwd(partials, n_shards, B, h, x, gamma, residual_grad, eps, dX,
                                      dgamma, dbeta, static_cast<float*>(ws), kLnBwdMaxCtas, s,
-                                     d.num_sms) == 0
+                                     d.num_sms, d.err) == 0
              ? TP_OK
              : TP_ERR_CUDA;
 }
@@ -1209,7 +1209,7 @@ static tp_status layer_backward_impl(const uint16_t* X, int64_t batch, int64_t s
     TraceScope ts(tpk::KID_LAYERNORM_BWD, s);
     if (tpk::launch_rows_sum_ln_bwd(mb.part, n_shards, M, h, h1, w->ln2_gamma, dY, ln_eps, dh1,
                                     g->ln2_gamma, g->ln2_beta, lnb, kLnBwdMaxCtas, s, d.num_sms,
-                                    spn, sb, sq) != 0)
+                                    d.err, spn, sb, sq) != 0)
       return TP_ERR_CUDA;
   }
   if (sp) {  // the attention block's input gradient is needed in token order
@@ -1226,7 +1226,7 @@ static tp_status layer_backward_impl(const uint16_t* X, int64_t batch, int64_t s
   TraceScope ts(tpk::KID_LAYERNORM_BWD, s);
   return tpk::launch_rows_sum_ln_bwd(ab.part, n_shards, M, h, X, w->ln1_gamma, dh1, ln_eps, dX,
                                      g->ln1_gamma, g->ln1_beta, lnb, kLnBwdMaxCtas, s, d.num_sms,
-                                     spn, sb, sq) == 0
+                                     d.err, spn, sb, sq) == 0
              ? TP_OK
              : TP_ERR_CUDA;
 }

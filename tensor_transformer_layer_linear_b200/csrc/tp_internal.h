@@ -119,13 +119,14 @@ int launch_slab_sum(const float* partial, int slabs, int cols, float* out, cudaS
 // LayerNorm backward fused with the sum of N fp32 partials (the gradient at
 // the LN output) and a residual gradient: dx = residual + LN'(x)^T sum_i P_i
 // (bf16), dgamma, dbeta (fp32). part holds 2 * max_ctas * h floats of
-// per-CTA column sums. h % 8 == 0, h <= 16384. With sp_n > 0, x, residual
+// per-CTA column sums. h % 8 == 0, h <= 16384. A wait that gives up sets a
+// bit in *err. With sp_n > 0, x, residual
 // and dx use the sequence-sharded layout (partials stay in token order).
 int launch_rows_sum_ln_bwd(const float* P, int n_shards, int64_t rows, int64_t h, const void* x,
                            const void* gamma, const void* residual, float eps, void* dx,
                            float* dgamma, float* dbeta, float* part, int max_ctas,
-                           cudaStream_t s, int num_sms, int sp_n = 0, int sp_batch = 0,
-                           int sp_seq = 0);
+                           cudaStream_t s, int num_sms, unsigned* err, int sp_n = 0,
+                           int sp_batch = 0, int sp_seq = 0);
 
 // One thread waits, for at most limit_ns, on an mbarrier nothing arrives on,
 // then ORs ERR_WAIT_SELFTEST into *err (the bounded-wait failure path).

@@ -36,7 +36,12 @@ def _ws(tp, kind, M, h, F, n):
 
 
 @pytest.mark.parametrize("n,B,h", [(1, 64, 256), (2, 300, 1000), (3, 77, 512), (4, 130, 4096),
-                                   (8, 257, 4096), (2, 40, 12288)])
+                                   (8, 257, 4096), (2, 40, 12288),
+                                   # more shards than ring stages per row, many rows per CTA
+                                   (16, 1000, 1024), (5, 333, 1536),
+                                   # rows of two stages (the second one ragged or full)
+                                   (3, 17, 4104), (2, 150, 6152), (8, 64, 8192),
+                                   (1, 20, 16384)])
 def test_reduce_partials_layernorm_backward(tp, n, B, h):
     rng = np.random.default_rng(1400 + n + h)
     P = rng.standard_normal((n, B, h)).astype(np.float32)
