@@ -316,10 +316,13 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       const int b = it & 1;
       const float* lse_h = p.lse + head_row(it) * p.stride + row_base;
       const float* d_h = p.dsum + head_row(it) * p.stride + row_base;
-      if (!mbar_wait(bar(AB_SDP + b), (it >> 1) & 1, abort_flag) ||
-          (p.ld_bulk && !mbar_wait(bar(AB_LDFULL + b), (it >> 1) & 1, abort_flag)) ||
+      const bool got =
+          mbar_wait(bar(AB_SDP + b), (it >> 1) & 1, abort_flag) &&
+          (!p.ld_bulk || mbar_wait(bar(AB_LDFULL + b), (it >> 1) & 1, abort_flag)) &&
           // dS^T buffer b is free once dK and dQ^T of block it - 2 are done
-          (it >= 2 && !mbar_wait(bar(AB_DQFULL + b), ((it - 2) >> 1) & 1, abort_flag))) {
+          (it < 2 || mbar_wait(bar(AB_DQFULL + b), ((it - 2) >> 1) & 1, abort_flag));
+      // the warp leaves together (the TMEM accesses below are warp-collective)
+      if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
@@ -397,7 +400,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     if (!ok) {
       if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
       *abort_flag = 1;
-    } else if (mbar_wait(bar(AB_DONE), 0, abort_flag)) {
+    } else if (__all_sync(0xffffffffu, mbar_wait(bar(AB_DONE), 0, abort_flag))) {
       tc_fence_after();
       // tcgen05.ld is warp-collective: every lane loads, only rows inside
       // the sequence are stored; each group writes half of the 128 columns
@@ -441,9 +444,10 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(rq * 32) << 16;
     // accumulator rows [stride][128]: a warp's 32 lanes cover 128 contiguous bytes
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
+    for (int it = 0; ok && it < n_it; ++it) {
       const int b = it & 1;
-      if (!mbar_wait(bar(AB_DQFULL + b), (it >> 1) & 1, abort_flag)) {
+      // the warp leaves together (the TMEM loads are warp-collective)
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(AB_DQFULL + b), (it >> 1) & 1, abort_flag))) {
         ok = false;
         break;
       }
@@ -477,35 +481,42 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
   }
 }
 
-// D[(shard, head)][token] = sum_d dO * O over the head's 128 columns (fp32),
-// one warp per (shard, token, head).
-__global__ void __launch_bounds__(256) attn_bwd_dsum_kernel(const uint16_t* __restrict__ O,
-                                                            const uint16_t* __restrict__ dO,
-                                                            float* __restrict__ dsum,
-                                                            int64_t n_warps, int hps, int64_t M,
-                                                            int64_t stride) {
-  const int64_t w = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= n_warps) return;
-  const int head = static_cast<int>(w % hps);
-  const int64_t gr = w / hps;  // shard * M + token
-  const int64_t g = gr / M, tok = gr % M;
-  const int64_t off = gr * (static_cast<int64_t>(hps) * AB_D) + head * AB_D + lane * 4;
-  const uint2 o = __ldg(reinterpret_cast<const uint2*>(O + off));
-  const uint2 d = __ldg(reinterpret_cast<const uint2*>(dO + off));
-  float s = bf16_lo(o.x) * bf16_lo(d.x);
-  s = fmaf(bf16_hi(o.x), bf16_hi(d.x), s);
-  s = fmaf(bf16_lo(o.y), bf16_lo(d.y), s);
-  s = fmaf(bf16_hi(o.y), bf16_hi(d.y), s);
+// Before the main kernel: D[(shard, head)][token] = sum_d dO * O over the
+// head's 128 columns (fp32), and the token's row of the dQ accumulator
+// zeroed. 16 threads per (shard, token, head), 8 columns each.
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(
+    const uint16_t* __restrict__ O, const uint16_t* __restrict__ dO, float* __restrict__ dsum,
+    float* __restrict__ dq_acc, int64_t n_units, int hps, int64_t M, int64_t stride) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t u = i >> 4;
+  const int c8 = static_cast<int>(i & 15);
+  float s = 0.f;
+  int64_t hb = 0, tok = 0;
+  if (u < n_units) {
+    const int head = static_cast<int>(u % hps);
+    const int64_t gr = u / hps;  // shard * M + token
+    const int64_t g = gr / M;
+    tok = gr % M;
+    hb = g * hps + head;
+    const int64_t off = gr * (static_cast<int64_t>(hps) * AB_D) + head * AB_D + c8 * 8;
+    const uint4 o = __ldg(reinterpret_cast<const uint4*>(O + off));
+    const uint4 d = __ldg(reinterpret_cast<const uint4*>(dO + off));
+    s = bf16_lo(o.x) * bf16_lo(d.x);
+    s = fmaf(bf16_hi(o.x), bf16_hi(d.x), s);
+    s = fmaf(bf16_lo(o.y), bf16_lo(d.y), s);
+    s = fmaf(bf16_hi(o.y), bf16_hi(d.y), s);
+    s = fmaf(bf16_lo(o.z), bf16_lo(d.z), s);
+    s = fmaf(bf16_hi(o.z), bf16_hi(d.z), s);
+    s = fmaf(bf16_lo(o.w), bf16_lo(d.w), s);
+    s = fmaf(bf16_hi(o.w), bf16_hi(d.w), s);
+    float4* acc = reinterpret_cast<float4*>(dq_acc + (hb * stride + tok) * AB_D + c8 * 8);
+    acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // the 16 threads of a unit are 16 consecutive lanes of one warp
 #pragma unroll
-  for (int k = 16; k >= 1; k >>= 1) s += __shfl_xor_sync(0xffffffffu, s, k);
-  if (lane == 0) dsum[(g * hps + head) * stride + tok] = s;
-}
-
-__global__ void __launch_bounds__(256) zero_f32x4_kernel(float4* __restrict__ p, int64_t n4) {
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 8; k >= 1; k >>= 1) s += __shfl_xor_sync(0xffffffffu, s, k);
+  if (u < n_units && c8 == 0) dsum[hb * stride + tok] = s;
 }
 
 // dQ (bf16, scaled) into the Q columns of dQKV from the [stride][128]
@@ -581,22 +592,19 @@ int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const f
   if (!encode_rows(enc, &tm_do, dO, q_w, M, n_shards, AB_BQ)) return 1;
 
   const int64_t heads_total = static_cast<int64_t>(n_shards) * hps;
-  // dQ accumulator to zero, D = rowsum(dO * O)
-  const int64_t n4 = heads_total * AB_D * stride / 4;
-  int64_t zb = (n4 + 255) / 256;
-  if (zb > 8LL * num_sms) zb = 8LL * num_sms;
-  zero_f32x4_kernel<<<static_cast<unsigned>(zb), 256, 0, s>>>(reinterpret_cast<float4*>(dq_acc), n4);
-  const int64_t n_warps = static_cast<int64_t>(n_shards) * M * hps;
-  attn_bwd_dsum_kernel<<<static_cast<unsigned>((n_warps * 32 + 255) / 256), 256, 0, s>>>(
-      static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), dsum, n_warps, hps, M,
-      stride);
+  const int nq = static_cast<int>((seq + AB_BQ - 1) / AB_BQ);
+  // D = rowsum(dO * O) and the dQ accumulator's token rows zeroed
+  const int64_t n_units = heads_total * M;
+  attn_bwd_prep_kernel<<<static_cast<unsigned>((n_units * 16 + 255) / 256), 256, 0, s>>>(
+      static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), dsum, dq_acc, n_units,
+      hps, M, stride);
 
   AttnBwdParams p;
   p.seq = static_cast<int>(seq);
   p.batch = static_cast<int>(batch);
   p.hps = hps;
   p.causal = causal;
-  p.nq = static_cast<int>((seq + AB_BQ - 1) / AB_BQ);
+  p.nq = nq;
   p.kvl = kvl;
   p.group = hps / kvl;
   p.q_w = static_cast<int>(q_w);

@@ -433,6 +433,22 @@ static size_t attn_core_bwd_bytes(size_t M, size_t H) {
   const size_t rows = M + 128;
   return round256(H / 128 * rows * 4) + round256(H * rows * 4);
 }
+
+// The attention backward's scratch inside a workspace of attn_core_bwd_bytes
+// (n_q heads of 128 columns).
+struct AttnBwdScratch {
+  float* dsum;
+  float* dq_acc;
+};
+static AttnBwdScratch attn_bwd_scratch(void* base, size_t M, size_t n_q) {
+  const size_t rows = M + 128;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  AttnBwdScratch sc;
+  sc.dsum = reinterpret_cast<float*>(p);
+  p += round256(n_q * rows * 4);
+  sc.dq_acc = reinterpret_cast<float*>(p);
+  return sc;
+}
 static size_t attn_bwd_bytes(size_t M, size_t H, size_t N) {
   // core + QKV, dQKV, O, dO (bf16) + lse + dX partials + column-sum slabs
   return attn_core_bwd_bytes(M, H) + 2 * round256(M * 3 * H * 2) + 2 * round256(M * H * 2) +
@@ -951,15 +967,12 @@ tp_status tp_attention_backward(const uint16_t* QKV_shards, const uint16_t* O_sh
   DevInfo d;
   tp_status st = device_info(&d);
   if (st != TP_OK) return st;
-  const size_t rows = static_cast<size_t>(M) + 128;
-  float* dsum = static_cast<float*>(ws);
-  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                           round256(static_cast<size_t>(h) / 128 * rows * 4));
+  const AttnBwdScratch sc = attn_bwd_scratch(ws, static_cast<size_t>(M), n_heads);
   TraceScope ts(tpk::KID_ATTENTION_BWD, as_stream(stream));
   const int rc = tpk::launch_attention_bwd(QKV_shards, O_shards, dO_shards, lse, batch, seq,
                                            n_heads, n_heads / n_shards, n_shards, causal ? 1 : 0,
-                                           dQKV_shards, dsum, dq_acc, as_stream(stream), d.err,
-                                           d.num_sms);
+                                           dQKV_shards, sc.dsum, sc.dq_acc,
+                                           as_stream(stream), d.err, d.num_sms);
   return rc == 0 ? TP_OK : TP_ERR_CUDA;
 }
 
@@ -1008,13 +1021,11 @@ static tp_status attn_backward_core(const DevInfo& d, void* stream, const uint16
                           H, false);
   if (st != TP_OK) return st;
   {
-    const size_t rows = static_cast<size_t>(M) + 128;
-    float* dsum = static_cast<float*>(b.core);
-    float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(b.core) +
-                                             round256(static_cast<size_t>(n_q) * rows * 4));
+    const AttnBwdScratch sc = attn_bwd_scratch(b.core, static_cast<size_t>(M), n_q);
     TraceScope ts(tpk::KID_ATTENTION_BWD, s);
     if (tpk::launch_attention_bwd(b.qkv, b.o, b.dO, b.lse, batch, seq, n_q, kvl, n_shards,
-                                  causal ? 1 : 0, b.dqkv, dsum, dq_acc, s, d.err, d.num_sms) != 0)
+                                  causal ? 1 : 0, b.dqkv, sc.dsum, sc.dq_acc, s, d.err,
+                                  d.num_sms) != 0)
       return TP_ERR_CUDA;
   }
   // dW_QKV,i^T = dQKV_i^T X (packed like Wqkv_shards), dW_O,i^T = dY^T O_i (like Wo_shards)
@@ -1288,14 +1299,11 @@ tp_status tp_attention_gqa_backward(const uint16_t* QKV_shards, const uint16_t* 
   DevInfo d;
   tp_status st = device_info(&d);
   if (st != TP_OK) return st;
-  const size_t rows = static_cast<size_t>(M) + 128;
-  float* dsum = static_cast<float*>(ws);
-  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                           round256(static_cast<size_t>(n_q) * rows * 4));
+  const AttnBwdScratch sc = attn_bwd_scratch(ws, static_cast<size_t>(M), n_q);
   TraceScope ts(tpk::KID_ATTENTION_BWD, as_stream(stream));
   const int rc = tpk::launch_attention_bwd(QKV_shards, O_shards, dO_shards, lse, batch, seq, n_q,
                                            gqa_kv_local(n_kv, n_shards), n_shards,
-                                           causal ? 1 : 0, dQKV_shards, dsum, dq_acc,
+                                           causal ? 1 : 0, dQKV_shards, sc.dsum, sc.dq_acc,
                                            as_stream(stream), d.err, d.num_sms);
   return rc == 0 ? TP_OK : TP_ERR_CUDA;
 }
