@@ -27,7 +27,9 @@
 //              of dV += P^T dO), and dS^T = P^T * (dP^T - D) in bf16 into a
 //              swizzled shared tile, the K-major A operand of dK += dS^T Q
 //              and the MN-major B operand of dQ^T = K^T dS^T; at the end they
-//              write dK (scaled) and dV in bf16, half of the columns each;
+//              write dK (scaled) and dV in bf16, half of the columns each,
+//              through 128-byte-swizzled tiles in the (then idle) Q ring and
+//              TMA tensor stores (direct stores for rows past the sequence);
 //   warps 8-11 one thread per head-dimension column (TMEM lane): drain the
 //              block's dQ^T from TMEM into an fp32 accumulator in global
 //              memory with reductions (every key block of the sequence
@@ -108,7 +110,8 @@ __device__ __forceinline__ void red_add_f32(float* addr, uint32_t v) {
 __global__ void __launch_bounds__(AB_THREADS, 1)
     attention_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
                             const __grid_constant__ CUtensorMap tm_q,
-                            const __grid_constant__ CUtensorMap tm_do, const AttnBwdParams p) {
+                            const __grid_constant__ CUtensorMap tm_do,
+                            const __grid_constant__ CUtensorMap tm_st, const AttnBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* sm = smem_raw + pad;
@@ -160,6 +163,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     tma_prefetch_desc(&tm_kv);
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_st);
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_holder), 512);
   tc_fence_before();
@@ -402,36 +406,55 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       *abort_flag = 1;
     } else if (__all_sync(0xffffffffu, mbar_wait(bar(AB_DONE), 0, abort_flag))) {
       tc_fence_after();
-      // tcgen05.ld is warp-collective: every lane loads, only rows inside
-      // the sequence are stored; each group writes half of the 128 columns
+      // tcgen05.ld is warp-collective: every lane loads. The warp's 32 keys x
+      // 64 columns of dK (scaled) and of dV go to its two 4 KB tiles in the Q
+      // ring (idle once every MMA is done), 128-byte swizzled, and leave with
+      // two TMA stores when all 32 keys are inside the sequence; otherwise
+      // the keys inside it are stored directly.
+      const uint32_t tile = s0 + AOFF_Q + static_cast<uint32_t>(grp * 4 + rq) * 8192u;
+      const uint32_t trow = tile + static_cast<uint32_t>(lane) * 128u;
+      const bool box_inside = kv0 + rq * 32 + 32 <= p.seq;
       uint16_t* base = p.dqkv + (static_cast<int64_t>(g) * p.M + row_base + key) * p.ld +
-                       p.q_w + kvh * AB_D;  // dK here, dV kvl x 128 columns further
-#pragma unroll 1
-      for (int c = 4 * grp; c < 4 * grp + 4; ++c) {  // 16 columns at a time
-        uint32_t kv[16], vv[16];
-        tmem_ld_32x32b_x16(tmem + lane_addr + 384u + c * 16, kv);
-        tmem_ld_32x32b_x16(tmem + lane_addr + 256u + c * 16, vv);
-        tmem_ld_wait();
-        if (key < p.seq) {
+                       p.q_w + kvh * AB_D + grp * 64;  // dK here, dV kvl x 128 columns further
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            uint4 wk, wv;
-            wk.x = pack_bf16x2(__uint_as_float(kv[8 * e + 0]) * p.scale,
-                               __uint_as_float(kv[8 * e + 1]) * p.scale);
-            wk.y = pack_bf16x2(__uint_as_float(kv[8 * e + 2]) * p.scale,
-                               __uint_as_float(kv[8 * e + 3]) * p.scale);
-            wk.z = pack_bf16x2(__uint_as_float(kv[8 * e + 4]) * p.scale,
-                               __uint_as_float(kv[8 * e + 5]) * p.scale);
-            wk.w = pack_bf16x2(__uint_as_float(kv[8 * e + 6]) * p.scale,
-                               __uint_as_float(kv[8 * e + 7]) * p.scale);
-            wv.x = pack_bf16x2(__uint_as_float(vv[8 * e + 0]), __uint_as_float(vv[8 * e + 1]));
-            wv.y = pack_bf16x2(__uint_as_float(vv[8 * e + 2]), __uint_as_float(vv[8 * e + 3]));
-            wv.z = pack_bf16x2(__uint_as_float(vv[8 * e + 4]), __uint_as_float(vv[8 * e + 5]));
-            wv.w = pack_bf16x2(__uint_as_float(vv[8 * e + 6]), __uint_as_float(vv[8 * e + 7]));
-            *reinterpret_cast<uint4*>(base + c * 16 + 8 * e) = wk;
-            *reinterpret_cast<uint4*>(base + p.kvl * AB_D + c * 16 + 8 * e) = wv;
+      for (int kv = 0; kv < 2; ++kv) {  // dK, then dV
+        const float sc = kv == 0 ? p.scale : 1.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {  // 32 columns at a time
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + lane_addr + (kv == 0 ? 384u : 256u) + grp * 64 + c * 32, v);
+          tmem_ld_wait();
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
+          if (box_inside) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint32_t chunk = static_cast<uint32_t>(c * 4 + u);
+              st_shared_v4(trow + kv * 4096u + ((chunk ^ (static_cast<uint32_t>(lane) & 7u)) << 4),
+                           w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+            }
+          } else if (key < p.seq) {
+            uint4* dst = reinterpret_cast<uint4*>(base + kv * p.kvl * AB_D + c * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
           }
         }
+      }
+      if (box_inside) {
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          const int col = p.q_w + kvh * AB_D + grp * 64;
+          const int trow0 = row_base + kv0 + rq * 32;
+          tma_store_3d(&tm_st, tile, col, trow0, g);
+          tma_store_3d(&tm_st, tile + 4096u, col + p.kvl * AB_D, trow0, g);
+          bulk_commit();
+          bulk_wait<0>();  // written before the CTA (and its shared memory) goes away
+        }
+        __syncwarp();
       }
     } else {
       if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
@@ -586,10 +609,11 @@ int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const f
   const int64_t stride = M + 128;
   auto enc = bwd_map_encoder();
   if (enc == nullptr) return 1;
-  CUtensorMap tm_kv, tm_q, tm_do;
+  CUtensorMap tm_kv, tm_q, tm_do, tm_st;
   if (!encode_rows(enc, &tm_kv, QKV, ld, M, n_shards, AB_BK)) return 1;
   if (!encode_rows(enc, &tm_q, QKV, ld, M, n_shards, AB_BQ)) return 1;
   if (!encode_rows(enc, &tm_do, dO, q_w, M, n_shards, AB_BQ)) return 1;
+  if (!encode_rows(enc, &tm_st, dQKV, ld, M, n_shards, 32)) return 1;  // dK / dV stores
 
   const int64_t heads_total = static_cast<int64_t>(n_shards) * hps;
   const int nq = static_cast<int>((seq + AB_BQ - 1) / AB_BQ);
@@ -623,7 +647,7 @@ int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const f
                        AB_SMEM);
   const dim3 grid(static_cast<unsigned>(static_cast<int64_t>(n_shards) * kvl * batch),
                   static_cast<unsigned>((seq + AB_BK - 1) / AB_BK));
-  attention_bwd_tc_kernel<<<grid, AB_THREADS, AB_SMEM, s>>>(tm_kv, tm_q, tm_do, p);
+  attention_bwd_tc_kernel<<<grid, AB_THREADS, AB_SMEM, s>>>(tm_kv, tm_q, tm_do, tm_st, p);
 
   const int64_t n = heads_total * M * (AB_D / 8);
   attn_bwd_dq_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
