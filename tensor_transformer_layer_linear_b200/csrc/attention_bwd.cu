@@ -419,15 +419,18 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {  // dK, then dV
         const float sc = kv == 0 ? p.scale : 1.f;
+        // both 32-column halves in flight before the first wait
+        uint32_t v[2][32];
+        tmem_ld_32x32b_x32(tmem + lane_addr + (kv == 0 ? 384u : 256u) + grp * 64, v[0]);
+        tmem_ld_32x32b_x32(tmem + lane_addr + (kv == 0 ? 384u : 256u) + grp * 64 + 32, v[1]);
+        tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 2; ++c) {  // 32 columns at a time
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tmem + lane_addr + (kv == 0 ? 384u : 256u) + grp * 64 + c * 32, v);
-          tmem_ld_wait();
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
+            w[e] = pack_bf16x2(__uint_as_float(v[c][2 * e]) * sc,
+                               __uint_as_float(v[c][2 * e + 1]) * sc);
           if (box_inside) {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -452,7 +455,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
           tma_store_3d(&tm_st, tile, col, trow0, g);
           tma_store_3d(&tm_st, tile + 4096u, col + p.kvl * AB_D, trow0, g);
           bulk_commit();
-          bulk_wait<0>();  // written before the CTA (and its shared memory) goes away
+          bulk_wait_read<0>();  // the tiles are read before the CTA's shared memory goes away
         }
         __syncwarp();
       }
