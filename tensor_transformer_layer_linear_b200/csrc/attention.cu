@@ -24,19 +24,22 @@
 //              [shard][token][3h/N] output (128-byte swizzle).
 //   warp 6     TMA: the V blocks into their own 2-deep ring.
 //   warp 5     TMEM owner and the single MMA-issuing thread.
-// S is double-buffered in TMEM, so the MMAs of a key block overlap the
-// softmax of the previous one. Blocks are numbered over the CTA's whole work
-// list, and the MMA order is
-//   S_0 = Q K_0^T | S_1 = Q K_1^T | O = P_0 V_0 | S_2 = Q K_2^T |
-//   O += P_1 V_1 | S_3 = Q K_3^T | ...
+// S has three buffers in TMEM, so the MMAs of the next key blocks overlap
+// the softmax of the current one. Blocks are numbered over the CTA's whole
+// work list, and the MMA order is
+//   S_0 = Q K_0^T | S_1 | S_2 | O = P_0 V_0 | S_3 | O += P_1 V_1 | S_4 | ...
 // running on across tile boundaries (S of the next tile's first blocks is
-// computed while the softmax finishes the current tile). S_{n+2} overwrites
+// computed while the softmax finishes the current tile). S_{n+3} overwrites
 // the buffer holding P_n right after the MMA that reads it, relying on one
 // thread's tcgen05.mma operations executing in issue order. A commit after
 // every PV tells the softmax when O holds exactly the blocks before its own
 // (needed only for a rescale); a commit after a tile's last PV releases its O
 // to the softmax warps, whose next P arrival in turn releases the columns.
-// TMEM: S / P buffer b at columns [128 b, 128 b + 128), O at [256, 384).
+// When the softmax sees S_n, PV_{n-3} is complete but PV_{n-2} may not be,
+// so both commits alternate between two barriers (by block and by tile
+// parity): a parity wait on one barrier is then never two phases behind.
+// TMEM: S / P buffer b at columns [128 b, 128 b + 128) (b < 3), O at
+// [384, 512).
 // Causal tiles stop at their diagonal block. Every barrier wait is bounded;
 // a role that gives up records an error bit and the CTA leaves through the
 // common exit after waiting (bounded) for its copies and MMAs in flight.
@@ -60,13 +63,14 @@ constexpr int OFF_Q = 0;                    // 2 buffers (the next tile's Q load
 constexpr int OFF_K = OFF_Q + 2 * FA_TILE;  // 2 buffers
 constexpr int OFF_V = OFF_K + 2 * FA_TILE;  // 2 buffers
 constexpr int OFF_BAR = OFF_V + 2 * FA_TILE;
-constexpr int FA_NUM_BARS = 20;
+constexpr int FA_NUM_BARS = 23;
+constexpr int FA_SBUF = 3;                  // S / P buffers in TMEM
 constexpr int FA_SMEM = 1024 + OFF_BAR + FA_NUM_BARS * 8 + 16;
 static_assert(FA_SMEM <= 232448, "shared memory budget");
 
 // barrier indices (Q, K, V, S and P per buffer b)
 constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = 6, B_VFULL = 8, B_VEMPTY = 10,
-              B_SFULL = 12, B_PFULL = 14, B_OUPD = 16, B_ODONE = 17, B_DRAIN = 18;
+              B_SFULL = 12, B_PFULL = 15, B_OUPD = 18, B_ODONE = 20, B_DRAIN = 22;
 
 struct AttnParams {
   int seq, batch, hps, causal, nq;
@@ -168,11 +172,15 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       mbar_init(bar(B_KEMPTY + b), 1);
       mbar_init(bar(B_VFULL + b), 1);
       mbar_init(bar(B_VEMPTY + b), 1);
+    }
+    for (int b = 0; b < FA_SBUF; ++b) {
       mbar_init(bar(B_SFULL + b), 1);
       mbar_init(bar(B_PFULL + b), 4);  // one arrival per softmax warp
     }
-    mbar_init(bar(B_OUPD), 1);
-    mbar_init(bar(B_ODONE), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(B_OUPD + b), 1);   // PV of blocks b, b + 2, ... complete
+      mbar_init(bar(B_ODONE + b), 1);  // O of tiles b, b + 2, ... complete
+    }
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -267,9 +275,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
       };
       bool ok = true;
-      // S_blk = Q K_blk^T into buffer blk & 1
+      // S_blk = Q K_blk^T into buffer blk % FA_SBUF (K from ring slot blk & 1)
       auto qk = [&]() -> bool {
-        const int qb = cq.tile & 1, b = cq.blk & 1;
+        const int qb = cq.tile & 1, b = cq.blk & 1, sb = cq.blk % FA_SBUF;
         if (cq.j == 0 && !mbar_wait(bar(B_QFULL + qb), (cq.tile >> 1) & 1, abort_flag)) return false;
         if (!mbar_wait(bar(B_KFULL + b), (cq.blk >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
@@ -277,21 +285,21 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < FA_D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * FA_SUB + (kk & 3) * 32;
-          umma_bf16(tmem + b * FA_BN, desc_advance(dq, off), desc_advance(dk, off), idesc_s,
+          umma_bf16(tmem + sb * FA_BN, desc_advance(dq, off), desc_advance(dk, off), idesc_s,
                     kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(B_KEMPTY + b));
-        umma_commit(bar(B_SFULL + b));
+        umma_commit(bar(B_SFULL + sb));
         if (cq.j == cq.t.nb - 1) umma_commit(bar(B_QEMPTY + qb));  // the tile's last QK^T
         advance(cq);
         return true;
       };
-      for (int n = 0; ok && n < 2 && cq.t.valid; ++n) ok = qk();
+      for (int n = 0; ok && n < FA_SBUF && cq.t.valid; ++n) ok = qk();
       while (ok && cp.t.valid) {
-        const int b = cp.blk & 1;
-        const uint32_t ph = (cp.blk >> 1) & 1;
+        const int b = cp.blk & 1, pb = cp.blk % FA_SBUF;
+        const uint32_t ph = (cp.blk >> 1) & 1, pph = (cp.blk / FA_SBUF) & 1;
         if (!mbar_wait(bar(B_VFULL + b), ph, abort_flag) ||
-            !mbar_wait(bar(B_PFULL + b), ph, abort_flag)) {
+            !mbar_wait(bar(B_PFULL + pb), pph, abort_flag)) {
           ok = false;
           break;
         }
@@ -299,11 +307,11 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         const uint64_t dv = b ? dv1 : dv0;
 #pragma unroll
         for (int kk = 0; kk < FA_BN / 16; ++kk)             // O (+)= P V
-          umma_bf16_tmem_a(tmem + 2 * FA_BN, tmem + b * FA_BN + kk * 8,
+          umma_bf16_tmem_a(tmem + FA_SBUF * FA_BN, tmem + pb * FA_BN + kk * 8,
                            desc_advance(dv, kk * 2048), idesc_o, (cp.j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(B_VEMPTY + b));
-        umma_commit(bar(B_OUPD));
-        if (cp.j == cp.t.nb - 1) umma_commit(bar(B_ODONE));  // the tile's O is complete
+        umma_commit(bar(B_OUPD + (cp.blk & 1)));
+        if (cp.j == cp.t.nb - 1) umma_commit(bar(B_ODONE + (cp.tile & 1)));  // the tile's O is complete
         advance(cp);
         if (cq.t.valid) ok = qk();                           // reuses the buffer P was in
       }
@@ -320,7 +328,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     // ------------------------------------------------------------ softmax
     const int r = warp * 32 + lane;  // row within the tile (= TMEM lane)
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t o_cols = tmem + lane_addr + 2 * FA_BN;
+    const uint32_t o_cols = tmem + lane_addr + FA_SBUF * FA_BN;
     const float sl2 = p.scale_log2;
     bool ok = true;
     // A tile's O: normalise and store it. It runs after the next tile's first
@@ -328,7 +336,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     // that P's arrival, which is what lets the next tile's first PV
     // overwrite the O columns.
     auto epilogue = [&](const AttnTile& tl, int tile, float m_used, float l) -> bool {
-      if (!mbar_wait(bar(B_ODONE), tile & 1, abort_flag)) return false;
+      if (!mbar_wait(bar(B_ODONE + (tile & 1)), (tile >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
       const int t = tl.q0 + r;
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -370,8 +378,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       const int t = q0 + r;  // query position within the sequence
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < tl.nb; ++j, ++blk) {
-        const int b = blk & 1;
-        if (!mbar_wait(bar(B_SFULL + b), (blk >> 1) & 1, abort_flag)) {
+        const int b = blk % FA_SBUF;
+        if (!mbar_wait(bar(B_SFULL + b), (blk / FA_SBUF) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -408,7 +416,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
         if (__any_sync(0xffffffffu, need && j > 0)) {
           // O must hold exactly the tile's blocks before j: wait for the previous PV
-          if (!mbar_wait(bar(B_OUPD), (blk - 1) & 1, abort_flag)) {
+          if (!mbar_wait(bar(B_OUPD + ((blk - 1) & 1)), ((blk - 1) >> 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
