@@ -54,8 +54,8 @@ NCU_TRAFFIC = {
     (DEFAULT_WORKLOAD, "gemm_column_parallel"): 280.2e6,
     # W_O 540.5 MB and MLP-down 765.1 MB -> mean per launch
     (DEFAULT_WORKLOAD, "gemm_row_parallel"): 652.8e6,
-    # persistent attention (packed softmax): 151.3 MB read + 14.6 MB written
-    (DEFAULT_WORKLOAD, "attention"): 165.9e6,
+    # persistent attention (three S buffers): 134.1 MB read + 14.2 MB written
+    (DEFAULT_WORKLOAD, "attention"): 148.3e6,
     # the reductions and LN1 (profiles/reduce_partials_ncu.md): read + write per launch
     (DEFAULT_WORKLOAD, "reduce_partials"): 574.0e6,
     (DEFAULT_WORKLOAD, "reduce_partials_layernorm"): 591.8e6,
