@@ -10,7 +10,7 @@
 //   dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d),
 // where P is rebuilt from the forward's log-sum-exp.
 //
-// One CTA per (shard, sequence, key/value head, 128-key block), 16 warps,
+// One CTA per (shard, sequence, key/value head, 128-key block), 22 warps,
 // stepping through the 64-query blocks of every query head that uses the
 // key/value head (one for multi-head attention, the group for grouped-query
 // attention: the key block's dK and dV sum over the group):
@@ -20,25 +20,26 @@
 //              its lse and D into a 2-deep shared ring (bulk copies when the
 //              rows are 16-byte aligned);
 //   warp 1     TMEM owner and the single MMA-issuing thread;
-//   warps 4-7, 12-15
-//              two threads per key (TMEM lane), each for 32 of the block's 64
-//              queries: P^T = exp2(S^T scale - lse), masked, stored as bf16
-//              pairs over the S^T columns the thread has read (the A operand
-//              of dV += P^T dO), and dS^T = P^T * (dP^T - D) in bf16 into a
-//              swizzled shared tile, the K-major A operand of dK += dS^T Q
-//              and the MN-major B operand of dQ^T = K^T dS^T; at the end they
-//              write dK (scaled) and dV in bf16, half of the columns each,
-//              through 128-byte-swizzled tiles in the (then idle) Q ring and
-//              TMA tensor stores (direct stores for rows past the sequence);
-//   warps 8-11 one thread per head-dimension column (TMEM lane): drain the
+//   warps 2-5  one thread per head-dimension column (TMEM lane): drain the
 //              block's dQ^T from TMEM into an fp32 accumulator in global
 //              memory with reductions (every key block of the sequence
-//              contributes to it).
+//              contributes to it);
+//   warps 6-21 four threads per key (TMEM lane), each for 16 of the block's
+//              64 queries: P^T = exp2(S^T scale - lse), masked, stored as
+//              bf16 pairs over the first 8 of the 16 S^T columns the thread
+//              has read (the A operand of dV += P^T dO), and
+//              dS^T = P^T * (dP^T - D) in bf16 into a swizzled shared tile,
+//              the K-major A operand of dK += dS^T Q and the MN-major B
+//              operand of dQ^T = K^T dS^T; at the end each writes 32 columns
+//              of dK (scaled) and dV in bf16 through tiles in the (then idle)
+//              Q ring and TMA tensor stores (direct stores for rows past the
+//              sequence).
 // S^T and dP^T are double-buffered in TMEM, so the tensor cores compute the
 // next block's S^T = K Q^T and dP^T = V dO^T while the key threads work on
 // the current one; dQ^T of a block lands in that block's dP^T columns once
-// they are read. TMEM: buffer b in [128 b, 128 b + 128) (S^T, then P^T in its
-// columns [0, 16) and [32, 48); dP^T, then dQ^T, in its last 64), dV
+// they are read. TMEM: buffer b in [128 b, 128 b + 128) (S^T, then P^T of
+// queries [16 k, 16 k + 16) in its columns [16 k, 16 k + 8); dP^T, then dQ^T,
+// in its last 64), dV
 // [256, 384), dK [384, 512). Causal key blocks start at the first query block that sees
 // them; the heaviest (first) key blocks launch first. Every barrier wait is
 // bounded; a role that gives up records an error bit and the CTA leaves
@@ -57,7 +58,7 @@ namespace tpk {
 constexpr int AB_BK = 128;        // keys per CTA
 constexpr int AB_BQ = 64;         // queries per step
 constexpr int AB_D = 128;         // head dim
-constexpr int AB_THREADS = 512;
+constexpr int AB_THREADS = 704;  // 22 warps
 constexpr int AB_NST = 4;         // Q / dO ring depth
 constexpr int AB_KSUB = 128 * 128;          // [128 rows][64 cols] bf16: 16 KB
 constexpr int AB_KTILE = 2 * AB_KSUB;       // [128][128] bf16: K or V
@@ -149,11 +150,11 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(AB_SDP + b), 1);
-      mbar_init(bar(AB_DS + b), 8);       // one arrival per key warp
+      mbar_init(bar(AB_DS + b), 16);      // one arrival per key warp
       mbar_init(bar(AB_DQFULL + b), 1);
       mbar_init(bar(AB_DQEMPTY + b), 4);  // one arrival per drain warp
       mbar_init(bar(AB_LDFULL + b), 1);
-      mbar_init(bar(AB_LDEMPTY + b), 8);  // one arrival per key warp
+      mbar_init(bar(AB_LDEMPTY + b), 16); // one arrival per key warp
     }
     mbar_init(bar(AB_DONE), 1);
     *abort_flag = 0;
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       // dV += P^T dO: P^T (keys x queries, bf16 pairs) from TMEM
 #pragma unroll
       for (int kk = 0; kk < AB_BQ / 16; ++kk)
-        umma_bf16_tmem_a(tmem + 256u, tS + kk * 8 + (kk >= 2 ? 16 : 0),  // P^T of queries 16 kk..
+        umma_bf16_tmem_a(tmem + 256u, tS + kk * 16,  // P^T of queries 16 kk.. (8 columns)
                          desc_advance(dO_mn, kk * 2048),
                          idesc_kmn, (it > 0 || kk > 0) ? 1u : 0u);
       // dK += dS^T Q
@@ -307,10 +308,10 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     umma_commit(bar(AB_DONE));
     int never = 0;
     if (!mbar_wait(bar(AB_DONE), 0, &never)) atomicOr(p.err, ERR_WAIT_DRAIN);
-  } else if ((warp >= 4 && warp < 8) || warp >= 12) {
+  } else if (warp >= 6) {
     // ------------------------------------------------------------ P^T, dS^T
     const int rq = warp & 3;
-    const int grp = warp >= 12 ? 1 : 0;  // queries [32 grp, 32 grp + 32) of each block
+    const int grp = (warp - 6) >> 2;     // queries [16 grp, 16 grp + 16) of each block
     const int row = rq * 32 + lane;      // key within the block (= TMEM lane)
     const int key = kv0 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(rq * 32) << 16;
@@ -339,23 +340,23 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       const uint32_t s_lse = s0 + AOFF_LD + b * (2 * AB_BQ * 4), s_d = s_lse + AB_BQ * 4;
       const uint32_t ds_row = s0 + AOFF_DS + b * AB_DSTILE + static_cast<uint32_t>(row) * 128u;
       {
-        // this thread's 32 queries [32 grp, 32 grp + 32): one TMEM round trip
-        const int c = grp;
-        uint32_t sv[32], dv[32];
-        tmem_ld_32x32b_x32(tS + c * 32, sv);
-        tmem_ld_32x32b_x32(tP + c * 32, dv);
+        // this thread's 16 queries [16 grp, 16 grp + 16): one TMEM round trip
+        const int c0 = grp * 16;
+        uint32_t sv[16], dv[16];
+        tmem_ld_32x32b_x16(tS + c0, sv);
+        tmem_ld_32x32b_x16(tP + c0, dv);
         tmem_ld_wait();
-        uint32_t pk[16], dk[16];
+        uint32_t pk[8], dk[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
+        for (int e = 0; e < 16; e += 4) {
           // lse and D of these 4 queries: the same for every key thread
           float4 l4, d4;
           if (p.ld_bulk) {
-            l4 = ld_shared_v4f(s_lse + (c * 32 + e) * 4);
-            d4 = ld_shared_v4f(s_d + (c * 32 + e) * 4);
+            l4 = ld_shared_v4f(s_lse + (c0 + e) * 4);
+            d4 = ld_shared_v4f(s_d + (c0 + e) * 4);
           } else {
-            const float* lp = lse_h + q0 + c * 32 + e;
-            const float* dp = d_h + q0 + c * 32 + e;
+            const float* lp = lse_h + q0 + c0 + e;
+            const float* dp = d_h + q0 + c0 + e;
             l4 = make_float4(__ldg(lp), __ldg(lp + 1), __ldg(lp + 2), __ldg(lp + 3));
             d4 = make_float4(__ldg(dp), __ldg(dp + 1), __ldg(dp + 2), __ldg(dp + 3));
           }
@@ -367,7 +368,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
             const float pv = ex2_approx(fmaf(__uint_as_float(sv[e + u]), sl2, -lq[u]));
             const float dsv = pv * (__uint_as_float(dv[e + u]) - dq[u]);
             if (need_mask) {
-              const int q = q0 + c * 32 + e + u;
+              const int q = q0 + c0 + e + u;
               const bool valid = key < p.seq && q < p.seq && (!p.causal || q >= key);
               pp[u] = valid ? pv : 0.f;
               ds[u] = valid ? dsv : 0.f;
@@ -381,13 +382,14 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
           dk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
           dk[(e >> 1) + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        // P^T of the 32 queries into 16 columns of S^T this thread has read
-        tmem_st_32x32b_x16(tS + c * 32, pk);
-        // dS^T row `row`, queries [32 c, 32 c + 32): four 16-byte chunks of
-        // the 128-byte swizzled row
+        // P^T of the 16 queries into the first 8 of the 16 S^T columns this
+        // thread has read
+        tmem_st_32x32b_x8(tS + c0, pk);
+        // dS^T row `row`, queries [16 grp, 16 grp + 16): two 16-byte chunks
+        // of the 128-byte swizzled row
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t chunk = static_cast<uint32_t>(c * 4 + u);
+        for (int u = 0; u < 2; ++u) {
+          const uint32_t chunk = static_cast<uint32_t>(grp * 2 + u);
           st_shared_v4(ds_row + ((chunk ^ (static_cast<uint32_t>(row) & 7u)) << 4), dk[4 * u],
                        dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
@@ -407,53 +409,47 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
     } else if (__all_sync(0xffffffffu, mbar_wait(bar(AB_DONE), 0, abort_flag))) {
       tc_fence_after();
       // tcgen05.ld is warp-collective: every lane loads. The warp's 32 keys x
-      // 64 columns of dK (scaled) and of dV go to its two 4 KB tiles in the Q
-      // ring (idle once every MMA is done), 128-byte swizzled, and leave with
-      // two TMA stores when all 32 keys are inside the sequence; otherwise
-      // the keys inside it are stored directly.
-      const uint32_t tile = s0 + AOFF_Q + static_cast<uint32_t>(grp * 4 + rq) * 8192u;
-      const uint32_t trow = tile + static_cast<uint32_t>(lane) * 128u;
+      // 32 columns of dK (scaled) and of dV go to its two 2 KB tiles in the Q
+      // ring (idle once every MMA is done), 64-byte rows, and leave with two
+      // TMA stores when all 32 keys are inside the sequence; otherwise the
+      // keys inside it are stored directly.
+      const uint32_t tile = s0 + AOFF_Q + static_cast<uint32_t>(grp * 4 + rq) * 4096u;
+      const uint32_t trow = tile + static_cast<uint32_t>(lane) * 64u;
       const bool box_inside = kv0 + rq * 32 + 32 <= p.seq;
       uint16_t* base = p.dqkv + (static_cast<int64_t>(g) * p.M + row_base + key) * p.ld +
-                       p.q_w + kvh * AB_D + grp * 64;  // dK here, dV kvl x 128 columns further
+                       p.q_w + kvh * AB_D + grp * 32;  // dK here, dV kvl x 128 columns further
+      uint32_t v[2][32];  // dK, dV: both loads in flight before the wait
+      tmem_ld_32x32b_x32(tmem + lane_addr + 384u + grp * 32, v[0]);
+      tmem_ld_32x32b_x32(tmem + lane_addr + 256u + grp * 32, v[1]);
+      tmem_ld_wait();
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {  // dK, then dV
         const float sc = kv == 0 ? p.scale : 1.f;
-        // both 32-column halves in flight before the first wait
-        uint32_t v[2][32];
-        tmem_ld_32x32b_x32(tmem + lane_addr + (kv == 0 ? 384u : 256u) + grp * 64, v[0]);
-        tmem_ld_32x32b_x32(tmem + lane_addr + (kv == 0 ? 384u : 256u) + grp * 64 + 32, v[1]);
-        tmem_ld_wait();
+        uint32_t w[16];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {  // 32 columns at a time
-          uint32_t w[16];
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(v[kv][2 * e]) * sc,
+                             __uint_as_float(v[kv][2 * e + 1]) * sc);
+        if (box_inside) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(v[c][2 * e]) * sc,
-                               __uint_as_float(v[c][2 * e + 1]) * sc);
-          if (box_inside) {
+          for (int u = 0; u < 4; ++u)
+            st_shared_v4(trow + kv * 2048u + (static_cast<uint32_t>(u) << 4), w[4 * u],
+                         w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        } else if (key < p.seq) {
+          uint4* dst = reinterpret_cast<uint4*>(base + kv * p.kvl * AB_D);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const uint32_t chunk = static_cast<uint32_t>(c * 4 + u);
-              st_shared_v4(trow + kv * 4096u + ((chunk ^ (static_cast<uint32_t>(lane) & 7u)) << 4),
-                           w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-            }
-          } else if (key < p.seq) {
-            uint4* dst = reinterpret_cast<uint4*>(base + kv * p.kvl * AB_D + c * 32);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-          }
+          for (int u = 0; u < 4; ++u)
+            dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
         }
       }
       if (box_inside) {
         fence_proxy_async_shared();
         __syncwarp();
         if (lane == 0) {
-          const int col = p.q_w + kvh * AB_D + grp * 64;
+          const int col = p.q_w + kvh * AB_D + grp * 32;
           const int trow0 = row_base + kv0 + rq * 32;
           tma_store_3d(&tm_st, tile, col, trow0, g);
-          tma_store_3d(&tm_st, tile + 4096u, col + p.kvl * AB_D, trow0, g);
+          tma_store_3d(&tm_st, tile + 2048u, col + p.kvl * AB_D, trow0, g);
           bulk_commit();
           bulk_wait_read<0>();  // the tiles are read before the CTA's shared memory goes away
         }
@@ -463,7 +459,7 @@ __global__ void __launch_bounds__(AB_THREADS, 1)
       if (lane == 0) atomicOr(p.err, ERR_WAIT_ATTN);
       *abort_flag = 1;
     }
-  } else if (warp >= 8 && warp < 12) {
+  } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------ dQ^T
     const int rq = warp & 3;
     const int dcol = rq * 32 + lane;  // head-dimension column (= TMEM lane)
@@ -588,15 +584,17 @@ static PFN_cuTensorMapEncodeTiled_v12000 bwd_map_encoder() {
 }
 
 static bool encode_rows(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base,
-                        int64_t cols, int64_t rows, int shards, uint32_t box_rows) {
+                        int64_t cols, int64_t rows, int shards, uint32_t box_rows,
+                        uint32_t box_cols = 64, bool swizzle = true) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(shards)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols * 2),
                            static_cast<cuuint64_t>(rows * cols * 2)};
-  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -616,7 +614,8 @@ int launch_attention_bwd(const void* QKV, const void* O, const void* dO, const f
   if (!encode_rows(enc, &tm_kv, QKV, ld, M, n_shards, AB_BK)) return 1;
   if (!encode_rows(enc, &tm_q, QKV, ld, M, n_shards, AB_BQ)) return 1;
   if (!encode_rows(enc, &tm_do, dO, q_w, M, n_shards, AB_BQ)) return 1;
-  if (!encode_rows(enc, &tm_st, dQKV, ld, M, n_shards, 32)) return 1;  // dK / dV stores
+  // dK / dV stores: 32 keys x 32 columns, dense 64-byte rows
+  if (!encode_rows(enc, &tm_st, dQKV, ld, M, n_shards, 32, 32, false)) return 1;
 
   const int64_t heads_total = static_cast<int64_t>(n_shards) * hps;
   const int nq = static_cast<int>((seq + AB_BQ - 1) / AB_BQ);
